@@ -1,0 +1,248 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) top-k routed Mixture-of-Experts FFN
+ * layer forward pass.
+ *
+ * What is computed (page title, section):
+ *   - the router picks a fixed set of k experts per token ("PCoMoE" summary,
+ *     "The Limitation of Monolithic Expert Selection"); gates are the softmax
+ *     of the selected logits (renormalised over the k);
+ *   - routing decisions are flattened into a task list, grouped by expert id
+ *     and sorted by token id inside each group, then run as a grouped GEMM
+ *     that loads each block of expert weights once for a batch of tokens
+ *     ("OmniMoE" technical summary, 2.2 Expert-Centric Scheduling);
+ *   - experts: SwiGLU FFN experts y = W_down (silu(W_gate x) * (W_up x));
+ *     always-on shared experts ("OmniMoE" 2.1, Shared Dense MLP); MoE++
+ *     zero (output 0), copy (output x) and constant (a1 x + a2 v) experts,
+ *     and gating residuals that add the previous layer's logits ("MoE++"
+ *     summary, "Approach"); OmniMoE atomic experts
+ *     E_i(x) = GELU(x . u_i) v_i found by a Cartesian-product router that
+ *     scores the row and column halves of a 2-D expert grid separately
+ *     ("OmniMoE" 2.1 Atomic Experts, 2.2 Cartesian Product Router).
+ *
+ * Conventions (all entry points):
+ *   - Ownership: the caller owns every buffer.  Pointers to tensors are
+ *     DEVICE pointers (cudaMalloc / PyTorch CUDA memory) unless stated; the
+ *     descriptor and weight structs are read on the host during the call.
+ *     The library allocates no device memory: scratch space is the
+ *     caller's `workspace` of at least the size the *_workspace_size calls
+ *     return (256-byte aligned).  The library keeps host-side caches of TMA
+ *     descriptors only.
+ *   - Layout: row-major, C order.  d_model: a multiple of 64 (bf16) or 8 (fp32).  Expert weights are K-contiguous:
+ *     w_gate, w_up [n_ffn, hidden, d_model]; w_down [n_ffn, d_model, hidden].
+ *     Every tensor base must be 16-byte aligned.
+ *   - Types: x, weights and y are `dtype` (fp32 or bf16); accumulation is
+ *     fp32; routing outputs are fp32 / int32.
+ *   - Asynchrony: every call only enqueues kernels on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream) and returns; nothing is
+ *     synchronised.
+ *   - Errors: argument errors are detected on the host and returned at
+ *     once (nothing enqueued).  Errors found by the kernels (an expert id
+ *     out of range, a wait that timed out) are recorded in a per-device
+ *     status word and returned by moe_get_device_status().  No kernel traps.
+ *   - Expert ids: 0..n_ffn-1 are FFN experts, then n_zero zero experts,
+ *     n_copy copy experts, n_const constant experts.  Atomic experts have ids
+ *     r * pk_cols + c for grid row r and column c.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad descriptor, null or misaligned pointer   */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (shape limits)     */
+    MOE_ERR_WORKSPACE = 3,     /* workspace smaller than required              */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed            */
+    MOE_ERR_DEVICE_BOUNDS = 5, /* a kernel saw an index out of range           */
+    MOE_ERR_TIMEOUT = 6        /* a kernel wait exceeded its time limit        */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_EXPERT_SWIGLU = 0, MOE_EXPERT_ATOMIC_GELU = 1 } moe_expert_kind;
+
+/* Sizes of one layer.  Unused fields must be 0. */
+typedef struct moe_layer_desc {
+    int32_t T;             /* tokens in the batch (>= 0)                          */
+    int32_t d_model;       /* width of x and y                                    */
+    int32_t top_k;         /* experts per token (atomic: K of the product router) */
+    int32_t dtype;         /* moe_dtype of x, weights and y                       */
+    int32_t kind;          /* moe_expert_kind                                     */
+    int32_t n_ffn;         /* routed SwiGLU experts                               */
+    int32_t hidden;        /* their hidden width H                                */
+    int32_t n_shared;      /* always-on SwiGLU experts (weight 1)                 */
+    int32_t hidden_shared; /* their hidden width (must equal hidden if n_shared)  */
+    int32_t n_zero;        /* MoE++ zero experts                                  */
+    int32_t n_copy;        /* MoE++ copy experts                                  */
+    int32_t n_const;       /* MoE++ constant experts                              */
+    int32_t pk_rows;       /* atomic: grid rows N_r (row sub-keys)                */
+    int32_t pk_cols;       /* atomic: grid columns N_c (column sub-keys)          */
+    int32_t pk_topk_half;  /* atomic: sub-keys kept per half                      */
+    int32_t d_query;       /* atomic: query width (two halves of d_query / 2)     */
+    int32_t out_f32;       /* 0: y is `dtype`; 1: y is fp32 (the fp32 combine     *
+                            * before its final rounding; the dtype output is its *
+                            * round-to-nearest-even)                              */
+} moe_layer_desc;
+
+/* Device pointers to the layer's parameters (NULL where the layer has none). */
+typedef struct moe_layer_weights {
+    const void* w_router;     /* [n_ffn + n_zero + n_copy + n_const, d_model]            */
+    const float* router_bias; /* [same rows] fp32, added to the logits; nullable         */
+    const void* w_const_mix;  /* [n_const, 2, d_model]: (a1, a2) = softmax(W_c x)        */
+    const void* const_vec;    /* [n_const, d_model]: the constant experts' vectors v     */
+    const void* w_gate;       /* [n_ffn, hidden, d_model]                                */
+    const void* w_up;         /* [n_ffn, hidden, d_model]                                */
+    const void* w_down;       /* [n_ffn, d_model, hidden]                                */
+    const void* ws_gate;      /* [n_shared, hidden_shared, d_model]                      */
+    const void* ws_up;        /* [n_shared, hidden_shared, d_model]                      */
+    const void* ws_down;      /* [n_shared, d_model, hidden_shared]                      */
+    const void* w_query;      /* atomic: [d_query, d_model]                              */
+    const void* subkeys_row;  /* atomic: [pk_rows, d_query / 2]                          */
+    const void* subkeys_col;  /* atomic: [pk_cols, d_query / 2]                          */
+    const void* u;            /* atomic: [pk_rows * pk_cols, d_model] input vectors      */
+    const void* v;            /* atomic: [pk_rows * pk_cols, d_model] output vectors     */
+} moe_layer_weights;
+
+/* Number of expert groups of the grouped step: n_ffn + n_shared (SwiGLU) or
+ * pk_rows * pk_cols (atomic).  expert_offsets has groups + 1 entries. */
+MOE_API int64_t moe_num_groups(const moe_layer_desc* desc);
+
+/* Row capacity of x_sorted / y_sorted / token_of: T*top_k + n_shared*T
+ * (SwiGLU) or T*top_k (atomic). */
+MOE_API int64_t moe_row_capacity(const moe_layer_desc* desc);
+
+/* Scratch bytes needed by moe_route, moe_permute and moe_grouped_ffn (the
+ * largest of the three); -1 for an invalid descriptor. */
+MOE_API int64_t moe_workspace_size(const moe_layer_desc* desc);
+
+/* Bytes needed by moe_layer_forward: all intermediates plus the scratch. */
+MOE_API int64_t moe_layer_workspace_size(const moe_layer_desc* desc);
+
+/*
+ * Router ("PCoMoE" summary, top-k selection; "MoE++" Approach, gating
+ * residuals; "OmniMoE" 2.2 Cartesian Product Router).
+ * SwiGLU kind: z[t] = W_router x_t + router_bias + prev_logits[t] (fp32);
+ *   topk_idx[t] = the k largest z in descending order, ties to the lower id;
+ *   topk_gate[t, j] = exp(z_sel[j] - z_sel[0]) / sum over the k selected;
+ *   const_mix[t, c] = softmax(W_c,c x_t) for each constant expert.
+ * Atomic kind: q = W_query x_t (fp32), s_row = subkeys_row q[:dq/2],
+ *   s_col = subkeys_col q[dq/2:]; the pk_topk_half best of each half; the
+ *   pk_topk_half^2 candidates (r, c) score s_row[r] + s_col[c] (compared
+ *   exactly, ties to the lower id r*pk_cols + c); the top_k best with softmax
+ *   gates.
+ * x [T, d_model]; prev_logits [T, rows of w_router] fp32 nullable;
+ * logits_out (nullable): SwiGLU [T, rows of w_router] fp32 z; atomic
+ *   [T, pk_rows + pk_cols] fp32 (s_row then s_col);
+ * topk_idx [T, top_k] int32; topk_gate [T, top_k] fp32;
+ * const_mix [T, n_const, 2] fp32 (required iff n_const > 0).
+ */
+MOE_API moe_status moe_route(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
+                     const float* prev_logits, float* logits_out, int32_t* topk_idx,
+                     float* topk_gate, float* const_mix, void* workspace, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
+ * Expert-centric grouping ("OmniMoE" 2.2: task collection, grouping by
+ * expert id, sorting by token id within each group): a per-expert
+ * histogram, an exclusive prefix sum and a stable permutation.
+ * expert_offsets [groups + 1]: group g holds rows [off[g], off[g+1]).
+ *   SwiGLU: groups 0..n_ffn-1 are the FFN experts' tasks in (expert, token)
+ *   order; group n_ffn + s holds all T tokens in order for shared expert s.
+ *   Zero-computation slots are not grouped.
+ * row_of [T*top_k]: row of slot (t, j), -1 for a zero-computation expert.
+ * token_of [row capacity]: SwiGLU: token of each row; atomic: flat slot id
+ *   t*top_k + j of each task.
+ * x_sorted [row capacity, d_model]: SwiGLU only, x_sorted[r] = x[token_of[r]];
+ *   NULL for the atomic kind.  Rows past expert_offsets[groups] are untouched.
+ * An id outside [0, n_ffn + n_zero + n_copy + n_const) (or the atomic grid)
+ * sets MOE_ERR_DEVICE_BOUNDS in the device status and is skipped.
+ */
+MOE_API moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* token_of,
+                       void* x_sorted, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Grouped expert step ("OmniMoE" 2.2 Grouped GEMM; 2.1 Atomic Experts).
+ * SwiGLU: y_sorted[r] = W_down[e] (silu(W_gate[e] x_sorted[r]) * (W_up[e]
+ *   x_sorted[r])) for r in group e (shared groups use the ws_* weights),
+ *   on tcgen05 tensor cores (bf16) or fp32 SIMT cores (fp32); the hidden
+ *   activation is rounded to dtype in the workspace, the expert outputs are
+ *   kept in fp32.  y_sorted [row capacity, d_model] fp32.  token_of, x,
+ *   topk_gate unused.
+ * Atomic: c[s] = topk_gate[s] * GELU(u_e . x_t) for each task s = t*K + j of
+ *   expert e, computed expert by expert (each u_e read once); y_sorted is
+ *   float c[T*K] in slot order.  x_sorted unused.
+ */
+MOE_API moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_layer_weights* w,
+                           const void* x_sorted, const int32_t* expert_offsets,
+                           const int32_t* token_of, const void* x, const float* topk_gate,
+                           void* y_sorted, void* workspace, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/*
+ * The two grouped GEMMs of the SwiGLU step, one per call (same arguments as
+ * moe_grouped_ffn): phase 1 writes the hidden activation h into the
+ * workspace, phase 2 reads it and writes y_sorted.  Calling phase 1 then
+ * phase 2 on the same workspace equals moe_grouped_ffn.  SwiGLU kind only.
+ */
+MOE_API moe_status moe_grouped_ffn_phase(const moe_layer_desc* desc, const moe_layer_weights* w,
+                                 int phase, const void* x_sorted,
+                                 const int32_t* expert_offsets, void* y_sorted,
+                                 void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Gate-weighted combine back to token order ("OmniMoE" 2.1 Dynamic Expert
+ * Assembly; "MoE++" Approach).
+ * SwiGLU: y_t = sum_s y_sorted[off[n_ffn + s] + t]
+ *             + sum_j topk_gate[t, j] * O_j, with O_j = y_sorted[row_of[t, j]]
+ *   (y_sorted fp32 as written by moe_grouped_ffn)
+ *   for an FFN expert, 0 for a zero expert, x_t for a copy expert and
+ *   a1 x_t + a2 v_c for constant expert c (const_mix, w->const_vec);
+ *   accumulated in fp32 in slot order, rounded once to dtype.
+ * Atomic: y_t = sum_j c[t*K + j] * v_{topk_idx[t, j]} (y_sorted = c).
+ * y [T, d_model] in dtype, or fp32 if desc->out_f32.
+ */
+MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weights* w,
+                       const void* y_sorted, const int32_t* expert_offsets,
+                       const int32_t* row_of, const int32_t* topk_idx, const float* topk_gate,
+                       const float* const_mix, const void* x, void* y, moe_stream_t stream);
+
+/*
+ * The whole layer: moe_route, moe_permute, moe_grouped_ffn and moe_combine
+ * on `stream`, intermediates in `workspace` (moe_layer_workspace_size bytes).
+ * x [T, d_model]; y [T, d_model] (dtype, or fp32 if desc->out_f32);
+ * prev_logits nullable; logits_out nullable (as in moe_route).
+ */
+MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* w,
+                             const void* x, const float* prev_logits, void* y,
+                             float* logits_out, void* workspace, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* Synchronises `stream`, returns the current device's status word in *out
+ * (MOE_OK if no kernel reported an error) and clears it if reset != 0. */
+MOE_API moe_status moe_get_device_status(moe_status* out, int reset, moe_stream_t stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Number of kernels the last call on this host thread enqueued. */
+MOE_API int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

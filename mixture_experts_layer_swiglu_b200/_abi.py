@@ -1,0 +1,198 @@
+"""ctypes binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch
+CUDA tensors (or None for a NULL pointer).  Nothing here computes any part of
+the layer; if the library cannot be loaded the import fails.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libmoe.so"
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
+MOE_ERR_CUDA, MOE_ERR_DEVICE_BOUNDS, MOE_ERR_TIMEOUT = 4, 5, 6
+MOE_F32, MOE_BF16 = 0, 1
+MOE_EXPERT_SWIGLU, MOE_EXPERT_ATOMIC_GELU = 0, 1
+
+EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_layer_workspace_size",
+            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
+            "moe_layer_forward", "moe_get_device_status", "moe_status_string",
+            "moe_last_launch_count")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+class MoELayerDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "T", "d_model", "top_k", "dtype", "kind", "n_ffn", "hidden", "n_shared", "hidden_shared",
+        "n_zero", "n_copy", "n_const", "pk_rows", "pk_cols", "pk_topk_half", "d_query", "out_f32")]
+
+
+class MoELayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_router", "router_bias", "w_const_mix", "const_vec", "w_gate", "w_up", "w_down",
+        "ws_gate", "ws_up", "ws_down", "w_query", "subkeys_row", "subkeys_col", "u", "v")]
+
+
+_lib = None
+
+
+def load(path: Path | str | None = None):
+    """Load libmoe.so (building it in-tree with nvcc first if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = Path(path) if path else LIB_PATH
+    if not p.exists():
+        from . import build as _build
+        _build.build()
+    L = ctypes.CDLL(str(p))
+    P, VP, I32, I64, SZ = ctypes.POINTER, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    D, W = P(MoELayerDesc), P(MoELayerWeights)
+    for name in ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_layer_workspace_size"):
+        getattr(L, name).argtypes = [D]
+        getattr(L, name).restype = I64
+    L.moe_route.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_permute.argtypes = [D, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_grouped_ffn.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_grouped_ffn_phase.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, SZ, VP]
+    L.moe_combine.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, VP, VP]
+    L.moe_layer_forward.argtypes = [D, W, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_get_device_status.argtypes = [P(ctypes.c_int), ctypes.c_int, VP]
+    L.moe_status_string.argtypes = [ctypes.c_int]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_last_launch_count.restype = I32
+    for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
+                 "moe_layer_forward", "moe_get_device_status"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(int(status)).decode()
+
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libmoe takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoEError(fn, status)
+
+
+def weights_struct(w: dict) -> MoELayerWeights:
+    """MoELayerWeights from a dict of device tensors (missing keys -> NULL)."""
+    s = MoELayerWeights()
+    for name, _ in MoELayerWeights._fields_:
+        setattr(s, name, _p(w.get(name)))
+    return s
+
+
+# ------------------------------------------------------------ entry points
+
+def moe_num_groups(desc: MoELayerDesc) -> int:
+    return int(load().moe_num_groups(ctypes.byref(desc)))
+
+
+def moe_row_capacity(desc: MoELayerDesc) -> int:
+    return int(load().moe_row_capacity(ctypes.byref(desc)))
+
+
+def moe_workspace_size(desc: MoELayerDesc) -> int:
+    return int(load().moe_workspace_size(ctypes.byref(desc)))
+
+
+def moe_layer_workspace_size(desc: MoELayerDesc) -> int:
+    return int(load().moe_layer_workspace_size(ctypes.byref(desc)))
+
+
+def moe_route(desc, weights, x, prev_logits, logits_out, topk_idx, topk_gate, const_mix, workspace,
+              stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_route", load().moe_route(ctypes.byref(desc), ctypes.byref(ws), _p(x), _p(prev_logits),
+                                         _p(logits_out), _p(topk_idx), _p(topk_gate), _p(const_mix),
+                                         _p(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def moe_permute(desc, topk_idx, x, expert_offsets, row_of, token_of, x_sorted, workspace,
+                stream=None) -> None:
+    _check("moe_permute", load().moe_permute(ctypes.byref(desc), _p(topk_idx), _p(x), _p(expert_offsets),
+                                             _p(row_of), _p(token_of), _p(x_sorted), _p(workspace),
+                                             _nbytes(workspace), _stream(stream)))
+
+
+def moe_grouped_ffn(desc, weights, x_sorted, expert_offsets, token_of, x, topk_gate, y_sorted, workspace,
+                    stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_grouped_ffn", load().moe_grouped_ffn(ctypes.byref(desc), ctypes.byref(ws), _p(x_sorted),
+                                                     _p(expert_offsets), _p(token_of), _p(x), _p(topk_gate),
+                                                     _p(y_sorted), _p(workspace), _nbytes(workspace),
+                                                     _stream(stream)))
+
+
+def moe_grouped_ffn_phase(desc, weights, phase, x_sorted, expert_offsets, y_sorted, workspace,
+                          stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_grouped_ffn_phase",
+           load().moe_grouped_ffn_phase(ctypes.byref(desc), ctypes.byref(ws), int(phase), _p(x_sorted),
+                                        _p(expert_offsets), _p(y_sorted), _p(workspace), _nbytes(workspace),
+                                        _stream(stream)))
+
+
+def moe_combine(desc, weights, y_sorted, expert_offsets, row_of, topk_idx, topk_gate, const_mix, x, y,
+                stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_combine", load().moe_combine(ctypes.byref(desc), ctypes.byref(ws), _p(y_sorted),
+                                             _p(expert_offsets), _p(row_of), _p(topk_idx), _p(topk_gate),
+                                             _p(const_mix), _p(x), _p(y), _stream(stream)))
+
+
+def moe_layer_forward(desc, weights, x, prev_logits, y, logits_out, workspace, stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_layer_forward", load().moe_layer_forward(ctypes.byref(desc), ctypes.byref(ws), _p(x),
+                                                         _p(prev_logits), _p(y), _p(logits_out),
+                                                         _p(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def moe_get_device_status(reset: bool = True, stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check("moe_get_device_status", load().moe_get_device_status(ctypes.byref(out), int(bool(reset)),
+                                                                 _stream(stream)))
+    return int(out.value)
+
+
+def moe_last_launch_count() -> int:
+    return int(load().moe_last_launch_count())

@@ -1,0 +1,320 @@
+// combine.cu -- gate-weighted combine back to token order, MoE++
+// zero-computation experts, and the two passes of the atomic-expert layer.
+//
+// Combine ("OmniMoE" technical summary, 2.1: the routed outputs are
+// assembled per token, the shared dense branch is always added; "MoE++"
+// summary, "Approach": zero expert = discard, copy expert = identity,
+// constant expert = trainable vector mixed with the input):
+//   y_t = sum_s y_sorted[shared row of t] + sum_j g_tj O_tj
+// accumulated in fp32 in slot order and rounded once.  One warp per token,
+// 16-byte vector loads of the rows (HBM-bound: reads the k expert rows and,
+// for copy/constant experts, x; writes y).
+//
+// Atomic experts ("OmniMoE" 2.1 Atomic Experts E_i(x) = sigma(x . u_i) v_i,
+// Dynamic Expert Assembly; 2.2 Expert-Centric Scheduling):
+//   phase A, expert by expert: each touched u_e is read once from HBM and
+//     dotted with the x rows of its tasks (x stays in L2):
+//     c[s] = g[s] * GELU(u_e . x_t);
+//   phase B, token by token: y_t = sum_j c[t, j] v_{e_tj}, fp32 in slot order.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+template <typename T> struct Chunk;
+template <> struct Chunk<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ static void load(const void* p, long long i, float (&v)[8])
+    {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+        v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+    }
+    __device__ static void store(void* p, long long i, const float (&v)[8])
+    {
+        reinterpret_cast<uint4*>(p)[i] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                    pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    }
+};
+template <> struct Chunk<float> {
+    static constexpr int N = 4;
+    __device__ static void load(const void* p, long long i, float (&v)[4])
+    {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(p) + i);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    }
+    __device__ static void store(void* p, long long i, const float (&v)[4])
+    {
+        reinterpret_cast<float4*>(p)[i] = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+
+constexpr int CMB_MAXK = 32;
+
+// y_sorted rows are fp32 (expert outputs are not rounded before the combine);
+// x, the constant vectors and y are T.  Chunks of 8 elements for both types.
+template <typename T>
+__device__ __forceinline__ void load8(const void* p, long long i8, float (&v)[8])
+{
+    if constexpr (sizeof(T) == 2) {
+        Chunk<__nv_bfloat16>::load(p, i8, v);
+    } else {
+        float a[4], b[4];
+        Chunk<float>::load(p, 2 * i8, a);
+        Chunk<float>::load(p, 2 * i8 + 1, b);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { v[i] = a[i]; v[4 + i] = b[i]; }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store8(void* p, long long i8, const float (&v)[8])
+{
+    if constexpr (sizeof(T) == 2) {
+        Chunk<__nv_bfloat16>::store(p, i8, v);
+    } else {
+        const float a[4] = {v[0], v[1], v[2], v[3]}, b[4] = {v[4], v[5], v[6], v[7]};
+        Chunk<float>::store(p, 2 * i8, a);
+        Chunk<float>::store(p, 2 * i8 + 1, b);
+    }
+}
+
+template <typename T, typename TO>
+__global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a)
+{
+    constexpr int V = 8;
+    const int lane = threadIdx.x & 31;
+    const int vecs = a.d / V;
+    const int zero0 = a.n_ffn, copy0 = zero0 + a.n_zero, const0 = copy0 + a.n_copy;
+    const int n_ids = const0 + a.n_const;
+    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+    __shared__ int s_e[8][CMB_MAXK], s_r[8][CMB_MAXK];
+    __shared__ float s_g[8][CMB_MAXK], s_a1[8][CMB_MAXK], s_a2[8][CMB_MAXK];
+    const int wib = threadIdx.x >> 5;
+    for (long long t = blockIdx.x * (long long)(blockDim.x >> 5) + wib; t < a.T; t += nw) {
+        // slot j's id, gate, row and constant mix, staged by lane j
+        if (lane < a.k) {
+            int e = a.idx[t * a.k + lane];
+            const int r = a.row_of[t * a.k + lane];
+            bool bad = e < 0 || e >= n_ids;
+            if (!bad && e < zero0 && (r < 0 || r >= a.rows_cap)) bad = true;
+            if (bad) { set_status(MOE_ERR_DEVICE_BOUNDS); e = -1; }
+            float a1 = 0.f, a2 = 0.f;
+            if (e >= const0) {
+                const int c = e - const0;
+                a1 = a.const_mix[(t * a.n_const + c) * 2 + 0];
+                a2 = a.const_mix[(t * a.n_const + c) * 2 + 1];
+            }
+            s_e[wib][lane] = e;
+            s_r[wib][lane] = r;
+            s_g[wib][lane] = a.gate[t * a.k + lane];
+            s_a1[wib][lane] = a1;
+            s_a2[wib][lane] = a2;
+        }
+        __syncwarp();
+        for (int i = lane; i < vecs; i += 32) {
+            float acc[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = 0.f;
+            for (int s = 0; s < a.n_shared; ++s) {
+                const long long r = (long long)a.offsets[a.n_ffn + s] + t;
+                if (r < a.rows_cap) {
+                    float w[V];
+                    load8<float>(a.ys, r * vecs + i, w);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[v] += w[v];
+                }
+            }
+            bool have_x = false;
+            float xv[V];
+            for (int j = 0; j < a.k; ++j) {
+                const int e = s_e[wib][j];
+                const float g = s_g[wib][j];
+                if (e < 0) continue;
+                if (e < zero0) {
+                    float w[V];
+                    load8<float>(a.ys, (long long)s_r[wib][j] * vecs + i, w);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[v] = fmaf(g, w[v], acc[v]);
+                } else if (e < copy0) {
+                    // zero expert: contributes nothing
+                } else {
+                    if (!have_x) { load8<T>(a.x, t * vecs + i, xv); have_x = true; }
+                    if (e < const0) {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[v] = fmaf(g, xv[v], acc[v]);
+                    } else {
+                        const float a1 = s_a1[wib][j], a2 = s_a2[wib][j];
+                        float cv[V];
+                        load8<T>(a.const_vec, (long long)(e - const0) * vecs + i, cv);
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[v] = fmaf(g, a1 * xv[v] + a2 * cv[v], acc[v]);
+                    }
+                }
+            }
+            store8<TO>(a.y, t * vecs + i, acc);
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------- atomic
+
+// phase A: one warp per expert; u_e kept in registers (NV uint4 per lane).
+template <int NV>
+__global__ void __launch_bounds__(256) atomic_phase_a_kernel(const AtomicArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const uint4* x = reinterpret_cast<const uint4*>(a.x);
+    const uint4* u = reinterpret_cast<const uint4*>(a.u);
+    const int vecs = a.d / 8;
+    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long e = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); e < a.N; e += nw) {
+        const int lo = a.offsets[e], hi = a.offsets[e + 1];
+        if (lo >= hi) continue;
+        float ue[NV][8];
+#pragma unroll
+        for (int q = 0; q < NV; ++q) {
+            const uint4 w = __ldg(u + e * vecs + q * 32 + lane);
+            ue[q][0] = bf16_lo(w.x); ue[q][1] = bf16_hi(w.x); ue[q][2] = bf16_lo(w.y); ue[q][3] = bf16_hi(w.y);
+            ue[q][4] = bf16_lo(w.z); ue[q][5] = bf16_hi(w.z); ue[q][6] = bf16_lo(w.w); ue[q][7] = bf16_hi(w.w);
+        }
+        for (int p = lo; p < hi; ++p) {
+            const int s = a.token_of[p];
+            const int t = s / a.K;
+            float dot = 0.f;
+#pragma unroll
+            for (int q = 0; q < NV; ++q) {
+                const uint4 w = __ldg(x + (long long)t * vecs + q * 32 + lane);
+                dot = fmaf(ue[q][0], bf16_lo(w.x), dot); dot = fmaf(ue[q][1], bf16_hi(w.x), dot);
+                dot = fmaf(ue[q][2], bf16_lo(w.y), dot); dot = fmaf(ue[q][3], bf16_hi(w.y), dot);
+                dot = fmaf(ue[q][4], bf16_lo(w.z), dot); dot = fmaf(ue[q][5], bf16_hi(w.z), dot);
+                dot = fmaf(ue[q][6], bf16_lo(w.w), dot); dot = fmaf(ue[q][7], bf16_hi(w.w), dot);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(FULL, dot, o);
+            if (lane == 0) {
+                const float gel = 0.5f * dot * (1.0f + erff(dot * 0.70710678118654752f));
+                a.c[s] = a.gate[s] * gel;
+            }
+        }
+    }
+}
+
+// phase B: one warp per token; 4 v rows in flight per lane.
+template <int NV>
+__global__ void __launch_bounds__(256) atomic_phase_b_kernel(const AtomicArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const uint4* v = reinterpret_cast<const uint4*>(a.v);
+    const int vecs = a.d / 8;
+    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long t = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += nw) {
+        float acc[NV][8];
+#pragma unroll
+        for (int q = 0; q < NV; ++q)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[q][i] = 0.f;
+        for (int j0 = 0; j0 < a.K; j0 += 32) {
+            const int my_e = (j0 + lane < a.K) ? a.idx[t * a.K + j0 + lane] : -1;
+            const float my_c = (j0 + lane < a.K) ? a.c[t * a.K + j0 + lane] : 0.f;
+            const int jn = min(32, a.K - j0);
+            for (int jj = 0; jj < jn; ++jj) {
+                const int e = __shfl_sync(FULL, my_e, jj);
+                const float c = __shfl_sync(FULL, my_c, jj);
+                if (e < 0 || e >= a.N) { if (lane == 0) set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
+                uint4 w[NV];
+#pragma unroll
+                for (int q = 0; q < NV; ++q) w[q] = __ldg(v + (long long)e * vecs + q * 32 + lane);
+#pragma unroll
+                for (int q = 0; q < NV; ++q) {
+                    acc[q][0] = fmaf(c, bf16_lo(w[q].x), acc[q][0]); acc[q][1] = fmaf(c, bf16_hi(w[q].x), acc[q][1]);
+                    acc[q][2] = fmaf(c, bf16_lo(w[q].y), acc[q][2]); acc[q][3] = fmaf(c, bf16_hi(w[q].y), acc[q][3]);
+                    acc[q][4] = fmaf(c, bf16_lo(w[q].z), acc[q][4]); acc[q][5] = fmaf(c, bf16_hi(w[q].z), acc[q][5]);
+                    acc[q][6] = fmaf(c, bf16_lo(w[q].w), acc[q][6]); acc[q][7] = fmaf(c, bf16_hi(w[q].w), acc[q][7]);
+                }
+            }
+        }
+        if (a.out_f32) {
+            float4* y = reinterpret_cast<float4*>(a.y);
+#pragma unroll
+            for (int q = 0; q < NV; ++q) {
+                const long long o = (t * vecs + q * 32 + lane) * 2;
+                y[o] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+                y[o + 1] = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
+            }
+        } else {
+            uint4* y = reinterpret_cast<uint4*>(a.y);
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+                y[t * vecs + q * 32 + lane] = make_uint4(pack_bf16(acc[q][0], acc[q][1]), pack_bf16(acc[q][2], acc[q][3]),
+                                                         pack_bf16(acc[q][4], acc[q][5]), pack_bf16(acc[q][6], acc[q][7]));
+        }
+    }
+}
+
+template <template <int> class K, typename... Args>
+moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
+{
+    switch (nv) {
+        case 1: K<1>::launch(grid, st, a); break;
+        case 2: K<2>::launch(grid, st, a); break;
+        case 4: K<4>::launch(grid, st, a); break;
+        case 8: K<8>::launch(grid, st, a); break;
+        default: return MOE_ERR_UNSUPPORTED;
+    }
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+template <int NV> struct PhaseA {
+    static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
+    {
+        atomic_phase_a_kernel<NV><<<grid, 256, 0, st>>>(a);
+    }
+};
+template <int NV> struct PhaseB {
+    static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
+    {
+        atomic_phase_b_kernel<NV><<<grid, 256, 0, st>>>(a);
+    }
+};
+
+}  // namespace
+
+moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st)
+{
+    if (a.T == 0) return MOE_OK;
+    if (a.k > CMB_MAXK) return MOE_ERR_UNSUPPORTED;
+    const int grid = std::max(1, std::min(cdiv(a.T, 8), num_sms() * 16));
+    if (dtype == MOE_BF16 && !a.out_f32) combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
+    else if (dtype == MOE_BF16) combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(a);
+    else combine_kernel<float, float><<<grid, 256, 0, st>>>(a);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st)
+{
+    const int grid = std::max(1, std::min(cdiv(a.N, 8), num_sms() * 16));
+    return launch_nv<PhaseA>(a.d / 256, grid, st, a);
+}
+
+moe_status launch_atomic_phase_b(const AtomicArgs& a, cudaStream_t st)
+{
+    if (a.T == 0) return MOE_OK;
+    const int grid = std::max(1, std::min(cdiv(a.T, 8), num_sms() * 16));
+    return launch_nv<PhaseB>(a.d / 256, grid, st, a);
+}
+
+}  // namespace moe

@@ -1,0 +1,451 @@
+// gemm_tc.cu -- persistent grouped GEMM on 5th-generation tensor cores.
+//
+// The expert-centric step of the layer ("OmniMoE" technical summary, 2.2
+// Expert-Centric Scheduling, Grouped GEMM): rows that chose the same expert
+// are contiguous, so one block of that expert's weights, once in shared
+// memory, serves up to 128 rows.  Groups have data-dependent sizes; the
+// tile schedule is built on the device from the group offsets, so nothing
+// is copied back to the host.
+//
+// Structure (one CTA per SM, 6 warps):
+//   warp 0   TMA producer: A tile [128 x 64] + B tile [256 x 64] per stage,
+//            128-byte swizzle, 4-stage mbarrier ring (no multicast).
+//   warp 1   TMEM allocator and MMA issuer: tcgen05.mma kind::f16,
+//            M=128 N=256 K=16, fp32 accumulators in TMEM, two accumulator
+//            buffers (512 columns) so the epilogue of one tile overlaps the
+//            MMAs of the next.
+//   warps 2-5 epilogue: tcgen05.ld of their 32-lane quarter, fused
+//            activation (SwiGLU: silu(gate) * up), bf16/fp32 store.
+// Every mbarrier wait is bounded (2 s); a timeout sets MOE_ERR_TIMEOUT, all
+// roles leave their loops, in-flight TMA copies are drained and TMEM freed.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN_MMA = 256;
+constexpr int STAGES = 4;
+constexpr int TILE_A = BM * BK * 2;        // 16 KB
+constexpr int TILE_B = BN_MMA * BK * 2;    // 32 KB
+constexpr int STAGE_BYTES = TILE_A + TILE_B;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int NTHREADS = 192;
+constexpr int SMEM_TABLE_INTS = 3 * kMaxGemmGroups + 1;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + SMEM_TABLE_INTS * 4;
+
+struct DevArgs {
+    const int32_t* offsets;
+    int n_groups, n_first, group_rows, N, K;
+    void* out;
+    long long ldo;
+    long long rows_cap;
+    int pk_T, pk_dq;
+};
+
+struct TileInfo {
+    int g;        // group
+    int row0;     // first A row of the tile
+    int rows;     // valid rows in the tile (<= BM)
+    int n;        // n-tile index inside the group
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int tile, const int* tile_start, const int* g_lo,
+                                                const int* g_cnt, int n_groups)
+{
+    int lo = 0, hi = n_groups - 1;   // last g with tile_start[g] <= tile
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    TileInfo ti;
+    ti.g = lo;
+    const int cnt = g_cnt[lo];
+    const int mt = cdiv(cnt, BM);
+    const int local = tile - tile_start[lo];
+    const int m = local % mt;       // m-tiles of a group are adjacent: they share B
+    ti.n = local / mt;
+    ti.row0 = g_lo[lo] + m * BM;
+    ti.rows = min(BM, cnt - m * BM);
+    return ti;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const DevArgs& a, uint32_t tacc, const TileInfo& ti,
+                                              int r)
+{
+    const long long grow = (long long)ti.row0 + r;
+    const bool valid = (r < ti.rows) && (grow < a.rows_cap);
+    if constexpr (EPI == EPI_SWIGLU) {
+        // accumulator columns [0,128) = gate, [128,256) = up for h columns n*128 ...
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+        const int col0 = ti.n * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(tacc + c * 32, g);
+            tmem_ld32(tacc + 128 + c * 32, u);
+            tc_wait_ld();
+            if (valid) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                    float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                    float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                    float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                    pk[i] = pack_bf16(h0, h1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(out + grow * a.ldo + col0 + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+    } else if constexpr (EPI == EPI_BF16) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+        const int col0 = ti.n * 256;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tacc + c * 32, v);
+            tc_wait_ld();
+            if (valid && col0 + c * 32 < a.N) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                uint4* dst = reinterpret_cast<uint4*>(out + grow * a.ldo + col0 + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+    } else if constexpr (EPI == EPI_F32) {
+        float* out = reinterpret_cast<float*>(a.out);
+        const int col0 = ti.n * 256;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tacc + c * 32, v);
+            tc_wait_ld();
+            if (valid && col0 + c * 32 < a.N) {
+                uint4* dst = reinterpret_cast<uint4*>(out + grow * a.ldo + col0 + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    } else {   // EPI_PK_SPLIT: q = x W_q^T split into three bf16 parts per half
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+        const int col0 = ti.n * 256;
+        const int half = a.pk_dq / 2;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tacc + c * 32, v);
+            tc_wait_ld();
+            const int col = col0 + c * 32;
+            if (valid && col < a.N) {
+                const int hf = col / half, cc = col % half;
+                __nv_bfloat16* dst = out + ((long long)hf * a.pk_T + grow) * a.ldo + cc;
+                uint32_t p0[16], p1[16], p2[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float q0 = __uint_as_float(v[2 * i]), q1 = __uint_as_float(v[2 * i + 1]);
+                    __nv_bfloat16 a0 = __float2bfloat16_rn(q0), a1 = __float2bfloat16_rn(q1);
+                    float r0 = q0 - __bfloat162float(a0), r1 = q1 - __bfloat162float(a1);
+                    __nv_bfloat16 b0 = __float2bfloat16_rn(r0), b1 = __float2bfloat16_rn(r1);
+                    float s0 = r0 - __bfloat162float(b0), s1 = r1 - __bfloat162float(b1);
+                    p0[i] = pack_bf16(__bfloat162float(a0), __bfloat162float(a1));
+                    p1[i] = pack_bf16(__bfloat162float(b0), __bfloat162float(b1));
+                    p2[i] = pack_bf16(s0, s1);
+                }
+                uint4* d0 = reinterpret_cast<uint4*>(dst);
+                uint4* d1 = reinterpret_cast<uint4*>(dst + half);
+                uint4* d2 = reinterpret_cast<uint4*>(dst + 2 * half);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    d0[i] = make_uint4(p0[4 * i], p0[4 * i + 1], p0[4 * i + 2], p0[4 * i + 3]);
+                    d1[i] = make_uint4(p1[4 * i], p1[4 * i + 1], p1[4 * i + 2], p1[4 * i + 3]);
+                    d2[i] = make_uint4(p2[4 * i], p2[4 * i + 1], p2[4 * i + 2], p2[4 * i + 3]);
+                }
+            }
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NTHREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                    const __grid_constant__ CUtensorMap tmB3, const DevArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * TILE_A;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * TILE_B);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* tile_start = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 256);
+    int* g_lo = tile_start + (kMaxGemmGroups + 1);
+    int* g_cnt = g_lo + kMaxGemmGroups;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ntn = (EPI == EPI_SWIGLU) ? cdiv(a.N, 128) : cdiv(a.N, 256);
+
+    // ---- group table: first row, row count and first tile of every group
+    if (warp == 0) {
+        const int n = a.n_groups;
+        const int chunk = cdiv(n, 32);
+        const int g0 = min(n, lane * chunk), g1 = min(n, g0 + chunk);
+        int local = 0;
+        for (int g = g0; g < g1; ++g) {
+            int lo, hi;
+            if (a.offsets) { lo = a.offsets[g]; hi = a.offsets[g + 1]; }
+            else { lo = g * a.group_rows; hi = lo + a.group_rows; }
+            int cnt = hi - lo;
+            if (cnt < 0 || lo < 0) { set_status(MOE_ERR_DEVICE_BOUNDS); cnt = 0; lo = 0; }
+            g_lo[g] = lo;
+            g_cnt[g] = cnt;
+            local += cdiv(cnt, BM) * ntn;
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int g = g0; g < g1; ++g) {
+            tile_start[g] = run;
+            run += cdiv(g_cnt[g], BM) * ntn;
+        }
+        if (lane == 31) tile_start[n] = incl;
+    }
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 128); }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+    if (threadIdx.x == 64) {
+        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB0); tma_prefetch_desc(&tmB1);
+        tma_prefetch_desc(&tmB2); tma_prefetch_desc(&tmB3);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[a.n_groups];
+    const int nk = cdiv(a.K, BK);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t armed = 0, arm_par = 0;   // per stage: copies in flight, their parity
+            bool bad = false;
+            for (int tile = blockIdx.x; tile < total && !bad; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(tile, tile_start, g_lo, g_cnt, a.n_groups);
+                const bool first = ti.g < a.n_first;
+                const int gb = first ? ti.g : ti.g - a.n_first;
+                const CUtensorMap* mlo = first ? &tmB0 : &tmB2;
+                const CUtensorMap* mhi;
+                int brow_lo, brow_hi;
+                if (EPI == EPI_SWIGLU) {
+                    mhi = first ? &tmB1 : &tmB3;
+                    brow_lo = gb * a.N + ti.n * 128;
+                    brow_hi = brow_lo;
+                } else {
+                    mhi = mlo;
+                    brow_lo = gb * a.N + ti.n * 256;
+                    brow_hi = brow_lo + 128;
+                }
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
+                    armed &= ~(1u << s);
+                    mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                    tma_load_2d(sA + s * TILE_A, &tmA, &full[s], kb * BK, ti.row0);
+                    tma_load_2d(sB + s * TILE_B, mlo, &full[s], kb * BK, brow_lo);
+                    tma_load_2d(sB + s * TILE_B + TILE_B / 2, mhi, &full[s], kb * BK, brow_hi);
+                    armed |= 1u << s;
+                    arm_par = (arm_par & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                }
+            }
+            if (bad) {   // let copies already in flight land before the CTA exits
+                for (int i = 0; i < STAGES; ++i)
+                    if (armed & (1u << i)) mbar_wait(&full[i], (arm_par >> i) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            const uint32_t idesc = idesc_bf16_f32(BM, BN_MMA);
+            int s = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            bool bad = false;
+            for (int tile = blockIdx.x; tile < total && !bad; tile += gridDim.x) {
+                if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (*abort_flag || !mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * TILE_A));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * TILE_B));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    tc_commit(&empty[s]);
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                }
+                if (bad) break;
+                tc_commit(&acc_full[acc]);
+                if (++acc == 2) { acc = 0; aph ^= 1; }
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;            // row of the tile
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(tile, tile_start, g_lo, g_cnt, a.n_groups);
+            if (*abort_flag || !mbar_wait(&acc_full[acc], aph)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+            epilogue_tile<EPI>(a, tacc, ti, r);
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            if (++acc == 2) { acc = 0; aph ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 [rows, K] row-major, box {64 (K), 128 rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K)
+{
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    if (rows <= 0 || base == nullptr) {   // unused operand: point at something valid
+        rows = 128;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int EPI>
+moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
+{
+    CUtensorMap mA, m0, m1, m2, m3;
+    const void* b1 = p.B1 ? p.B1 : p.B0;
+    const void* b2 = p.B2 ? p.B2 : p.B0;
+    const void* b3 = p.B3 ? p.B3 : (p.B2 ? p.B2 : b1);
+    const long long r23 = p.B2 ? p.b23_rows : p.b01_rows;
+    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, p.K) ||
+        !make_map(&m1, b1, p.b01_rows, p.K) || !make_map(&m2, b2, r23, p.K) ||
+        !make_map(&m3, b3, r23, p.K))
+        return MOE_ERR_CUDA;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        attr_done = true;
+    }
+    DevArgs a;
+    a.offsets = p.offsets;
+    a.n_groups = p.n_groups;
+    a.n_first = p.n_first;
+    a.group_rows = p.group_rows;
+    a.N = p.N;
+    a.K = p.K;
+    a.out = p.out;
+    a.ldo = p.ldo;
+    a.rows_cap = p.rows_cap;
+    a.pk_T = p.pk_T;
+    a.pk_dq = p.pk_dq;
+    const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
+    const long long tiles_ub = (long long)(cdiv((int)std::min<long long>(p.rows_cap, 1ll << 30), BM) + p.n_groups) * ntn;
+    const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms()));
+    grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st)
+{
+    if (p.n_groups <= 0 || p.n_groups > kMaxGemmGroups || p.K <= 0 || p.K % 8 != 0 || p.N <= 0 ||
+        p.N % 32 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (p.epi == EPI_SWIGLU && p.N % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    switch (p.epi) {
+        case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(p, st);
+        case EPI_BF16: return launch_epi<EPI_BF16>(p, st);
+        case EPI_F32: return launch_epi<EPI_F32>(p, st);
+        case EPI_PK_SPLIT: return launch_epi<EPI_PK_SPLIT>(p, st);
+        default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,145 @@
+// internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Kernel launches enqueued by the current C-ABI call (per host thread).
+extern thread_local int t_launches;
+inline void count_launch(int n = 1) { t_launches += n; }
+
+moe_status cuda_status(cudaError_t e);
+int num_sms();
+
+// ------------------------------------------------------------ grouped GEMM
+enum EpiKind { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_F32 = 2, EPI_PK_SPLIT = 3 };
+
+constexpr int kMaxGemmGroups = 1024;
+
+// One grouped GEMM  out[r, :] = epi(A[r, :] . B_g^T)  for rows r of group g.
+// A [a_rows, K] bf16 row-major.  B for groups g < n_first: rows
+// [g*N, (g+1)*N) of B0 (and of B1 for SwiGLU); for g >= n_first the same rows
+// (g - n_first) of B2 (/B3).  SwiGLU: B0/B2 are W_gate, B1/B3 W_up and the
+// output h has N columns.  Groups: offsets [n_groups+1] on the device, or
+// uniform groups of group_rows rows when offsets == nullptr.
+struct GemmProblem {
+    int epi;
+    const void* A;
+    long long a_rows;
+    int K;
+    const void* B0;
+    const void* B1;
+    long long b01_rows;
+    const void* B2;
+    const void* B3;
+    long long b23_rows;
+    const int32_t* offsets;
+    int n_groups;
+    int n_first;
+    int group_rows;
+    int N;
+    void* out;
+    long long ldo;
+    long long rows_cap;   // rows of `out` (stores beyond are dropped)
+    int pk_T;             // EPI_PK_SPLIT: tokens
+    int pk_dq;            // EPI_PK_SPLIT: query width
+};
+
+moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st);
+
+// ------------------------------------------------------------ router
+struct RouterArgs {
+    const void* x;
+    const void* w_router;
+    const void* w_const_mix;
+    const float* bias;
+    const float* prev;
+    float* logits_out;
+    int32_t* idx;
+    float* gate;
+    float* const_mix;
+    int T, d, E_r, n_const, k;
+};
+moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st);
+
+struct PkSelectArgs {
+    const float* s_row;   // [T, rows]
+    const float* s_col;   // [T, cols]
+    float* logits_out;    // [T, rows + cols] nullable
+    int32_t* idx;         // [T, K]
+    float* gate;          // [T, K]
+    int T, rows, cols, kh, K;
+};
+moe_status launch_pk_select(const PkSelectArgs& a, cudaStream_t st);
+moe_status launch_pk_prep_keys(const void* k_row, const void* k_col, void* w3, int rows,
+                               int cols, int half, cudaStream_t st);
+
+// ------------------------------------------------------------ permute
+struct PermuteArgs {
+    const int32_t* idx;
+    const void* x;
+    int32_t* offsets;
+    int32_t* row_of;
+    int32_t* token_of;
+    void* x_sorted;
+    int32_t* ws_counts;   // [n_blocks, n_ffn] (SwiGLU) or [N] (atomic)
+    int32_t* ws_cursor;   // atomic: [N]
+    int32_t* ws_blocksum; // atomic scan: [scan blocks]
+    int T, k, d, n_ffn, n_shared, n_ids, elt_bytes;
+};
+moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st);
+moe_status launch_permute_atomic(const PermuteArgs& a, cudaStream_t st);
+int permute_blocks(int T);
+int atomic_scan_blocks(int N);
+
+// ------------------------------------------------------------ experts
+struct FfnF32Args {
+    const float* xs;
+    const int32_t* offsets;
+    const float* wg; const float* wu; const float* wd;      // routed
+    const float* sg; const float* su; const float* sd;      // shared
+    float* h;
+    float* ys;
+    int n_groups, n_first, d, H;
+    long long rows_cap;
+};
+moe_status launch_ffn_f32(const FfnF32Args& a, int phase, cudaStream_t st);
+
+struct AtomicArgs {
+    const void* x;        // [T, d] bf16
+    const void* u;        // [N, d]
+    const void* v;        // [N, d]
+    const int32_t* offsets;
+    const int32_t* token_of;   // task -> slot id
+    const int32_t* idx;        // [T, K]
+    const float* gate;         // [T, K]
+    float* c;                  // [T*K]
+    void* y;                   // [T, d] bf16, or fp32 if out_f32
+    int T, d, K, N;
+    int out_f32;
+};
+moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st);
+moe_status launch_atomic_phase_b(const AtomicArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------ combine
+struct CombineArgs {
+    const void* ys;
+    const int32_t* offsets;
+    const int32_t* row_of;
+    const int32_t* idx;
+    const float* gate;
+    const float* const_mix;
+    const void* const_vec;
+    const void* x;
+    void* y;
+    int T, d, k, n_ffn, n_shared, n_zero, n_copy, n_const;
+    long long rows_cap;
+    int out_f32;               // y fp32 whatever the input dtype
+};
+moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,579 @@
+// moe_api.cu -- the C ABI: argument checks, workspace layout, and the order
+// of kernel launches for each entry point.  Everything here runs on the
+// host; every step of the layer runs in the kernels of the other files.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+__device__ int g_status = 0;
+thread_local int t_launches = 0;
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int num_sms()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
+inline size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int elt(const moe_layer_desc* d) { return d->dtype == MOE_F32 ? 4 : 2; }
+inline int n_router_rows(const moe_layer_desc* d) { return d->n_ffn + d->n_zero + d->n_copy + d->n_const; }
+
+moe_status check_desc(const moe_layer_desc* d)
+{
+    if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->d_model <= 0 || d->top_k <= 0) return MOE_ERR_INVALID_ARG;
+    if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (d->out_f32 != 0 && d->out_f32 != 1) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        if (d->n_ffn < 0 || d->n_shared < 0 || d->n_zero < 0 || d->n_copy < 0 || d->n_const < 0)
+            return MOE_ERR_INVALID_ARG;
+        const int E = n_router_rows(d);
+        if (E <= 0 || d->top_k > E) return MOE_ERR_INVALID_ARG;
+        if (d->n_ffn > 0 && d->hidden <= 0) return MOE_ERR_INVALID_ARG;
+        if (d->n_shared > 0 && d->hidden_shared != d->hidden) return MOE_ERR_UNSUPPORTED;
+        if (d->top_k > 32 || E + 2 * d->n_const > 256 || d->n_ffn > 1024) return MOE_ERR_UNSUPPORTED;
+        if (d->n_ffn + d->n_shared > kMaxGemmGroups) return MOE_ERR_UNSUPPORTED;
+        if (d->pk_rows || d->pk_cols || d->pk_topk_half || d->d_query) return MOE_ERR_INVALID_ARG;
+        if (d->dtype == MOE_BF16) {
+            if (d->d_model % 64 != 0 || (d->n_ffn + d->n_shared > 0 && d->hidden % 128 != 0))
+                return MOE_ERR_UNSUPPORTED;
+        } else {
+            if (d->d_model % 8 != 0 || (d->hidden > 0 && d->hidden % 4 != 0)) return MOE_ERR_UNSUPPORTED;
+        }
+        const long long cap = (long long)d->T * d->top_k + (long long)d->n_shared * d->T;
+        if (cap >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+        return MOE_OK;
+    }
+    if (d->kind == MOE_EXPERT_ATOMIC_GELU) {
+        if (d->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+        if (d->n_ffn || d->n_shared || d->n_zero || d->n_copy || d->n_const || d->hidden)
+            return MOE_ERR_INVALID_ARG;
+        if (d->pk_rows <= 0 || d->pk_cols <= 0 || d->pk_topk_half <= 0 || d->d_query <= 0)
+            return MOE_ERR_INVALID_ARG;
+        if (d->pk_topk_half > d->pk_rows || d->pk_topk_half > d->pk_cols) return MOE_ERR_INVALID_ARG;
+        if (d->top_k > d->pk_topk_half * d->pk_topk_half) return MOE_ERR_INVALID_ARG;
+        if (d->pk_rows != d->pk_cols || d->pk_rows % 32 != 0 || d->pk_rows > 1024) return MOE_ERR_UNSUPPORTED;
+        if (d->pk_topk_half > 32 || d->top_k > 128) return MOE_ERR_UNSUPPORTED;
+        if (d->d_query % 64 != 0) return MOE_ERR_UNSUPPORTED;
+        const int nv = d->d_model / 256;
+        if (d->d_model % 256 != 0 || !(nv == 1 || nv == 2 || nv == 4 || nv == 8)) return MOE_ERR_UNSUPPORTED;
+        if ((long long)d->pk_rows * d->pk_cols >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+        if ((long long)d->T * d->top_k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+        return MOE_OK;
+    }
+    return MOE_ERR_INVALID_ARG;
+}
+
+// -------------------------------------------------------------- workspace
+
+struct Scratch {   // byte sizes of each call's scratch
+    size_t route, permute, ffn;
+};
+
+Scratch scratch_sizes(const moe_layer_desc* d)
+{
+    Scratch s{0, 0, 0};
+    const long long cap = moe_row_capacity(d);
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        s.permute = al((size_t)permute_blocks(d->T) * std::max(d->n_ffn, 1) * 4);
+        s.ffn = (d->n_ffn + d->n_shared > 0) ? al((size_t)cap * d->hidden * elt(d)) : 0;
+    } else {
+        const size_t half = d->d_query / 2;
+        s.route = al((size_t)2 * d->T * 3 * half * 2) + al((size_t)(d->pk_rows + d->pk_cols) * 3 * half * 2) +
+                  al((size_t)2 * d->T * d->pk_rows * 4);
+        const size_t N = (size_t)d->pk_rows * d->pk_cols;
+        s.permute = al(N * 4) * 2 + al((size_t)atomic_scan_blocks((int)N) * 4);
+    }
+    return s;
+}
+
+size_t scratch_max(const moe_layer_desc* d)
+{
+    const Scratch s = scratch_sizes(d);
+    return std::max(std::max(s.route, s.permute), std::max(s.ffn, (size_t)256));
+}
+
+struct LayerBufs {
+    int32_t* idx;
+    float* gate;
+    float* cmix;
+    int32_t* offsets;
+    int32_t* row_of;
+    int32_t* token_of;
+    void* xs;
+    void* ys;
+    void* scratch;
+    size_t scratch_bytes;
+    size_t total;
+};
+
+LayerBufs layer_layout(const moe_layer_desc* d, void* base)
+{
+    LayerBufs b;
+    char* p = static_cast<char*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { char* r = p ? p + o : nullptr; o += al(bytes); return r; };
+    const long long Tk = (long long)d->T * d->top_k;
+    const long long cap = moe_row_capacity(d);
+    b.idx = reinterpret_cast<int32_t*>(take(Tk * 4));
+    b.gate = reinterpret_cast<float*>(take(Tk * 4));
+    b.cmix = reinterpret_cast<float*>(take((size_t)d->T * std::max(d->n_const, 0) * 2 * 4));
+    b.offsets = reinterpret_cast<int32_t*>(take((moe_num_groups(d) + 1) * 4));
+    b.row_of = reinterpret_cast<int32_t*>(take(Tk * 4));
+    b.token_of = reinterpret_cast<int32_t*>(take(cap * 4));
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        b.xs = take((size_t)cap * d->d_model * elt(d));
+        b.ys = take((size_t)cap * d->d_model * 4);
+    } else {
+        b.xs = nullptr;
+        b.ys = take((size_t)Tk * 4);
+    }
+    b.scratch_bytes = scratch_max(d);
+    b.scratch = take(b.scratch_bytes);
+    b.total = o;
+    return b;
+}
+
+// --------------------------------------------------------- implementations
+
+moe_status route_impl(const moe_layer_desc* d, const moe_layer_weights* w, const void* x,
+                      const float* prev, float* logits_out, int32_t* idx, float* gate, float* cmix,
+                      void* ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (d->T == 0) return MOE_OK;
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        if (!w->w_router || !aligned16(w->w_router) || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+        if (d->n_const > 0 && (!cmix || !w->w_const_mix || !aligned16(w->w_const_mix)))
+            return MOE_ERR_INVALID_ARG;
+        RouterArgs a;
+        a.x = x;
+        a.w_router = w->w_router;
+        a.w_const_mix = w->w_const_mix;
+        a.bias = w->router_bias;
+        a.prev = prev;
+        a.logits_out = logits_out;
+        a.idx = idx;
+        a.gate = gate;
+        a.const_mix = cmix;
+        a.T = d->T;
+        a.d = d->d_model;
+        a.E_r = n_router_rows(d);
+        a.n_const = d->n_const;
+        a.k = d->top_k;
+        return launch_router(d->dtype, a, st);
+    }
+    // atomic: q = W_q x split into bf16 parts -> sub-key scores -> selection
+    if (!w->w_query || !w->subkeys_row || !w->subkeys_col) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->w_query) || !aligned16(w->subkeys_row) || !aligned16(w->subkeys_col) || !aligned16(x))
+        return MOE_ERR_INVALID_ARG;
+    const Scratch sc = scratch_sizes(d);
+    if (!ws || ws_bytes < sc.route || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    const int half = d->d_query / 2;
+    char* p = static_cast<char*>(ws);
+    void* a3 = p;
+    p += al((size_t)2 * d->T * 3 * half * 2);
+    void* w3 = p;
+    p += al((size_t)(d->pk_rows + d->pk_cols) * 3 * half * 2);
+    float* scores = reinterpret_cast<float*>(p);
+    moe_status s = launch_pk_prep_keys(w->subkeys_row, w->subkeys_col, w3, d->pk_rows, d->pk_cols, half, st);
+    if (s != MOE_OK) return s;
+    GemmProblem q{};
+    q.epi = EPI_PK_SPLIT;
+    q.A = x;
+    q.a_rows = d->T;
+    q.K = d->d_model;
+    q.B0 = w->w_query;
+    q.b01_rows = d->d_query;
+    q.offsets = nullptr;
+    q.n_groups = 1;
+    q.n_first = 1;
+    q.group_rows = d->T;
+    q.N = d->d_query;
+    q.out = a3;
+    q.ldo = 3 * half;
+    q.rows_cap = d->T;
+    q.pk_T = d->T;
+    q.pk_dq = d->d_query;
+    if ((s = launch_grouped_gemm(q, st)) != MOE_OK) return s;
+    GemmProblem g{};
+    g.epi = EPI_F32;
+    g.A = a3;
+    g.a_rows = 2ll * d->T;
+    g.K = 3 * half;
+    g.B0 = w3;
+    g.b01_rows = d->pk_rows + d->pk_cols;
+    g.offsets = nullptr;
+    g.n_groups = 2;
+    g.n_first = 2;
+    g.group_rows = d->T;
+    g.N = d->pk_rows;
+    g.out = scores;
+    g.ldo = d->pk_rows;
+    g.rows_cap = 2ll * d->T;
+    if ((s = launch_grouped_gemm(g, st)) != MOE_OK) return s;
+    PkSelectArgs ps;
+    ps.s_row = scores;
+    ps.s_col = scores + (size_t)d->T * d->pk_rows;
+    ps.logits_out = logits_out;
+    ps.idx = idx;
+    ps.gate = gate;
+    ps.T = d->T;
+    ps.rows = d->pk_rows;
+    ps.cols = d->pk_cols;
+    ps.kh = d->pk_topk_half;
+    ps.K = d->top_k;
+    return launch_pk_select(ps, st);
+}
+
+moe_status permute_impl(const moe_layer_desc* d, const int32_t* idx, const void* x, int32_t* offsets,
+                        int32_t* row_of, int32_t* token_of, void* xs, void* ws, size_t ws_bytes,
+                        cudaStream_t st)
+{
+    const Scratch sc = scratch_sizes(d);
+    if (!ws || ws_bytes < sc.permute || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    PermuteArgs a{};
+    a.idx = idx;
+    a.x = x;
+    a.offsets = offsets;
+    a.row_of = row_of;
+    a.token_of = token_of;
+    a.x_sorted = xs;
+    a.T = d->T;
+    a.k = d->top_k;
+    a.d = d->d_model;
+    a.elt_bytes = elt(d);
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        if (xs && (!x || !aligned16(x) || !aligned16(xs))) return MOE_ERR_INVALID_ARG;
+        a.ws_counts = static_cast<int32_t*>(ws);
+        a.n_ffn = d->n_ffn;
+        a.n_shared = d->n_shared;
+        a.n_ids = n_router_rows(d);
+        return launch_permute_swiglu(a, st);
+    }
+    const size_t N = (size_t)d->pk_rows * d->pk_cols;
+    char* p = static_cast<char*>(ws);
+    a.ws_counts = reinterpret_cast<int32_t*>(p);
+    a.ws_cursor = reinterpret_cast<int32_t*>(p + al(N * 4));
+    a.ws_blocksum = reinterpret_cast<int32_t*>(p + 2 * al(N * 4));
+    a.n_ffn = 0;
+    a.n_shared = 0;
+    a.n_ids = (int)N;
+    a.x_sorted = nullptr;
+    return launch_permute_atomic(a, st);
+}
+
+moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* xs,
+                          const int32_t* offsets, void* ys, void* ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (d->n_ffn + d->n_shared == 0) return MOE_OK;
+    const Scratch sc = scratch_sizes(d);
+    if (!ws || ws_bytes < sc.ffn || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (d->n_ffn > 0 && (!w->w_gate || !w->w_up || !w->w_down)) return MOE_ERR_INVALID_ARG;
+    if (d->n_shared > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_ERR_INVALID_ARG;
+    const long long cap = moe_row_capacity(d);
+    if (d->dtype == MOE_F32) {
+        FfnF32Args a;
+        a.xs = static_cast<const float*>(xs);
+        a.offsets = offsets;
+        a.wg = static_cast<const float*>(w->w_gate);
+        a.wu = static_cast<const float*>(w->w_up);
+        a.wd = static_cast<const float*>(w->w_down);
+        a.sg = static_cast<const float*>(w->ws_gate);
+        a.su = static_cast<const float*>(w->ws_up);
+        a.sd = static_cast<const float*>(w->ws_down);
+        a.h = static_cast<float*>(ws);
+        a.ys = static_cast<float*>(ys);
+        a.n_groups = d->n_ffn + d->n_shared;
+        a.n_first = d->n_ffn;
+        a.d = d->d_model;
+        a.H = d->hidden;
+        a.rows_cap = cap;
+        return launch_ffn_f32(a, phase, st);
+    }
+    const void* ptrs[8] = {xs, ys, w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    GemmProblem g{};
+    g.offsets = offsets;
+    g.n_groups = d->n_ffn + d->n_shared;
+    g.n_first = d->n_ffn;
+    g.rows_cap = cap;
+    if (phase == 1) {
+        g.epi = EPI_SWIGLU;
+        g.A = xs;
+        g.a_rows = cap;
+        g.K = d->d_model;
+        g.B0 = d->n_ffn ? w->w_gate : w->ws_gate;
+        g.B1 = d->n_ffn ? w->w_up : w->ws_up;
+        g.b01_rows = (long long)std::max(d->n_ffn, 1) * d->hidden;
+        g.B2 = w->ws_gate;
+        g.B3 = w->ws_up;
+        g.b23_rows = (long long)d->n_shared * d->hidden;
+        g.N = d->hidden;
+        g.out = ws;
+        g.ldo = d->hidden;
+    } else {
+        g.epi = EPI_F32;
+        g.A = ws;
+        g.a_rows = cap;
+        g.K = d->hidden;
+        g.B0 = d->n_ffn ? w->w_down : w->ws_down;
+        g.b01_rows = (long long)std::max(d->n_ffn, 1) * d->d_model;
+        g.B2 = w->ws_down;
+        g.b23_rows = (long long)d->n_shared * d->d_model;
+        g.N = d->d_model;
+        g.out = ys;
+        g.ldo = d->d_model;
+    }
+    return launch_grouped_gemm(g, st);
+}
+
+moe_status ffn_impl(const moe_layer_desc* d, const moe_layer_weights* w, const void* xs,
+                    const int32_t* offsets, const int32_t* token_of, const void* x, const float* gate,
+                    void* ys, void* ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (d->kind == MOE_EXPERT_SWIGLU) {
+        moe_status s = ffn_phase_impl(d, w, 1, xs, offsets, ys, ws, ws_bytes, st);
+        if (s != MOE_OK) return s;
+        return ffn_phase_impl(d, w, 2, xs, offsets, ys, ws, ws_bytes, st);
+    }
+    if (!w->u || !aligned16(w->u) || !x || !aligned16(x) || !gate || !token_of) return MOE_ERR_INVALID_ARG;
+    AtomicArgs a{};
+    a.x = x;
+    a.u = w->u;
+    a.v = w->v;
+    a.offsets = offsets;
+    a.token_of = token_of;
+    a.gate = gate;
+    a.c = static_cast<float*>(ys);
+    a.T = d->T;
+    a.d = d->d_model;
+    a.K = d->top_k;
+    a.N = d->pk_rows * d->pk_cols;
+    return launch_atomic_phase_a(a, st);
+}
+
+moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, const void* ys,
+                        const int32_t* offsets, const int32_t* row_of, const int32_t* idx,
+                        const float* gate, const float* cmix, const void* x, void* y, cudaStream_t st)
+{
+    if (d->T == 0) return MOE_OK;
+    if (!y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_ATOMIC_GELU) {
+        if (!w->v || !aligned16(w->v)) return MOE_ERR_INVALID_ARG;
+        AtomicArgs a{};
+        a.v = w->v;
+        a.idx = idx;
+        a.c = const_cast<float*>(static_cast<const float*>(ys));
+        a.y = y;
+        a.T = d->T;
+        a.d = d->d_model;
+        a.K = d->top_k;
+        a.N = d->pk_rows * d->pk_cols;
+        a.out_f32 = d->out_f32;
+        return launch_atomic_phase_b(a, st);
+    }
+    if ((d->n_copy + d->n_const > 0) && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    if (d->n_const > 0 && (!cmix || !w->const_vec || !aligned16(w->const_vec))) return MOE_ERR_INVALID_ARG;
+    if ((d->n_ffn + d->n_shared > 0) && (!ys || !aligned16(ys))) return MOE_ERR_INVALID_ARG;
+    CombineArgs a{};
+    a.ys = ys;
+    a.offsets = offsets;
+    a.row_of = row_of;
+    a.idx = idx;
+    a.gate = gate;
+    a.const_mix = cmix;
+    a.const_vec = w->const_vec;
+    a.x = x;
+    a.y = y;
+    a.T = d->T;
+    a.d = d->d_model;
+    a.k = d->top_k;
+    a.n_ffn = d->n_ffn;
+    a.n_shared = d->n_shared;
+    a.n_zero = d->n_zero;
+    a.n_copy = d->n_copy;
+    a.n_const = d->n_const;
+    a.rows_cap = moe_row_capacity(d);
+    a.out_f32 = d->out_f32;
+    return launch_combine(d->dtype, a, st);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_num_groups(const moe_layer_desc* d)
+{
+    if (check_desc(d) != MOE_OK) return -1;
+    if (d->kind == MOE_EXPERT_SWIGLU) return d->n_ffn + d->n_shared;
+    return (int64_t)d->pk_rows * d->pk_cols;
+}
+
+int64_t moe_row_capacity(const moe_layer_desc* d)
+{
+    if (check_desc(d) != MOE_OK) return -1;
+    const int64_t Tk = (int64_t)d->T * d->top_k;
+    if (d->kind == MOE_EXPERT_SWIGLU) return Tk + (int64_t)d->n_shared * d->T;
+    return Tk;
+}
+
+int64_t moe_workspace_size(const moe_layer_desc* d)
+{
+    if (check_desc(d) != MOE_OK) return -1;
+    return (int64_t)scratch_max(d);
+}
+
+int64_t moe_layer_workspace_size(const moe_layer_desc* d)
+{
+    if (check_desc(d) != MOE_OK) return -1;
+    return (int64_t)layer_layout(d, nullptr).total;
+}
+
+moe_status moe_route(const moe_layer_desc* d, const moe_layer_weights* w, const void* x,
+                     const float* prev_logits, float* logits_out, int32_t* topk_idx, float* topk_gate,
+                     float* const_mix, void* workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || (d->T > 0 && (!x || !topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
+    return route_impl(d, w, x, prev_logits, logits_out, topk_idx, topk_gate, const_mix, workspace, ws_bytes,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_permute(const moe_layer_desc* d, const int32_t* topk_idx, const void* x,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* token_of, void* x_sorted,
+                       void* workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!expert_offsets || (d->T > 0 && (!topk_idx || !row_of || !token_of))) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_SWIGLU && d->T > 0 && d->n_ffn + d->n_shared > 0 && !x_sorted)
+        return MOE_ERR_INVALID_ARG;
+    return permute_impl(d, topk_idx, x, expert_offsets, row_of, token_of, x_sorted, workspace, ws_bytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_grouped_ffn(const moe_layer_desc* d, const moe_layer_weights* w, const void* x_sorted,
+                           const int32_t* expert_offsets, const int32_t* token_of, const void* x,
+                           const float* topk_gate, void* y_sorted, void* workspace, size_t ws_bytes,
+                           moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || !expert_offsets || (d->T > 0 && !y_sorted)) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_SWIGLU && d->T > 0 && !x_sorted) return MOE_ERR_INVALID_ARG;
+    return ffn_impl(d, w, x_sorted, expert_offsets, token_of, x, topk_gate, y_sorted, workspace, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_grouped_ffn_phase(const moe_layer_desc* d, const moe_layer_weights* w, int phase,
+                                 const void* x_sorted, const int32_t* expert_offsets, void* y_sorted,
+                                 void* workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (d->kind != MOE_EXPERT_SWIGLU || (phase != 1 && phase != 2)) return MOE_ERR_INVALID_ARG;
+    if (!w || !expert_offsets || (d->T > 0 && (!x_sorted || !y_sorted))) return MOE_ERR_INVALID_ARG;
+    return ffn_phase_impl(d, w, phase, x_sorted, expert_offsets, y_sorted, workspace, ws_bytes,
+                          static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_layer_desc* d, const moe_layer_weights* w, const void* y_sorted,
+                       const int32_t* expert_offsets, const int32_t* row_of, const int32_t* topk_idx,
+                       const float* topk_gate, const float* const_mix, const void* x, void* y,
+                       moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || (d->T > 0 && (!topk_idx || !topk_gate || !y))) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_SWIGLU && d->T > 0 && (!row_of || !expert_offsets)) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_ATOMIC_GELU && d->T > 0 && !y_sorted) return MOE_ERR_INVALID_ARG;
+    return combine_impl(d, w, y_sorted, expert_offsets, row_of, topk_idx, topk_gate, const_mix, x, y,
+                        static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_layer_forward(const moe_layer_desc* d, const moe_layer_weights* w, const void* x,
+                             const float* prev_logits, void* y, float* logits_out, void* workspace,
+                             size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || (d->T > 0 && (!x || !y))) return MOE_ERR_INVALID_ARG;
+    const LayerBufs need = layer_layout(d, nullptr);
+    if (!workspace || ws_bytes < need.total || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
+    const LayerBufs b = layer_layout(d, workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d->T == 0) return MOE_OK;
+    if ((s = route_impl(d, w, x, prev_logits, logits_out, b.idx, b.gate, b.cmix, b.scratch, b.scratch_bytes, st)) != MOE_OK)
+        return s;
+    if ((s = permute_impl(d, b.idx, x, b.offsets, b.row_of, b.token_of, b.xs, b.scratch, b.scratch_bytes, st)) != MOE_OK)
+        return s;
+    if ((s = ffn_impl(d, w, b.xs, b.offsets, b.token_of, x, b.gate, b.ys, b.scratch, b.scratch_bytes, st)) != MOE_OK)
+        return s;
+    return combine_impl(d, w, b.ys, b.offsets, b.row_of, b.idx, b.gate, b.cmix, x, y, st);
+}
+
+moe_status moe_get_device_status(moe_status* out, int reset, moe_stream_t stream)
+{
+    if (!out) return MOE_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int))) != cudaSuccess) return MOE_ERR_CUDA;
+    if (reset) {
+        const int zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int))) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    *out = static_cast<moe_status>(v);
+    return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s)
+{
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE_BOUNDS: return "kernel saw an invalid index";
+        case MOE_ERR_TIMEOUT: return "kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t moe_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+"""CUDA path (through the C ABI) vs the fp64 oracle, element by element.
+
+Small cases compare every output; the full-size workloads compare routing and
+the permutation for every token and the outputs of sampled tokens.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from moe_workloads import get_config, make_inputs, scaled
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_swiglu_b200 as moe  # noqa: E402
+    from parity import check_atomic_layer, check_swiglu_layer, run_gpu, to_device  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    if torch.cuda.is_available():
+        moe.moe_get_device_status(reset=True)
+    yield
+
+
+def _report(name: str, rep: dict) -> None:
+    print(f"\n{name}: margin<1e-6 {rep['below_1e-6']}, within error {len(rep['near_tie'])}, "
+          f"routing mismatches {len(rep['mismatch'])} (margins {np.round(rep['mismatch_margins'][:6], 9)}), "
+          f"fp32 result err/rms {rep['rel_err']:.3e}, dtype output err/rms {rep['rel_err_out']:.3e}"
+          + (f", routed rows {rep['R']}" if "R" in rep else ""))
+
+
+def _sample(T: int, n: int, seed: int = 0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    s = set(rng.choice(T, size=min(n, T), replace=False).tolist()) | {0, T - 1}
+    return np.array(sorted(s), dtype=np.int32)
+
+
+# ------------------------------------------------------------ small, every output
+
+def test_tiny_f32_full_layer():
+    cfg = get_config("tiny_f32")
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["rel_err"] <= 1e-4
+
+
+def test_mixtral_shaped_small_ragged():
+    cfg = scaled(get_config("mixtral"), T=333, d=512, hidden=1024)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["R"] == 333 * 2
+
+
+def test_longtail_shared_experts():
+    cfg = scaled(get_config("longtail"), T=200)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["R"] == 200 * 6
+
+
+def test_moepp_zero_copy_const_residual():
+    cfg = scaled(get_config("moepp"), T=300, hidden=640)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["R"] < 300 * 2          # some slots went to zero-computation experts
+
+
+def test_atomic_small_grid():
+    cfg = scaled(get_config("atomic"), T=100, d=256, pk_rows=64, pk_cols=64, pk_topk_half=16,
+                 top_k=32, d_query=128)
+    check_atomic_layer(cfg, make_inputs(cfg))
+
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129])
+def test_bf16_token_counts_across_tile_edges(T):
+    cfg = scaled(get_config("mixtral"), T=T, d=256, hidden=384, n_ffn=4)
+    check_swiglu_layer(cfg, make_inputs(cfg))
+
+
+def test_all_tokens_one_expert_and_empty_experts():
+    cfg = scaled(get_config("mixtral"), T=300, d=256, hidden=256, n_ffn=6, top_k=1)
+    inp = make_inputs(cfg)
+    inp["router_bias"] = torch.tensor([0, 0, 0, 50.0, 0, 0])     # every token picks expert 3
+    rep = check_swiglu_layer(cfg, inp)
+    assert rep["R"] == 300
+
+
+def test_empty_batch_is_a_no_op():
+    cfg = scaled(get_config("mixtral"), T=0, d=256, hidden=256, n_ffn=4)
+    inp = to_device(make_inputs(scaled(cfg, T=1)))
+    desc = moe.desc_from(cfg)
+    x = inp["x"][:0]
+    y = torch.empty_like(x)
+    layer = moe.MoELayer(desc, inp)
+    layer.forward(x, y=y)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
+def test_layer_forward_equals_stages():
+    cfg = scaled(get_config("longtail"), T=150)
+    inp = to_device(make_inputs(cfg))
+    r = run_gpu(cfg, inp)
+    layer = moe.MoELayer(r["desc"], inp)
+    y = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(y, r["bufs"].y)
+
+
+def test_invalid_expert_id_sets_bounds_status():
+    cfg = scaled(get_config("mixtral"), T=64, d=256, hidden=256, n_ffn=4)
+    inp = to_device(make_inputs(cfg))
+    desc = moe.desc_from(cfg)
+    b = moe.StageBuffers(desc)
+    idx = torch.zeros((64, 2), dtype=torch.int32, device="cuda")
+    idx[:, 1] = 1
+    idx[5, 1] = 7            # out of range: 4 experts
+    moe.moe_permute(desc, idx, inp["x"], b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace)
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_ERR_DEVICE_BOUNDS
+    idx[5, 1] = 0            # same expert twice in one token
+    moe.moe_permute(desc, idx, inp["x"], b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace)
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_ERR_DEVICE_BOUNDS
+    idx[5, 1] = 1
+    moe.moe_permute(desc, idx, inp["x"], b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace)
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+
+
+def test_argument_errors_return_before_launch():
+    cfg = scaled(get_config("mixtral"), T=8, d=256, hidden=256, n_ffn=4)
+    inp = to_device(make_inputs(cfg))
+    desc = moe.desc_from(cfg)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        moe.moe_layer_forward(desc, inp, inp["x"], None, torch.empty_like(inp["x"]), None, small)
+    assert e.value.status == moe.MOE_ERR_WORKSPACE
+    bad = moe.desc_from(scaled(cfg, hidden=200))       # hidden not a multiple of 128 on bf16
+    assert moe.moe_layer_workspace_size(bad) == -1
+
+
+# ------------------------------------------------------------ full-size workloads
+
+def test_mixtral_full_size_sampled():
+    cfg = get_config("mixtral")
+    rep = check_swiglu_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 12), check_sorted=True)
+    _report("mixtral", rep)
+
+
+def test_longtail_full_size_sampled():
+    cfg = get_config("longtail")
+    rep = check_swiglu_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 24))
+    _report("longtail", rep)
+
+
+def test_moepp_full_size_sampled():
+    cfg = get_config("moepp")
+    rep = check_swiglu_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 24))
+    _report("moepp", rep)
+
+
+def test_atomic_full_size_sampled():
+    cfg = get_config("atomic")
+    rep = check_atomic_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 48))
+    _report("atomic", rep)
