@@ -1,0 +1,384 @@
+"""Benchmark of the MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (one rank per GPU)
+
+A step is one pass of the whole hot path -- router + top-k, histogram / scan
+/ permutation, grouped gate/up GEMM with SwiGLU, grouped down GEMM, combine --
+over one batch of the Mixtral-shaped workload (T=4096 tokens, d=4096, 8 SwiGLU
+experts of hidden 14336, top-2, bf16, seeded synthetic inputs).  Ranks run
+independent token batches on replicated weights (no collective on the data
+path; weak scaling); `value` is the tokens of all ranks per second, time
+being the max over ranks of the summed per-step device times.
+
+Prints one JSON line (rank 0).  Extra keys: per-kernel times, the roofline of
+the dominant kernel, the fp64 oracle timed on the host cores (cpu_baseline),
+the end-to-end figure through moe_layer_forward with host buffers (e2e), the
+SM clocks seen during the timed region, and the number of our kernels
+launched in it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+from moe_workloads import get_config, make_activations, make_weights  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec on 1 B200; % of bf16 tensor / HBM roofline"
+WORKLOAD = "mixtral"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--oracle-tokens", type=int, default=0,
+                   help="tokens in the CPU oracle sample (0: sized to ~15 s)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
+    p.add_argument("--experts", type=int, default=0, help="override the expert count (profiling)")
+    return p.parse_args()
+
+
+def bench_config(args):
+    from moe_workloads import scaled
+    cfg = get_config(WORKLOAD)
+    ch = {}
+    if args.tokens:
+        ch["T"] = args.tokens
+    if args.experts:
+        ch["n_ffn"] = args.experts
+    return scaled(cfg, **ch) if ch else cfg
+
+
+def workload_config(cfg) -> dict:
+    return {"workload": f"{cfg.name}_T{cfg.T}_d{cfg.d}_E{cfg.n_ffn}_H{cfg.hidden}_k{cfg.top_k}",
+            "T_per_gpu": cfg.T, "d_model": cfg.d, "experts": cfg.n_ffn, "hidden": cfg.hidden,
+            "top_k": cfg.top_k, "router": "softmax over top-k", "parallelism": "token-sharded replicas",
+            "l2": "flushed between steps (256 MiB write outside the step events)"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """SM clock and throttle reasons of one GPU, sampled every 20 ms via NVML
+    (read-only queries)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:   # match the CUDA device to the NVML device by PCI address
+                p = torch.cuda.get_device_properties(index)
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:   # noqa: BLE001
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:   # noqa: BLE001
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._reasons_fn(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:   # noqa: BLE001
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self) -> dict:
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
+    """The fp64 oracle as it stands on a bounded sample of the workload's
+    tokens (routing + experts of each token), on all host cores."""
+    import numpy as np
+
+    import oracle
+    threads = oracle.num_threads()
+    if n_tokens <= 0:   # size the sample: time a small probe first
+        t0 = time.perf_counter()
+        oracle.moe_tokens(cfg, inp, np.arange(threads, dtype=np.int32))
+        per_tok = (time.perf_counter() - t0) / threads
+        n_tokens = int(max(threads, min(cfg.T, seconds / max(per_tok, 1e-6))))
+    toks = np.linspace(0, cfg.T - 1, n_tokens).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.moe_tokens(cfg, inp, toks)
+    el = time.perf_counter() - t0
+    return {"value": n_tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_tokens} of the {cfg.T} tokens (evenly spaced), full routing + experts per token, "
+                      f"{el:.1f} s"}
+
+
+# ------------------------------------------------------------------- ours
+
+def run_ours(args, rank: int, world: int, dist) -> dict | None:
+    import mixture_experts_layer_swiglu_b200 as moe
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    cfg = bench_config(args)
+    w_cpu = make_weights(cfg, seed=0)
+    a_cpu = make_activations(cfg, seed=rank)           # each rank its own tokens
+    w = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in w_cpu.items()}
+    x = a_cpu["x"].to(dev)
+    desc = moe.desc_from(cfg)
+    ws = moe.weights_struct(w)
+    b = moe.StageBuffers(desc, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        """One pass of the hot path; events between the stages if given."""
+        launches = 0
+        if ev: ev[0].record(stream)
+        moe.moe_route(desc, ws, x, None, None, b.idx, b.gate, None, b.workspace, stream)
+        launches += moe.moe_last_launch_count()
+        if ev: ev[1].record(stream)
+        moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace, stream)
+        launches += moe.moe_last_launch_count()
+        if ev: ev[2].record(stream)
+        moe.moe_grouped_ffn_phase(desc, ws, 1, b.x_sorted, b.offsets, b.y_sorted, b.workspace, stream)
+        launches += moe.moe_last_launch_count()
+        if ev: ev[3].record(stream)
+        moe.moe_grouped_ffn_phase(desc, ws, 2, b.x_sorted, b.offsets, b.y_sorted, b.workspace, stream)
+        launches += moe.moe_last_launch_count()
+        if ev: ev[4].record(stream)
+        moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, None, x, b.y, stream)
+        launches += moe.moe_last_launch_count()
+        if ev: ev[5].record(stream)
+        return launches
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    with ClockSampler(dev.index) as clk:
+        for i in range(K):
+            flush.zero_()
+            launches += step(evs[i])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    status = moe.moe_get_device_status(reset=True)
+    assert status == moe.MOE_OK, moe.status_string(status)
+    names = ["router", "permute", "gate_up_gemm", "down_gemm", "combine"]
+    per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)] for j, n in enumerate(names)}
+    step_ms = [evs[i][0].elapsed_time(evs[i][5]) for i in range(K)]
+    total_ms = sum(step_ms)
+    R = int(b.offsets[-1].item())
+
+    # end to end through the public call with host buffers
+    x_host = a_cpu["x"].pin_memory()
+    y_host = torch.empty(x_host.shape, dtype=x_host.dtype).pin_memory()
+    layer = moe.MoELayer(desc, w)
+    x_dev = torch.empty_like(x)
+    y_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, y=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    KE = max(3, K // 4)
+    e2e_ms = 0.0
+    for _ in range(KE):
+        flush.zero_()
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, y=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+
+    mean = {n: sum(v) / K for n, v in per.items()}
+    res = {"total_ms": total_ms, "e2e_ms": e2e_ms / KE, "mean": mean, "R": R, "launches": launches,
+           "clocks": clk.summary(), "T": cfg.T}
+    if dist:   # max over ranks
+        t = torch.tensor([total_ms, res["e2e_ms"]] + [mean[n] for n in names], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        res["total_ms"], res["e2e_ms"] = float(t[0]), float(t[1])
+        res["mean"] = {n: float(t[2 + j]) for j, n in enumerate(names)}
+    if rank != 0:
+        return None
+
+    peaks = {}
+    pk = ROOT / "MEASURED_PEAKS.json"
+    if pk.exists():
+        peaks = json.loads(pk.read_text())
+    peak_tf = peaks.get("bf16_tflops")
+    peak_src = "measured burst (MEASURED_PEAKS.json)" if peak_tf else "fallback"
+    if not peak_tf:
+        peak_tf = 1590.0
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    d, H = cfg.d, cfg.hidden
+    flops_gu = 4.0 * R * d * H
+    flops_dn = 2.0 * R * d * H
+    gu_s = res["mean"]["gate_up_gemm"] / 1e3
+    achieved = flops_gu / gu_s / 1e12
+    traffic = _ncu_traffic("gate_up_gemm", WORKLOAD)
+    ms_step = res["total_ms"] / K
+    value = world * cfg.T / (ms_step / 1e3)
+    kern = {}
+    for n in names:
+        ms = res["mean"][n]
+        kern[n] = {"ms": round(ms, 4), "share": round(ms / ms_step, 4)}
+    kern["gate_up_gemm"]["tflops"] = round(flops_gu / (res["mean"]["gate_up_gemm"] / 1e3) / 1e12, 1)
+    kern["down_gemm"]["tflops"] = round(flops_dn / (res["mean"]["down_gemm"] / 1e3) / 1e12, 1)
+    e = cfg.elt_bytes
+    Tk = cfg.T * cfg.top_k
+    router_bytes = cfg.T * d * e + cfg.n_routed * d * e + Tk * 8
+    permute_bytes = cfg.T * d * e + R * d * e + Tk * 12
+    combine_bytes = R * d * 4 + cfg.T * d * e + Tk * 12
+    for n, by in (("router", router_bytes), ("permute", permute_bytes), ("combine", combine_bytes)):
+        kern[n]["gbs"] = round(by / (res["mean"][n] / 1e3) / 1e9, 1)
+        kern[n]["hbm_frac"] = round(kern[n]["gbs"] / hbm, 3)
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = y_host.numel() * y_host.element_size()
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights)",
+        "config": workload_config(cfg),
+        "roofline": {"bound": "tensor", "kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)",
+                     "achieved": round(achieved, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_tf, 4), "traffic": traffic,
+                     "peak_source": peak_src, "flops_per_launch": flops_gu},
+        "kernels": kern,
+        "step_tflops": round((flops_gu + flops_dn) / (ms_step / 1e3) / 1e12, 1),
+        "e2e": {"value": round(world * cfg.T / (res["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": "moe_layer_forward, x from pinned host, y to pinned host"},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        w_cpu.update(a_cpu)
+        out["cpu_baseline"] = cpu_oracle_leg(cfg, w_cpu, args.oracle_tokens)
+    return out
+
+
+def _ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if
+    one exists for the current kernel source (else null)."""
+    f = ROOT / "profiles" / f"{kernel}_{workload}.md"
+    if not f.exists():
+        return None
+    for line in f.read_text().splitlines():
+        if line.startswith("dram_bytes_per_launch:"):
+            try:
+                return float(line.split(":", 1)[1].split()[0])
+            except ValueError:
+                return None
+    return None
+
+
+# -------------------------------------------------------------- reference
+
+def run_reference(args, rank: int, world: int) -> dict | None:
+    """The reference arm: the fp64 CPU oracle on the host cores, each step a
+    bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import oracle
+    cfg = bench_config(args)
+    inp = make_weights(cfg, seed=0)
+    inp.update(make_activations(cfg, seed=0))
+    n = args.oracle_tokens or max(8, oracle.num_threads())
+    rng = np.random.default_rng(0)
+    for _ in range(min(args.warmup, 1)):
+        oracle.moe_tokens(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_tokens(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    base = {"value": round(value, 3), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} random tokens of the {cfg.T} per step (routing + experts per token)"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(cfg),
+            "cpu_baseline": base,
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        out = run_ours(args, rank, world, dist)
+        if dist:
+            dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -18,6 +18,8 @@ Recipe (the same for the CUDA path and the oracle):
 
 from __future__ import annotations
 
+import concurrent.futures as cf
+import os
 from pathlib import Path
 
 import torch
@@ -39,22 +41,43 @@ def _gen(seed: int, stream: int) -> torch.Generator:
     return g
 
 
-def _normal(shape, std: float, seed: int, stream: int, dtype: torch.dtype) -> torch.Tensor:
-    """fp32 N(0, std^2) draw in row chunks, cast to ``dtype``."""
+def _normal(shape, std: float, seed: int, stream: int, dtype: torch.dtype, out=None) -> torch.Tensor:
+    """fp32 N(0, std^2) draw in row chunks, cast to ``dtype`` (written into
+    ``out`` when given)."""
     shape = tuple(int(s) for s in shape)
     rows = shape[0]
     inner = shape[1:]
-    out = torch.empty(shape, dtype=dtype)
+    if out is None:
+        out = torch.empty(shape, dtype=dtype)
     if rows == 0:
         return out
+    buf = None
     for c, r0 in enumerate(range(0, rows, _CHUNK_ROWS)):
         r1 = min(rows, r0 + _CHUNK_ROWS)
-        a = torch.randn((r1 - r0,) + inner, generator=_gen(seed, stream + c * 65536),
-                        dtype=torch.float32)
+        if buf is None or buf.shape[0] != r1 - r0:
+            buf = torch.empty((r1 - r0,) + inner, dtype=torch.float32)
+        buf.normal_(generator=_gen(seed, stream + c * 65536))
         if std != 1.0:
-            a.mul_(std)
-        out[r0:r1] = a.to(dtype)
+            buf.mul_(std)
+        out[r0:r1].copy_(buf)
     return out
+
+
+def _fill_parallel(jobs, seed: int, dt: torch.dtype) -> None:
+    """Draw independent tensors on a thread pool (each has its own stream, so
+    the values do not depend on the order or the number of threads)."""
+    def one(job):
+        dst, i, shape, std, stream = job
+        _normal(shape, std, seed, stream, dt, out=dst[i])
+
+    threads = max(1, min(len(jobs), os.cpu_count() or 1))
+    prev = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        with cf.ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, jobs))
+    finally:
+        torch.set_num_threads(prev)
 
 
 def _dt(cfg: MoEConfig) -> torch.dtype:
@@ -95,8 +118,15 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
         w["w_query"] = _normal((dq, d), d ** -0.5, seed, _WQ, dt)
         w["subkeys_row"] = _normal((cfg.pk_rows, dq // 2), 1.0, seed, _KR, dt)
         w["subkeys_col"] = _normal((cfg.pk_cols, dq // 2), 1.0, seed, _KC, dt)
-        w["u"] = _normal((cfg.n_atomic, d), 1024 ** -0.5, seed, _U, dt)
-        w["v"] = _normal((cfg.n_atomic, d), 1024 ** -0.5, seed, _V, dt)
+        w["u"] = torch.empty((cfg.n_atomic, d), dtype=dt)
+        w["v"] = torch.empty((cfg.n_atomic, d), dtype=dt)
+        # row chunks of u and v drawn in parallel (same streams as a serial draw)
+        jobs = []
+        for name, stream in (("u", _U), ("v", _V)):
+            for c, r0 in enumerate(range(0, cfg.n_atomic, _CHUNK_ROWS)):
+                r1 = min(cfg.n_atomic, r0 + _CHUNK_ROWS)
+                jobs.append((w[name], slice(r0, r1), (r1 - r0, d), 1024 ** -0.5, stream + c * 65536))
+        _fill_parallel(jobs, seed, dt)
         return w
     H = cfg.hidden
     w["w_router"] = make_router_weight(cfg, seed)
@@ -105,12 +135,11 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
     wg = torch.empty((E, H, d), dtype=dt)
     wu = torch.empty((E, H, d), dtype=dt)
     wd = torch.empty((E, d, H), dtype=dt)
+    jobs = []
     for e in range(E):
         base = _EXPERT + e * 4 * 64
-        wg[e] = _normal((H, d), d ** -0.5, seed, base + 0, dt)
-        wu[e] = _normal((H, d), d ** -0.5, seed, base + 64, dt)
-        wd[e] = _normal((d, H), H ** -0.5, seed, base + 128, dt)
-    w["w_gate"], w["w_up"], w["w_down"] = wg, wu, wd
+        jobs += [(wg, e, (H, d), d ** -0.5, base + 0), (wu, e, (H, d), d ** -0.5, base + 64),
+                 (wd, e, (d, H), H ** -0.5, base + 128)]
     if cfg.n_shared:
         S, Hs = cfg.n_shared, cfg.hidden_shared
         sg = torch.empty((S, Hs, d), dtype=dt)
@@ -118,10 +147,11 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
         sd = torch.empty((S, d, Hs), dtype=dt)
         for s in range(S):
             base = _SHARED + s * 4 * 64
-            sg[s] = _normal((Hs, d), d ** -0.5, seed, base + 0, dt)
-            su[s] = _normal((Hs, d), d ** -0.5, seed, base + 64, dt)
-            sd[s] = _normal((d, Hs), Hs ** -0.5, seed, base + 128, dt)
+            jobs += [(sg, s, (Hs, d), d ** -0.5, base + 0), (su, s, (Hs, d), d ** -0.5, base + 64),
+                     (sd, s, (d, Hs), Hs ** -0.5, base + 128)]
         w["ws_gate"], w["ws_up"], w["ws_down"] = sg, su, sd
+    _fill_parallel(jobs, seed, dt)
+    w["w_gate"], w["w_up"], w["w_down"] = wg, wu, wd
     if cfg.n_const:
         w["w_const_mix"] = _normal((cfg.n_const, 2, d), d ** -0.5, seed, _WC, dt)
         w["const_vec"] = _normal((cfg.n_const, d), 1.0, seed, _CV, dt)
