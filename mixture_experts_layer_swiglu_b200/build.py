@@ -1,6 +1,8 @@
 """Builds libmoe.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m mixture_experts_layer_swiglu_b200.build [--force]
+    python mixture_experts_layer_swiglu_b200/build.py [--force]
+
+(run by path: importing the package loads the library this script builds)
 
 Each csrc/*.cu is compiled to an object with relocatable device code (the
 device status word is shared by all kernels), then nvcc links and

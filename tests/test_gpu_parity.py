@@ -27,8 +27,9 @@ def _clean_status():
 
 
 def _report(name: str, rep: dict) -> None:
-    print(f"\n{name}: margin<1e-6 {rep['below_1e-6']}, within error {len(rep['near_tie'])}, "
-          f"routing mismatches {len(rep['mismatch'])} (margins {np.round(rep['mismatch_margins'][:6], 9)}), "
+    print(f"\n{name}: margin<1e-6 {rep['below_1e-6']}, boundary within error {len(rep['near_tie'])}, "
+          f"set mismatches {len(rep['set_mismatch'])} (margins {np.round(rep['mismatch_margins'][:6], 9)}), "
+          f"order-only mismatches {len(rep['order_mismatch'])}, "
           f"fp32 result err/rms {rep['rel_err']:.3e}, dtype output err/rms {rep['rel_err_out']:.3e}"
           + (f", routed rows {rep['R']}" if "R" in rep else ""))
 
