@@ -231,6 +231,32 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
                              float* logits_out, void* workspace, size_t ws_bytes,
                              moe_stream_t stream);
 
+/*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory: for example a plugin inside a host framework that owns all device
+ * memory and offers the plugin no allocator, or a service whose device
+ * memory budget is fixed and fully committed at start-up.  (The pages have
+ * no counterpart: this is a property of the library, not of the method.)
+ * Same arguments, results and errors as moe_permute for the SwiGLU kind,
+ * minus the workspace: the per-block expert counts live in a fixed array in
+ * the library's own device memory (256 KiB, held by every GPU that loads the
+ * library until the process exits).  The call allocates nothing (no
+ * cudaMalloc / cudaFree, no allocating library routine).
+ * Limit: ceil(T / 256) * n_ffn <= 65536 (e.g. T <= 65536 with 256 experts,
+ *   T <= 2,097,152 with 8 experts); beyond it, or for the atomic kind, the
+ *   call returns MOE_ERR_UNSUPPORTED and enqueues nothing.
+ * The first call on a device looks up the array's device address (with that
+ *   device current) and may fail with MOE_ERR_CUDA; make that first call
+ *   before any stream capture.
+ * Every call on a device shares the one array and it keeps the last call's
+ *   contents (nothing needs clearing: each call overwrites every entry it
+ *   reads).  Calls whose kernels overlap on the GPU -- on two streams at once,
+ *   or from two host threads -- race on it and give wrong results; order them.
+ */
+MOE_API moe_status moe_permute_static(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x,
+                                      int32_t* expert_offsets, int32_t* row_of, int32_t* token_of,
+                                      void* x_sorted, moe_stream_t stream);
+
 /* Synchronises `stream`, returns the current device's status word in *out
  * (MOE_OK if no kernel reported an error) and clears it if reset != 0. */
 MOE_API moe_status moe_get_device_status(moe_status* out, int reset, moe_stream_t stream);

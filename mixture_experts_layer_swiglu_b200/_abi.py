@@ -23,7 +23,7 @@ MOE_EXPERT_SWIGLU, MOE_EXPERT_ATOMIC_GELU = 0, 1
 EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_layer_workspace_size",
             "moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
             "moe_layer_forward", "moe_get_device_status", "moe_status_string",
-            "moe_last_launch_count")
+            "moe_last_launch_count", "moe_permute_static")
 
 
 class MoEError(RuntimeError):
@@ -64,6 +64,7 @@ def load(path: Path | str | None = None):
         getattr(L, name).restype = I64
     L.moe_route.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_permute.argtypes = [D, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_permute_static.argtypes = [D, VP, VP, VP, VP, VP, VP, VP]
     L.moe_grouped_ffn.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_grouped_ffn_phase.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, SZ, VP]
     L.moe_combine.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, VP, VP]
@@ -73,7 +74,7 @@ def load(path: Path | str | None = None):
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_launch_count.restype = I32
     for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
-                 "moe_layer_forward", "moe_get_device_status"):
+                 "moe_layer_forward", "moe_get_device_status", "moe_permute_static"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -152,6 +153,13 @@ def moe_permute(desc, topk_idx, x, expert_offsets, row_of, token_of, x_sorted, w
     _check("moe_permute", load().moe_permute(ctypes.byref(desc), _p(topk_idx), _p(x), _p(expert_offsets),
                                              _p(row_of), _p(token_of), _p(x_sorted), _p(workspace),
                                              _nbytes(workspace), _stream(stream)))
+
+
+def moe_permute_static(desc, topk_idx, x, expert_offsets, row_of, token_of, x_sorted, stream=None) -> None:
+    """moe_permute without a workspace (its scratch is a fixed array inside the library)."""
+    _check("moe_permute_static", load().moe_permute_static(ctypes.byref(desc), _p(topk_idx), _p(x),
+                                                           _p(expert_offsets), _p(row_of), _p(token_of),
+                                                           _p(x_sorted), _stream(stream)))
 
 
 def moe_grouped_ffn(desc, weights, x_sorted, expert_offsets, token_of, x, topk_gate, y_sorted, workspace,

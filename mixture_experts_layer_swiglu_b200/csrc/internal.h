@@ -14,6 +14,7 @@ inline void count_launch(int n = 1) { t_launches += n; }
 
 moe_status cuda_status(cudaError_t e);
 int num_sms();
+moe_status validate_desc(const moe_layer_desc* d);   // the descriptor checks of every entry point
 
 // ------------------------------------------------------------ grouped GEMM
 enum EpiKind { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_F32 = 2, EPI_PK_SPLIT = 3 };

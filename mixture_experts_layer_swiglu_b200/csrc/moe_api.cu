@@ -422,6 +422,9 @@ moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, con
 }
 
 }  // namespace
+
+moe_status validate_desc(const moe_layer_desc* d) { return check_desc(d); }
+
 }  // namespace moe
 
 using namespace moe;
