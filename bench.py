@@ -52,12 +52,15 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
     p.add_argument("--experts", type=int, default=0, help="override the expert count (profiling)")
+    p.add_argument("--workload", default=WORKLOAD,
+                   help="tiny_f32 | mixtral | longtail | moepp | atomic (default: the Mixtral-shaped layer)")
+    p.add_argument("--no-library-ref", action="store_true", help="skip the cuBLAS same-shape reference")
     return p.parse_args()
 
 
 def bench_config(args):
     from moe_workloads import scaled
-    cfg = get_config(WORKLOAD)
+    cfg = get_config(args.workload)
     ch = {}
     if args.tokens:
         ch["T"] = args.tokens
@@ -67,10 +70,21 @@ def bench_config(args):
 
 
 def workload_config(cfg) -> dict:
-    return {"workload": f"{cfg.name}_T{cfg.T}_d{cfg.d}_E{cfg.n_ffn}_H{cfg.hidden}_k{cfg.top_k}",
-            "T_per_gpu": cfg.T, "d_model": cfg.d, "experts": cfg.n_ffn, "hidden": cfg.hidden,
-            "top_k": cfg.top_k, "router": "softmax over top-k", "parallelism": "token-sharded replicas",
-            "l2": "flushed between steps (256 MiB write outside the step events)"}
+    if cfg.kind == "atomic":
+        name = f"{cfg.name}_T{cfg.T}_d{cfg.d}_N{cfg.pk_rows}x{cfg.pk_cols}_K{cfg.top_k}_half{cfg.pk_topk_half}"
+        shape = {"experts": cfg.n_atomic, "d_query": cfg.d_query, "router": "Cartesian product, top-K of top-half^2"}
+    else:
+        name = f"{cfg.name}_T{cfg.T}_d{cfg.d}_E{cfg.n_ffn}_H{cfg.hidden}_k{cfg.top_k}"
+        if cfg.n_shared:
+            name += f"_S{cfg.n_shared}"
+        if cfg.n_zero + cfg.n_copy + cfg.n_const:
+            name += f"_zc{cfg.n_zero + cfg.n_copy + cfg.n_const}"
+        shape = {"experts": cfg.n_ffn, "hidden": cfg.hidden, "shared": cfg.n_shared,
+                 "zero_copy_const": [cfg.n_zero, cfg.n_copy, cfg.n_const], "router": "softmax over top-k"}
+    return {"workload": name, "T_per_gpu": cfg.T, "d_model": cfg.d, "top_k": cfg.top_k, **shape,
+            "parallelism": "token-sharded replicas",
+            "l2": "flushed between steps (256 MiB write outside the step events)",
+            "timing": "CUDA events around each step; the step is fully queued before its first event"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -132,6 +146,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------- CPU oracle
 
+def oracle_sample(cfg, inp, toks) -> None:
+    """The whole layer for the listed tokens with the fp64 oracle."""
+    import oracle
+    if cfg.kind == "atomic":
+        xs = inp["x"][torch.from_numpy(toks).long()]
+        sr, sc = oracle.pk_scores(xs, inp["w_query"], inp["subkeys_row"], inp["subkeys_col"])
+        idx, gate, _ = oracle.pk_select(sr, sc, cfg.pk_topk_half, cfg.top_k)
+        oracle.atomic_tokens(inp["x"], inp["u"], inp["v"], toks, idx, gate)
+    else:
+        oracle.moe_tokens(cfg, inp, toks)
+
+
 def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
     """The fp64 oracle as it stands on a bounded sample of the workload's
     tokens (routing + experts of each token), on all host cores."""
@@ -139,14 +165,18 @@ def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
 
     import oracle
     threads = oracle.num_threads()
+
+    def run(toks):
+        oracle_sample(cfg, inp, toks)
+
     if n_tokens <= 0:   # size the sample: time a small probe first
         t0 = time.perf_counter()
-        oracle.moe_tokens(cfg, inp, np.arange(threads, dtype=np.int32))
+        run(np.arange(threads, dtype=np.int32))
         per_tok = (time.perf_counter() - t0) / threads
         n_tokens = int(max(threads, min(cfg.T, seconds / max(per_tok, 1e-6))))
     toks = np.linspace(0, cfg.T - 1, n_tokens).astype(np.int32)
     t0 = time.perf_counter()
-    oracle.moe_tokens(cfg, inp, toks)
+    run(toks)
     el = time.perf_counter() - t0
     return {"value": n_tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{n_tokens} of the {cfg.T} tokens (evenly spaced), full routing + experts per token, "
@@ -154,6 +184,38 @@ def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
 
 
 # ------------------------------------------------------------------- ours
+
+def stage_names(cfg) -> list:
+    if cfg.kind == "atomic":
+        return ["router", "permute", "expert_dot", "expert_combine"]
+    return ["router", "permute", "gate_up_gemm", "down_gemm", "combine"]
+
+
+def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
+    """Algorithmic work of each stage: ("tensor", FLOPs) or ("hbm", bytes)."""
+    d, T, k, e = cfg.d, cfg.T, cfg.top_k, cfg.elt_bytes
+    if cfg.kind == "atomic":
+        dq, N = cfg.d_query, cfg.n_atomic
+        return {
+            "router": ("tensor", 2.0 * T * d * dq + 2.0 * (2 * T) * (1.5 * dq) * cfg.pk_rows),
+            "permute": ("hbm", T * k * 4 * 6 + N * 4 * 5),
+            "expert_dot": ("hbm", touched * d * e + T * k * 12),
+            "expert_combine": ("hbm", T * k * d * e + T * k * 8 + T * d * e),
+        }
+    H = cfg.hidden
+    E_r = cfg.n_routed
+    router = T * d * e + (E_r + 2 * cfg.n_const) * d * e + T * k * 8 + T * cfg.n_const * 8
+    if cfg.gating_residual:
+        router += T * E_r * 4
+    zc_x = T * d * e if (cfg.n_copy + cfg.n_const) else 0
+    return {
+        "router": ("hbm", router),
+        "permute": ("hbm", T * d * e + R_total * d * e + T * k * 12),
+        "gate_up_gemm": ("tensor", 4.0 * R_total * d * H),
+        "down_gemm": ("tensor", 2.0 * R_total * d * H),
+        "combine": ("hbm", R_total * d * 4 + T * d * e + zc_x + T * k * 12),
+    }
+
 
 def run_ours(args, rank: int, world: int, dist) -> dict | None:
     import mixture_experts_layer_swiglu_b200 as moe
@@ -165,31 +227,44 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     a_cpu = make_activations(cfg, seed=rank)           # each rank its own tokens
     w = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in w_cpu.items()}
     x = a_cpu["x"].to(dev)
+    zp = a_cpu["z_prev"].to(dev) if "z_prev" in a_cpu else None
     desc = moe.desc_from(cfg)
     ws = moe.weights_struct(w)
     b = moe.StageBuffers(desc, device=dev)
+    cm = b.const_mix if cfg.n_const else None
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    atomic = cfg.kind == "atomic"
+
+    def calls():
+        c = [lambda: moe.moe_route(desc, ws, x, zp, None, b.idx, b.gate, cm, b.workspace, stream),
+             lambda: moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace,
+                                     stream)]
+        if atomic:
+            c.append(lambda: moe.moe_grouped_ffn(desc, ws, None, b.offsets, b.token_of, x, b.gate, b.y_sorted,
+                                                 b.workspace, stream))
+        else:
+            c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 1, b.x_sorted, b.offsets, b.y_sorted,
+                                                       b.workspace, stream))
+            c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 2, b.x_sorted, b.offsets, b.y_sorted,
+                                                       b.workspace, stream))
+        c.append(lambda: moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, cm, x, b.y,
+                                         stream))
+        return c
+
+    stage_calls = calls()
+    names = stage_names(cfg)
 
     def step(ev=None):
         """One pass of the hot path; events between the stages if given."""
         launches = 0
-        if ev: ev[0].record(stream)
-        moe.moe_route(desc, ws, x, None, None, b.idx, b.gate, None, b.workspace, stream)
-        launches += moe.moe_last_launch_count()
-        if ev: ev[1].record(stream)
-        moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace, stream)
-        launches += moe.moe_last_launch_count()
-        if ev: ev[2].record(stream)
-        moe.moe_grouped_ffn_phase(desc, ws, 1, b.x_sorted, b.offsets, b.y_sorted, b.workspace, stream)
-        launches += moe.moe_last_launch_count()
-        if ev: ev[3].record(stream)
-        moe.moe_grouped_ffn_phase(desc, ws, 2, b.x_sorted, b.offsets, b.y_sorted, b.workspace, stream)
-        launches += moe.moe_last_launch_count()
-        if ev: ev[4].record(stream)
-        moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, None, x, b.y, stream)
-        launches += moe.moe_last_launch_count()
-        if ev: ev[5].record(stream)
+        for j, f in enumerate(stage_calls):
+            if ev:
+                ev[j].record(stream)
+            f()
+            launches += moe.moe_last_launch_count()
+        if ev:
+            ev[len(stage_calls)].record(stream)
         return launches
 
     for _ in range(args.warmup):
@@ -199,7 +274,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    nst = len(stage_calls)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(K)]
+    # ~0.5 ms of GPU sleep after each flush, outside the events: the host has
+    # queued the whole step before the device reaches the first event, so the
+    # events time the device, not the Python launch path.
+    sleep_cycles = int(0.5e-3 * torch.cuda.get_device_properties(dev).clock_rate * 1e3)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -207,17 +287,19 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     with ClockSampler(dev.index) as clk:
         for i in range(K):
             flush.zero_()
+            torch.cuda._sleep(sleep_cycles)
             launches += step(evs[i])
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
     status = moe.moe_get_device_status(reset=True)
     assert status == moe.MOE_OK, moe.status_string(status)
-    names = ["router", "permute", "gate_up_gemm", "down_gemm", "combine"]
     per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)] for j, n in enumerate(names)}
-    step_ms = [evs[i][0].elapsed_time(evs[i][5]) for i in range(K)]
-    total_ms = sum(step_ms)
-    R = int(b.offsets[-1].item())
+    total_ms = sum(evs[i][0].elapsed_time(evs[i][nst]) for i in range(K))
+    off = b.offsets.cpu()
+    R_total = int(off[-1].item())
+    R_ffn = int(off[cfg.n_ffn].item()) if not atomic else R_total
+    touched = int((off[1:] > off[:-1]).sum().item()) if atomic else 0
 
     # end to end through the public call with host buffers
     x_host = a_cpu["x"].pin_memory()
@@ -227,7 +309,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     y_dev = torch.empty_like(x)
     for _ in range(2):
         x_dev.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev, y=y_dev)
+        layer.forward(x_dev, prev_logits=zp, y=y_dev)
         y_host.copy_(y_dev, non_blocking=True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -235,9 +317,10 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     e2e_ms = 0.0
     for _ in range(KE):
         flush.zero_()
+        torch.cuda._sleep(sleep_cycles)
         e0.record(stream)
         x_dev.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev, y=y_dev)
+        layer.forward(x_dev, prev_logits=zp, y=y_dev)
         y_host.copy_(y_dev, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -245,9 +328,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
 
+    cublas = None
+    if not atomic and cfg.dtype == "bf16" and rank == 0 and not args.no_library_ref:
+        cublas = library_reference(cfg, R_total, dev)
+
     mean = {n: sum(v) / K for n, v in per.items()}
-    res = {"total_ms": total_ms, "e2e_ms": e2e_ms / KE, "mean": mean, "R": R, "launches": launches,
-           "clocks": clk.summary(), "T": cfg.T}
+    res = {"total_ms": total_ms, "e2e_ms": e2e_ms / KE, "mean": mean}
     if dist:   # max over ranks
         t = torch.tensor([total_ms, res["e2e_ms"]] + [mean[n] for n in names], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -261,54 +347,95 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     if pk.exists():
         peaks = json.loads(pk.read_text())
     peak_tf = peaks.get("bf16_tflops")
-    peak_src = "measured burst (MEASURED_PEAKS.json)" if peak_tf else "fallback"
+    peak_tf_sus = peaks.get("bf16_tflops_sustained")
+    peak_src = "of measured (MEASURED_PEAKS.json, burst)" if peak_tf else "of fallback"
     if not peak_tf:
         peak_tf = 1590.0
-    hbm = peaks.get("hbm_gbs") or 6650.0
-    d, H = cfg.d, cfg.hidden
-    flops_gu = 4.0 * R * d * H
-    flops_dn = 2.0 * R * d * H
-    gu_s = res["mean"]["gate_up_gemm"] / 1e3
-    achieved = flops_gu / gu_s / 1e12
-    traffic = _ncu_traffic("gate_up_gemm", WORKLOAD)
+    hbm = peaks.get("hbm_gbs")
+    hbm_src = "of measured (MEASURED_PEAKS.json)" if hbm else "of fallback"
+    hbm = hbm or 6650.0
+    work = work_model(cfg, R_total, R_ffn, touched)
     ms_step = res["total_ms"] / K
     value = world * cfg.T / (ms_step / 1e3)
     kern = {}
     for n in names:
         ms = res["mean"][n]
+        unit, amount = work[n]
         kern[n] = {"ms": round(ms, 4), "share": round(ms / ms_step, 4)}
-    kern["gate_up_gemm"]["tflops"] = round(flops_gu / (res["mean"]["gate_up_gemm"] / 1e3) / 1e12, 1)
-    kern["down_gemm"]["tflops"] = round(flops_dn / (res["mean"]["down_gemm"] / 1e3) / 1e12, 1)
-    e = cfg.elt_bytes
-    Tk = cfg.T * cfg.top_k
-    router_bytes = cfg.T * d * e + cfg.n_routed * d * e + Tk * 8
-    permute_bytes = cfg.T * d * e + R * d * e + Tk * 12
-    combine_bytes = R * d * 4 + cfg.T * d * e + Tk * 12
-    for n, by in (("router", router_bytes), ("permute", permute_bytes), ("combine", combine_bytes)):
-        kern[n]["gbs"] = round(by / (res["mean"][n] / 1e3) / 1e9, 1)
-        kern[n]["hbm_frac"] = round(kern[n]["gbs"] / hbm, 3)
-    h2d = x_host.numel() * x_host.element_size()
+        if unit == "tensor":
+            kern[n]["tflops"] = round(amount / (ms / 1e3) / 1e12, 1)
+            kern[n]["tensor_frac"] = round(kern[n]["tflops"] / peak_tf, 4)
+        else:
+            kern[n]["gbs"] = round(amount / (ms / 1e3) / 1e9, 1)
+            kern[n]["hbm_frac"] = round(kern[n]["gbs"] / hbm, 4)
+    dom = max(names, key=lambda n: res["mean"][n])
+    unit, amount = work[dom]
+    dom_s = res["mean"][dom] / 1e3
+    if unit == "tensor":
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(amount / dom_s / 1e12, 1), "peak": peak_tf,
+                "unit": "TFLOP/s", "peak_source": peak_src, "flops_per_launch": amount}
+        if peak_tf_sus:
+            roof["frac_of_sustained"] = round(roof["achieved"] / peak_tf_sus, 4)
+    else:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(amount / dom_s / 1e9, 1), "peak": hbm,
+                "unit": "GB/s", "peak_source": hbm_src, "bytes_per_launch": amount}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = _ncu_traffic(dom, cfg.name)
+    h2d = x_host.numel() * x_host.element_size() + (zp.numel() * 4 if zp is not None else 0)
     d2h = y_host.numel() * y_host.element_size()
+    flops = sum(a for u, a in work.values() if u == "tensor")
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights)",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights)",
         "config": workload_config(cfg),
-        "roofline": {"bound": "tensor", "kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)",
-                     "achieved": round(achieved, 1), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_tf, 4), "traffic": traffic,
-                     "peak_source": peak_src, "flops_per_launch": flops_gu},
+        "roofline": roof,
         "kernels": kern,
-        "step_tflops": round((flops_gu + flops_dn) / (ms_step / 1e3) / 1e12, 1),
+        "step_tflops": round(flops / (ms_step / 1e3) / 1e12, 1),
+        "rows": {"grouped": R_total, "ffn": R_ffn, "touched_experts": touched},
         "e2e": {"value": round(world * cfg.T / (res["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "moe_layer_forward, x from pinned host, y to pinned host"},
-        "gpu_launches": res["launches"],
-        "clocks": res["clocks"],
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
     }
+    if cublas:
+        out["library_reference"] = cublas
     if world == 1 and not args.no_cpu_baseline:
         w_cpu.update(a_cpu)
         out["cpu_baseline"] = cpu_oracle_leg(cfg, w_cpu, args.oracle_tokens)
+    return out
+
+
+def library_reference(cfg, R_total: int, dev) -> dict:
+    """cuBLAS (torch.bmm) on the same GEMM shapes with the rows split evenly
+    over the experts: context for the grouped tcgen05 GEMMs, not part of the
+    timed step."""
+    E = cfg.n_ffn + cfg.n_shared
+    m = max(1, R_total // max(E, 1))
+    d, H = cfg.d, cfg.hidden
+    g = torch.Generator(device=dev).manual_seed(1)
+    A = torch.randn((E, m, d), device=dev, generator=g).to(torch.bfloat16)
+    B = torch.randn((E, d, 2 * H), device=dev, generator=g).to(torch.bfloat16)
+    Hh = torch.randn((E, m, H), device=dev, generator=g).to(torch.bfloat16)
+    D = torch.randn((E, H, d), device=dev, generator=g).to(torch.bfloat16)
+    out = {}
+    for name, a, bm, fl in (("gate_up_bmm", A, B, 2.0 * E * m * d * 2 * H), ("down_bmm", Hh, D, 2.0 * E * m * H * d)):
+        for _ in range(3):
+            torch.bmm(a, bm)
+        ts = []
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.bmm(a, bm)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        out[name] = {"ms": round(ms, 4), "tflops": round(fl / (ms / 1e3) / 1e12, 1),
+                     "shape": f"{E} x [{m}, {a.shape[2]}] @ [{bm.shape[1]}, {bm.shape[2]}]"}
+    del A, B, Hh, D
+    torch.cuda.empty_cache()
     return out
 
 
@@ -343,10 +470,10 @@ def run_reference(args, rank: int, world: int) -> dict | None:
     n = args.oracle_tokens or max(8, oracle.num_threads())
     rng = np.random.default_rng(0)
     for _ in range(min(args.warmup, 1)):
-        oracle.moe_tokens(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
+        oracle_sample(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.moe_tokens(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
+        oracle_sample(cfg, inp, rng.choice(cfg.T, n, replace=False).astype(np.int32))
     el = time.perf_counter() - t0
     value = n * args.steps / el
     base = {"value": round(value, 3), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",

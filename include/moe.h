@@ -257,6 +257,15 @@ MOE_API moe_status moe_permute_static(const moe_layer_desc* desc, const int32_t*
                                       int32_t* expert_offsets, int32_t* row_of, int32_t* token_of,
                                       void* x_sorted, moe_stream_t stream);
 
+/*
+ * Self-test of the kernels' bounded waits (no counterpart on the pages): a
+ * one-thread kernel waits on an mbarrier that nothing arrives on, giving up
+ * after limit_ns nanoseconds (0 < limit_ns <= 2e9) the way every wait in the
+ * library does -- it writes 0 to *waited_ok (device int) and records
+ * MOE_ERR_TIMEOUT in the status word, and the CUDA context stays usable.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(uint64_t limit_ns, int32_t* waited_ok, moe_stream_t stream);
+
 /* Synchronises `stream`, returns the current device's status word in *out
  * (MOE_OK if no kernel reported an error) and clears it if reset != 0. */
 MOE_API moe_status moe_get_device_status(moe_status* out, int reset, moe_stream_t stream);

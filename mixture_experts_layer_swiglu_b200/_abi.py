@@ -23,7 +23,7 @@ MOE_EXPERT_SWIGLU, MOE_EXPERT_ATOMIC_GELU = 0, 1
 EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_layer_workspace_size",
             "moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
             "moe_layer_forward", "moe_get_device_status", "moe_status_string",
-            "moe_last_launch_count", "moe_permute_static")
+            "moe_last_launch_count", "moe_permute_static", "moe_selftest_wait_timeout")
 
 
 class MoEError(RuntimeError):
@@ -65,6 +65,7 @@ def load(path: Path | str | None = None):
     L.moe_route.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_permute.argtypes = [D, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_permute_static.argtypes = [D, VP, VP, VP, VP, VP, VP, VP]
+    L.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, VP, VP]
     L.moe_grouped_ffn.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_grouped_ffn_phase.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, SZ, VP]
     L.moe_combine.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, VP, VP]
@@ -74,7 +75,8 @@ def load(path: Path | str | None = None):
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_launch_count.restype = I32
     for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
-                 "moe_layer_forward", "moe_get_device_status", "moe_permute_static"):
+                 "moe_layer_forward", "moe_get_device_status", "moe_permute_static",
+                 "moe_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -200,6 +202,12 @@ def moe_get_device_status(reset: bool = True, stream=None) -> int:
     _check("moe_get_device_status", load().moe_get_device_status(ctypes.byref(out), int(bool(reset)),
                                                                  _stream(stream)))
     return int(out.value)
+
+
+def moe_selftest_wait_timeout(limit_ns: int, waited_ok, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (see include/moe.h)."""
+    _check("moe_selftest_wait_timeout", load().moe_selftest_wait_timeout(int(limit_ns), _p(waited_ok),
+                                                                         _stream(stream)))
 
 
 def moe_last_launch_count() -> int:

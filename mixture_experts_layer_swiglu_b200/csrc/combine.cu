@@ -6,9 +6,9 @@
 // summary, "Approach": zero expert = discard, copy expert = identity,
 // constant expert = trainable vector mixed with the input):
 //   y_t = sum_s y_sorted[shared row of t] + sum_j g_tj O_tj
-// accumulated in fp32 in slot order and rounded once.  One warp per token,
-// 16-byte vector loads of the rows (HBM-bound: reads the k expert rows and,
-// for copy/constant experts, x; writes y).
+// accumulated in fp32 in slot order and rounded once.  Four warps per token,
+// each a quarter of the row, 16- and 32-byte vector loads (HBM-bound: reads
+// the k expert rows and, for copy/constant experts, x; writes y).
 //
 // Atomic experts ("OmniMoE" 2.1 Atomic Experts E_i(x) = sigma(x . u_i) v_i,
 // Dynamic Expert Assembly; 2.2 Expert-Centric Scheduling):
@@ -89,21 +89,30 @@ __device__ __forceinline__ void store8(void* p, long long i8, const float (&v)[8
     }
 }
 
+// One token per group of CMB_SPLIT warps, each warp a contiguous quarter of
+// the row (more rows in flight per SM than one warp per token).
+constexpr int CMB_SPLIT = 4;
+
 template <typename T, typename TO>
-__global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a)
+__global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
 {
     constexpr int V = 8;
-    const int lane = threadIdx.x & 31;
+    constexpr int WPB = 256 / 32;                    // warps per block
+    constexpr int TPB = WPB / CMB_SPLIT;             // tokens per block
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int tib = wib / CMB_SPLIT, part = wib % CMB_SPLIT;
     const int vecs = a.d / V;
+    const int per = cdiv(vecs, CMB_SPLIT);
+    const int i0 = part * per, i1 = min(vecs, i0 + per);
     const int zero0 = a.n_ffn, copy0 = zero0 + a.n_zero, const0 = copy0 + a.n_copy;
     const int n_ids = const0 + a.n_const;
-    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-    __shared__ int s_e[8][CMB_MAXK], s_r[8][CMB_MAXK];
-    __shared__ float s_g[8][CMB_MAXK], s_a1[8][CMB_MAXK], s_a2[8][CMB_MAXK];
-    const int wib = threadIdx.x >> 5;
-    for (long long t = blockIdx.x * (long long)(blockDim.x >> 5) + wib; t < a.T; t += nw) {
-        // slot j's id, gate, row and constant mix, staged by lane j
-        if (lane < a.k) {
+    __shared__ int s_e[TPB][CMB_MAXK], s_r[TPB][CMB_MAXK];
+    __shared__ float s_g[TPB][CMB_MAXK], s_a1[TPB][CMB_MAXK], s_a2[TPB][CMB_MAXK];
+    for (long long base = (long long)blockIdx.x * TPB; base < a.T; base += (long long)gridDim.x * TPB) {
+        const long long t = base + tib;
+        const bool live = t < a.T;
+        // slot j's id, gate, row and constant mix, staged by lane j of part 0
+        if (live && part == 0 && lane < a.k) {
             int e = a.idx[t * a.k + lane];
             const int r = a.row_of[t * a.k + lane];
             bool bad = e < 0 || e >= n_ids;
@@ -115,56 +124,80 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a)
                 a1 = a.const_mix[(t * a.n_const + c) * 2 + 0];
                 a2 = a.const_mix[(t * a.n_const + c) * 2 + 1];
             }
-            s_e[wib][lane] = e;
-            s_r[wib][lane] = r;
-            s_g[wib][lane] = a.gate[t * a.k + lane];
-            s_a1[wib][lane] = a1;
-            s_a2[wib][lane] = a2;
+            s_e[tib][lane] = e;
+            s_r[tib][lane] = r;
+            s_g[tib][lane] = a.gate[t * a.k + lane];
+            s_a1[tib][lane] = a1;
+            s_a2[tib][lane] = a2;
         }
-        __syncwarp();
-        for (int i = lane; i < vecs; i += 32) {
-            float acc[V];
+        __syncthreads();
+        if (live) {
+            // two chunks per lane and step: their row loads are independent
+            for (int i = i0 + lane; i < i1; i += 64) {
+                const bool two = i + 32 < i1;
+                float acc[2][V];
 #pragma unroll
-            for (int v = 0; v < V; ++v) acc[v] = 0.f;
-            for (int s = 0; s < a.n_shared; ++s) {
-                const long long r = (long long)a.offsets[a.n_ffn + s] + t;
-                if (r < a.rows_cap) {
-                    float w[V];
-                    load8<float>(a.ys, r * vecs + i, w);
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int v = 0; v < V; ++v) acc[v] += w[v];
-                }
-            }
-            bool have_x = false;
-            float xv[V];
-            for (int j = 0; j < a.k; ++j) {
-                const int e = s_e[wib][j];
-                const float g = s_g[wib][j];
-                if (e < 0) continue;
-                if (e < zero0) {
-                    float w[V];
-                    load8<float>(a.ys, (long long)s_r[wib][j] * vecs + i, w);
+                    for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
+                for (int s = 0; s < a.n_shared; ++s) {
+                    const long long r = (long long)a.offsets[a.n_ffn + s] + t;
+                    if (r < a.rows_cap) {
+                        float w[2][V];
+                        load8<float>(a.ys, r * vecs + i, w[0]);
+                        if (two) load8<float>(a.ys, r * vecs + i + 32, w[1]);
 #pragma unroll
-                    for (int v = 0; v < V; ++v) acc[v] = fmaf(g, w[v], acc[v]);
-                } else if (e < copy0) {
-                    // zero expert: contributes nothing
-                } else {
-                    if (!have_x) { load8<T>(a.x, t * vecs + i, xv); have_x = true; }
-                    if (e < const0) {
+                        for (int u = 0; u < 2; ++u)
 #pragma unroll
-                        for (int v = 0; v < V; ++v) acc[v] = fmaf(g, xv[v], acc[v]);
-                    } else {
-                        const float a1 = s_a1[wib][j], a2 = s_a2[wib][j];
-                        float cv[V];
-                        load8<T>(a.const_vec, (long long)(e - const0) * vecs + i, cv);
-#pragma unroll
-                        for (int v = 0; v < V; ++v) acc[v] = fmaf(g, a1 * xv[v] + a2 * cv[v], acc[v]);
+                            for (int v = 0; v < V; ++v) acc[u][v] += w[u][v];
                     }
                 }
+                bool have_x = false;
+                float xv[2][V];
+                for (int j = 0; j < a.k; ++j) {
+                    const int e = s_e[tib][j];
+                    const float g = s_g[tib][j];
+                    if (e < 0) continue;
+                    if (e < zero0) {
+                        const long long rb = (long long)s_r[tib][j] * vecs;
+                        float w[2][V];
+                        load8<float>(a.ys, rb + i, w[0]);
+                        if (two) load8<float>(a.ys, rb + i + 32, w[1]);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u)
+#pragma unroll
+                            for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, w[u][v], acc[u][v]);
+                    } else if (e < copy0) {
+                        // zero expert: contributes nothing
+                    } else {
+                        if (!have_x) {
+                            load8<T>(a.x, t * vecs + i, xv[0]);
+                            if (two) load8<T>(a.x, t * vecs + i + 32, xv[1]);
+                            have_x = true;
+                        }
+                        if (e < const0) {
+#pragma unroll
+                            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, xv[u][v], acc[u][v]);
+                        } else {
+                            const float a1 = s_a1[tib][j], a2 = s_a2[tib][j];
+                            const long long cb = (long long)(e - const0) * vecs;
+                            float cv[2][V];
+                            load8<T>(a.const_vec, cb + i, cv[0]);
+                            if (two) load8<T>(a.const_vec, cb + i + 32, cv[1]);
+#pragma unroll
+                            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, a1 * xv[u][v] + a2 * cv[u][v], acc[u][v]);
+                        }
+                    }
+                }
+                store8<TO>(a.y, t * vecs + i, acc[0]);
+                if (two) store8<TO>(a.y, t * vecs + i + 32, acc[1]);
             }
-            store8<TO>(a.y, t * vecs + i, acc);
         }
-        __syncwarp();
+        __syncthreads();
     }
 }
 
@@ -296,7 +329,7 @@ moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
     if (a.k > CMB_MAXK) return MOE_ERR_UNSUPPORTED;
-    const int grid = std::max(1, std::min(cdiv(a.T, 8), num_sms() * 16));
+    const int grid = std::max(1, std::min(cdiv(a.T, 256 / 32 / CMB_SPLIT), num_sms() * 16));
     if (dtype == MOE_BF16 && !a.out_f32) combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else if (dtype == MOE_BF16) combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(a);
     else combine_kernel<float, float><<<grid, 256, 0, st>>>(a);

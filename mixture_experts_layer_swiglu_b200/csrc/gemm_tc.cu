@@ -62,6 +62,7 @@ struct TileInfo {
     int n;        // n-tile index inside the group
 };
 
+template <int TBM = BM>
 __device__ __forceinline__ TileInfo decode_tile(int tile, const int* tile_start, const int* g_lo,
                                                 const int* g_cnt, int n_groups)
 {
@@ -73,12 +74,12 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* tile_start,
     TileInfo ti;
     ti.g = lo;
     const int cnt = g_cnt[lo];
-    const int mt = cdiv(cnt, BM);
+    const int mt = cdiv(cnt, TBM);
     const int local = tile - tile_start[lo];
     const int m = local % mt;       // m-tiles of a group are adjacent: they share B
     ti.n = local / mt;
-    ti.row0 = g_lo[lo] + m * BM;
-    ti.rows = min(BM, cnt - m * BM);
+    ti.row0 = g_lo[lo] + m * TBM;
+    ti.rows = min(TBM, cnt - m * TBM);
     return ti;
 }
 
@@ -187,6 +188,40 @@ __device__ __forceinline__ void epilogue_tile(const DevArgs& a, uint32_t tacc, c
     }
 }
 
+// Warp 0 builds, for every group, its first row, its row count and the index
+// of its first output tile (tiles of TBM rows x one n-tile).
+template <int TBM>
+__device__ __forceinline__ void build_group_table(const DevArgs& a, int ntn, int lane, int* tile_start,
+                                                  int* g_lo, int* g_cnt)
+{
+    const int n = a.n_groups;
+    const int chunk = cdiv(n, 32);
+    const int g0 = min(n, lane * chunk), g1 = min(n, g0 + chunk);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+        int lo, hi;
+        if (a.offsets) { lo = a.offsets[g]; hi = a.offsets[g + 1]; }
+        else { lo = g * a.group_rows; hi = lo + a.group_rows; }
+        int cnt = hi - lo;
+        if (cnt < 0 || lo < 0) { set_status(MOE_ERR_DEVICE_BOUNDS); cnt = 0; lo = 0; }
+        g_lo[g] = lo;
+        g_cnt[g] = cnt;
+        local += cdiv(cnt, TBM) * ntn;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+        tile_start[g] = run;
+        run += cdiv(g_cnt[g], TBM) * ntn;
+    }
+    if (lane == 31) tile_start[n] = incl;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NTHREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -212,35 +247,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int lane = threadIdx.x & 31;
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(a.N, 128) : cdiv(a.N, 256);
 
-    // ---- group table: first row, row count and first tile of every group
-    if (warp == 0) {
-        const int n = a.n_groups;
-        const int chunk = cdiv(n, 32);
-        const int g0 = min(n, lane * chunk), g1 = min(n, g0 + chunk);
-        int local = 0;
-        for (int g = g0; g < g1; ++g) {
-            int lo, hi;
-            if (a.offsets) { lo = a.offsets[g]; hi = a.offsets[g + 1]; }
-            else { lo = g * a.group_rows; hi = lo + a.group_rows; }
-            int cnt = hi - lo;
-            if (cnt < 0 || lo < 0) { set_status(MOE_ERR_DEVICE_BOUNDS); cnt = 0; lo = 0; }
-            g_lo[g] = lo;
-            g_cnt[g] = cnt;
-            local += cdiv(cnt, BM) * ntn;
-        }
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - local;
-        for (int g = g0; g < g1; ++g) {
-            tile_start[g] = run;
-            run += cdiv(g_cnt[g], BM) * ntn;
-        }
-        if (lane == 31) tile_start[n] = incl;
-    }
+    if (warp == 0) build_group_table<BM>(a, ntn, lane, tile_start, g_lo, g_cnt);
     if (threadIdx.x == 32) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 128); }
@@ -353,6 +360,187 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 }
 
+// ------------------------------------------------------------ CTA-pair kernel
+//
+// Same schedule and epilogues, but each output tile is 256 rows x 256 columns
+// computed by a cluster of two CTAs on two SMs with tcgen05.mma.cta_group::2:
+// CTA r stages A rows [128 r, 128 r + 128) of the tile and half of B (SwiGLU:
+// CTA 0 the gate rows, CTA 1 the up rows; otherwise output columns
+// [128 r, 128 r + 128)), and holds accumulator rows [128 r, 128 r + 128) in
+// its own TMEM.  B is read from L2 once per pair instead of once per SM.
+// The leader CTA (rank 0) issues the MMAs; both CTAs' TMA copies complete on
+// the leader's stage barrier; the leader's commits arrive on both CTAs'
+// barriers; the peer's epilogue warps release the accumulator remotely.
+// No multicast loads.
+
+constexpr int P_BM = 256;
+#ifndef MOE_P_STAGES
+#define MOE_P_STAGES 6
+#endif
+#ifndef MOE_TMA_HINTS
+#define MOE_TMA_HINTS 0
+#endif
+constexpr int P_STAGES = MOE_P_STAGES;
+constexpr int P_TILE_A = 128 * BK * 2;       // 16 KB
+constexpr int P_TILE_B = 128 * BK * 2;       // 16 KB
+constexpr int P_STAGE_BYTES = P_TILE_A + P_TILE_B;
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + SMEM_TABLE_INTS * 4;
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                         const __grid_constant__ CUtensorMap tmB3, const DevArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + P_STAGES * P_TILE_A;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + P_STAGES * P_TILE_B);
+    uint64_t* empty = full + P_STAGES;
+    uint64_t* acc_full = empty + P_STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* mma_done = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* tile_start = reinterpret_cast<int*>(smem + P_STAGES * P_STAGE_BYTES + 256);
+    int* g_lo = tile_start + (kMaxGemmGroups + 1);
+    int* g_cnt = g_lo + kMaxGemmGroups;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int ntn = (EPI == EPI_SWIGLU) ? cdiv(a.N, 128) : cdiv(a.N, 256);
+
+    if (warp == 0) build_group_table<P_BM>(a, ntn, lane, tile_start, g_lo, g_cnt);
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) { tmem_alloc_pair(tmem_slot, TMEM_COLS); tmem_relinquish_pair(); }
+    if (threadIdx.x == 64) {
+        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB0); tma_prefetch_desc(&tmB1);
+        tma_prefetch_desc(&tmB2); tma_prefetch_desc(&tmB3);
+    }
+    tc_fence_before();
+    cluster_sync_all();          // both CTAs: barriers initialised, TMEM allocated
+    tc_fence_after();
+
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[a.n_groups];
+    const int nk = cdiv(a.K, BK);
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const uint32_t full_leader = mapa_shared(smem_u32(&full[0]), 0);
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // -------------------------------------------- TMA producer (both CTAs)
+            int s = 0;
+            uint32_t ph = 0;
+            bool bad = false;
+#if MOE_TMA_HINTS
+            const uint64_t pol_a = l2_policy_evict_last();
+            const uint64_t pol_b = l2_policy_evict_first();
+#endif
+            for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
+                const TileInfo ti = decode_tile<P_BM>(tile, tile_start, g_lo, g_cnt, a.n_groups);
+                const bool first = ti.g < a.n_first;
+                const int gb = first ? ti.g : ti.g - a.n_first;
+                const CUtensorMap* mb;
+                int brow;
+                if (EPI == EPI_SWIGLU) {
+                    mb = rank == 0 ? (first ? &tmB0 : &tmB2) : (first ? &tmB1 : &tmB3);
+                    brow = gb * a.N + ti.n * 128;
+                } else {
+                    mb = first ? &tmB0 : &tmB2;
+                    brow = gb * a.N + ti.n * 256 + (int)rank * 128;
+                }
+                const int arow = ti.row0 + (int)rank * 128;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
+#if MOE_TMA_HINTS
+                    // A rows (tokens) serve every n-tile of the group; each B
+                    // tile serves only the group's few m-tiles
+                    tma_load_2d_pair_hint(sA + s * P_TILE_A, &tmA, full_leader + 8 * s, kb * BK, arow, pol_a);
+                    tma_load_2d_pair_hint(sB + s * P_TILE_B, mb, full_leader + 8 * s, kb * BK, brow, pol_b);
+#else
+                    tma_load_2d_pair(sA + s * P_TILE_A, &tmA, full_leader + 8 * s, kb * BK, arow);
+                    tma_load_2d_pair(sB + s * P_TILE_B, mb, full_leader + 8 * s, kb * BK, brow);
+#endif
+                    if (++s == P_STAGES) { s = 0; ph ^= 1; }
+                }
+            }
+            if (bad) {   // copies already issued land within microseconds; let them
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) { }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // -------------------------------------------- MMA issuer (leader only)
+            const uint32_t idesc = idesc_bf16_f32(P_BM, BN_MMA);
+            int s = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            bool bad = false;
+            for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
+                if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (*abort_flag || !mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * P_TILE_A));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * P_TILE_B));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    tc_commit_pair(&empty[s], 0x3);
+                    if (++s == P_STAGES) { s = 0; ph ^= 1; }
+                }
+                if (bad) break;
+                tc_commit_pair(&acc_full[acc], 0x3);
+                if (++acc == 2) { acc = 0; aph ^= 1; }
+            }
+            // every MMA issued has completed before the CTAs may leave
+            tc_commit_pair(mma_done, 0x1);
+            mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int tile = cluster; tile < total; tile += n_clusters) {
+            TileInfo ti = decode_tile<P_BM>(tile, tile_start, g_lo, g_cnt, a.n_groups);
+            ti.row0 += (int)rank * 128;
+            ti.rows = max(0, min(128, ti.rows - (int)rank * 128));
+            if (*abort_flag || !mbar_wait(&acc_full[acc], aph)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+            epilogue_tile<EPI>(a, tacc, ti, r);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8 * acc);
+            if (++acc == 2) { acc = 0; aph ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();          // all MMAs done and all TMEM reads issued in both CTAs
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -404,13 +592,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
         !make_map(&m1, b1, p.b01_rows, p.K) || !make_map(&m2, b2, r23, p.K) ||
         !make_map(&m3, b3, r23, p.K))
         return MOE_ERR_CUDA;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_status(e);
-        attr_done = true;
-    }
+    static bool attr_done = false, attr_pair_done = false;
     DevArgs a;
     a.offsets = p.offsets;
     a.n_groups = p.n_groups;
@@ -424,9 +606,28 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     a.pk_T = p.pk_T;
     a.pk_dq = p.pk_dq;
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
-    const long long tiles_ub = (long long)(cdiv((int)std::min<long long>(p.rows_cap, 1ll << 30), BM) + p.n_groups) * ntn;
-    const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms()));
-    grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+    const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
+    if (p.pair) {
+        if (!attr_pair_done) {
+            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            if (e != cudaSuccess) return cuda_status(e);
+            attr_pair_done = true;
+        }
+        const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
+        const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
+        grouped_gemm_pair_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+    } else {
+        if (!attr_done) {
+            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            if (e != cudaSuccess) return cuda_status(e);
+            attr_done = true;
+        }
+        const long long tiles_ub = (long long)(cdiv((int)rows, BM) + p.n_groups) * ntn;
+        const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms()));
+        grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+    }
     count_launch();
     return cuda_status(cudaGetLastError());
 }

@@ -48,6 +48,7 @@ struct GemmProblem {
     long long rows_cap;   // rows of `out` (stores beyond are dropped)
     int pk_T;             // EPI_PK_SPLIT: tokens
     int pk_dq;            // EPI_PK_SPLIT: query width
+    int pair;             // 1: 256-row tiles on CTA pairs (cta_group::2); 0: 128-row tiles per CTA
 };
 
 moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st);

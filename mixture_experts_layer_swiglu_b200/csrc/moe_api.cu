@@ -216,6 +216,7 @@ moe_status route_impl(const moe_layer_desc* d, const moe_layer_weights* w, const
     q.rows_cap = d->T;
     q.pk_T = d->T;
     q.pk_dq = d->d_query;
+    q.pair = d->T >= 512 ? 1 : 0;
     if ((s = launch_grouped_gemm(q, st)) != MOE_OK) return s;
     GemmProblem g{};
     g.epi = EPI_F32;
@@ -232,6 +233,7 @@ moe_status route_impl(const moe_layer_desc* d, const moe_layer_weights* w, const
     g.out = scores;
     g.ldo = d->pk_rows;
     g.rows_cap = 2ll * d->T;
+    g.pair = d->T >= 512 ? 1 : 0;
     if ((s = launch_grouped_gemm(g, st)) != MOE_OK) return s;
     PkSelectArgs ps;
     ps.s_row = scores;
@@ -320,6 +322,10 @@ moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, i
     g.n_groups = d->n_ffn + d->n_shared;
     g.n_first = d->n_ffn;
     g.rows_cap = cap;
+    // 256-row tiles on CTA pairs halve the B traffic per SM; with small groups
+    // their padding costs more than that saves, so they need >= 512 rows per
+    // group on average (the group sizes are only known on the device).
+    g.pair = (long long)d->T * d->top_k >= 512ll * std::max(d->n_ffn, 1) ? 1 : 0;
     if (phase == 1) {
         g.epi = EPI_SWIGLU;
         g.A = xs;

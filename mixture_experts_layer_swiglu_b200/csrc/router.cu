@@ -7,8 +7,9 @@
 //   z = W_r x + bias + prev;  top-k by descending z, ties to the lower id;
 //   gates = softmax over the selected logits.  Constant experts' mixing
 //   logits W_c x are computed in the same pass over x.
-// The pass over x is the cost (x is read once from HBM): each warp takes
-// 4 tokens, lanes split d into 16-byte vectors, 8 router rows at a time are
+// The pass over x is the cost (x is read once from HBM): tiles of 32 tokens
+// are staged in shared memory with asynchronous copies, each warp takes 4
+// tokens, lanes split d into 16-byte vectors, 8 router rows at a time are
 // accumulated in fp32 and reduced across the warp with a transposing
 // butterfly (31 shuffles for 32 sums).
 //
@@ -35,7 +36,6 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int R_TPW = 4;         // tokens per warp
-constexpr int R_WARPS = 4;       // warps per block
 constexpr int R_MAXROWS = 256;   // router rows + constant-mix rows
 
 template <typename Tin> struct VecOf;
@@ -77,59 +77,161 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi)
     return v > bv || (v == bv && i < bi);
 }
 
+// Block: 8 warps x 4 tokens = a tile of 32 tokens.  The tile's x rows are
+// staged in shared memory in chunks of 1 KiB per row with cp.async (a ring of
+// 3 chunks, ~96 KiB in flight per SM), each warp computes its 4 tokens from
+// shared memory; router rows are read through L1.  If the whole tile fits
+// in the staging buffer (d <= 2048 for bf16) it is loaded once and every
+// group of 8 router rows reuses it.
+constexpr int R_WARPS = 8;
+constexpr int R_TILE = R_WARPS * R_TPW;      // 32 tokens
+constexpr int R_CHUNK_BYTES = 1024;          // per row per chunk
+constexpr int R_STAGES = 4;
+constexpr int R_W_BYTES = 8 * 4096;          // 8 router rows of <= 4 KiB (resident tiles)
+constexpr int R_SMEM = R_STAGES * R_TILE * R_CHUNK_BYTES + 2 * R_W_BYTES + R_WARPS * R_TPW * R_MAXROWS * 4;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <typename Tin>
 __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a)
 {
     constexpr int V = VecOf<Tin>::N;
-    __shared__ float s_logit[R_WARPS][R_TPW][R_MAXROWS];
+    constexpr int CE = R_CHUNK_BYTES / sizeof(Tin);          // elements per row per chunk
+    extern __shared__ __align__(16) uint8_t r_smem[];
+    uint8_t* xs = r_smem;                                     // [stage][32 rows][CE]
+    uint8_t* wbuf = r_smem + R_STAGES * R_TILE * R_CHUNK_BYTES;   // [2][8 rows][d] (resident tiles)
+    float (*s_logit)[R_TPW][R_MAXROWS] =
+        reinterpret_cast<float (*)[R_TPW][R_MAXROWS]>(wbuf + 2 * R_W_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = a.E_r + 2 * a.n_const;
-    const int n_tgroups = cdiv(a.T, R_TPW);
+    const int n_tiles = cdiv(a.T, R_TILE);
+    const int n_chunks = cdiv(a.d, CE);
+    // whole tile fits (and 8 router rows fit a W buffer): load once
+    const bool resident = n_chunks <= R_STAGES && a.d * (int)sizeof(Tin) <= R_W_BYTES / 8;
     const Tin* x = reinterpret_cast<const Tin*>(a.x);
     const Tin* wr = reinterpret_cast<const Tin*>(a.w_router);
     const Tin* wc = reinterpret_cast<const Tin*>(a.w_const_mix);
     float (*zs)[R_MAXROWS] = s_logit[warp];
 
-    for (int grp = blockIdx.x * R_WARPS + warp; grp < n_tgroups; grp += gridDim.x * R_WARPS) {
-        const int t0 = grp * R_TPW;
-        for (int rc = 0; rc < R; rc += 8) {
-            float acc[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-            for (int i = lane * V; i < a.d; i += 32 * V) {
-                float xv[R_TPW][V];
-#pragma unroll
-                for (int tt = 0; tt < R_TPW; ++tt) {
-                    if (t0 + tt < a.T) load_vec(x + (long long)(t0 + tt) * a.d + i, xv[tt]);
-                    else {
-#pragma unroll
-                        for (int v = 0; v < V; ++v) xv[tt][v] = 0.f;
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int r = rc + q;
-                    if (r < R) {
-                        const Tin* wrow = r < a.E_r ? wr + (long long)r * a.d
-                                                    : wc + (long long)(r - a.E_r) * a.d;
-                        float wv[V];
-                        load_vec(wrow + i, wv);
-#pragma unroll
-                        for (int tt = 0; tt < R_TPW; ++tt)
-#pragma unroll
-                            for (int v = 0; v < V; ++v)
-                                acc[tt * 8 + q] = fmaf(xv[tt][v], wv[v], acc[tt * 8 + q]);
-                    }
-                }
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int t_tile = tile * R_TILE;
+        // copy chunk c of the tile's 32 rows into stage st (rows past T repeat row T-1)
+        auto issue = [&](int c, int st) {
+            const int e0 = c * CE;
+            const int vec_per_row = min(CE, a.d - e0) / V;
+            for (int q = threadIdx.x; q < R_TILE * vec_per_row; q += blockDim.x) {
+                const int row = q / vec_per_row, vi = q % vec_per_row;
+                const long long t = min(t_tile + row, a.T - 1);
+                cp_async16(xs + ((size_t)st * R_TILE + row) * R_CHUNK_BYTES + vi * 16,
+                           x + t * a.d + e0 + (long long)vi * V);
             }
-            const float s = transpose_reduce32(acc, lane);
-            const int r = rc + (lane & 7);
-            if (r < R) zs[lane >> 3][r] = s;
+        };
+        // 8 router rows (rows past R repeat row R-1) into W buffer wb
+        const int row_bytes = a.d * (int)sizeof(Tin);
+        auto issue_w = [&](int rc, int wb) {
+            const int vec_per_row = a.d / V;
+            for (int q = threadIdx.x; q < 8 * vec_per_row; q += blockDim.x) {
+                const int qr = q / vec_per_row, vi = q % vec_per_row;
+                const int r = min(rc + qr, R - 1);
+                const Tin* wrow = r < a.E_r ? wr + (long long)r * a.d : wc + (long long)(r - a.E_r) * a.d;
+                cp_async16(wbuf + (size_t)wb * R_W_BYTES + (size_t)qr * row_bytes + vi * 16, wrow + (long long)vi * V);
+            }
+        };
+        const int passes = resident ? 1 : cdiv(R, 8);
+        for (int pass = 0; pass < passes; ++pass) {
+            __syncthreads();                                  // stage buffers free
+            const int npro = min(R_STAGES - 1, n_chunks);
+            for (int c = 0; c < (resident ? n_chunks : npro); ++c) { issue(c, c); cp_async_commit(); }
+            if (resident) { issue_w(0, 0); cp_async_commit(); }
+            const int rc_lo = resident ? 0 : pass * 8, rc_hi = resident ? R : min(R, pass * 8 + 8);
+            for (int rc = rc_lo; rc < rc_hi; rc += 8) {
+                float acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                const int wb = (rc / 8) & 1;
+                if (resident) {
+                    // next 8 rows in flight while these compute; x tile and
+                    // this W buffer complete
+                    if (rc + 8 < rc_hi) { issue_w(rc + 8, wb ^ 1); cp_async_commit(); cp_async_wait<1>(); }
+                    else cp_async_wait<0>();
+                    __syncthreads();
+                }
+                for (int c = 0; c < n_chunks; ++c) {
+                    const int st = resident ? c : c % R_STAGES;
+                    if (!resident) {
+                        if (c + R_STAGES - 1 < n_chunks) cp_async_wait<R_STAGES - 2>();
+                        else cp_async_wait<0>();
+                        __syncthreads();
+                    }
+                    const int e0 = c * CE;
+                    const int ce = min(CE, a.d - e0);
+                    for (int vi = lane; vi < ce / V; vi += 32) {
+                        float xv[R_TPW][V];
+#pragma unroll
+                        for (int tt = 0; tt < R_TPW; ++tt) {
+                            const Tin* src = reinterpret_cast<const Tin*>(
+                                xs + ((size_t)st * R_TILE + warp * R_TPW + tt) * R_CHUNK_BYTES) + vi * V;
+                            if constexpr (V == 8) {
+                                const uint4 u = *reinterpret_cast<const uint4*>(src);
+                                xv[tt][0] = bf16_lo(u.x); xv[tt][1] = bf16_hi(u.x); xv[tt][2] = bf16_lo(u.y); xv[tt][3] = bf16_hi(u.y);
+                                xv[tt][4] = bf16_lo(u.z); xv[tt][5] = bf16_hi(u.z); xv[tt][6] = bf16_lo(u.w); xv[tt][7] = bf16_hi(u.w);
+                            } else {
+                                const float4 f = *reinterpret_cast<const float4*>(src);
+                                xv[tt][0] = f.x; xv[tt][1] = f.y; xv[tt][2] = f.z; xv[tt][3] = f.w;
+                            }
+                        }
+                        // all 8 router-row loads issued together: rows past R
+                        // repeat row R-1 and land in accumulators never read
+                        float wv[8][V];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (resident) {
+                                const Tin* src = reinterpret_cast<const Tin*>(
+                                    wbuf + (size_t)wb * R_W_BYTES + (size_t)q * row_bytes) + e0 + vi * V;
+                                if constexpr (V == 8) {
+                                    const uint4 u = *reinterpret_cast<const uint4*>(src);
+                                    wv[q][0] = bf16_lo(u.x); wv[q][1] = bf16_hi(u.x); wv[q][2] = bf16_lo(u.y); wv[q][3] = bf16_hi(u.y);
+                                    wv[q][4] = bf16_lo(u.z); wv[q][5] = bf16_hi(u.z); wv[q][6] = bf16_lo(u.w); wv[q][7] = bf16_hi(u.w);
+                                } else {
+                                    const float4 f = *reinterpret_cast<const float4*>(src);
+                                    wv[q][0] = f.x; wv[q][1] = f.y; wv[q][2] = f.z; wv[q][3] = f.w;
+                                }
+                            } else {
+                                const int r = min(rc + q, R - 1);
+                                const Tin* wrow = r < a.E_r ? wr + (long long)r * a.d : wc + (long long)(r - a.E_r) * a.d;
+                                load_vec(wrow + e0 + vi * V, wv[q]);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+#pragma unroll
+                            for (int tt = 0; tt < R_TPW; ++tt)
+#pragma unroll
+                                for (int v = 0; v < V; ++v)
+                                    acc[tt * 8 + q] = fmaf(xv[tt][v], wv[q][v], acc[tt * 8 + q]);
+                    }
+                    if (!resident) {
+                        __syncthreads();                      // everyone done with stage st
+                        if (c + R_STAGES - 1 < n_chunks) { issue(c + R_STAGES - 1, (c + R_STAGES - 1) % R_STAGES); }
+                        cp_async_commit();
+                    }
+                }
+                if (resident) __syncthreads();                // W buffer wb free for rc + 16
+                const float sres = transpose_reduce32(acc, lane);
+                const int r = rc + (lane & 7);
+                if (r < R) zs[lane >> 3][r] = sres;
+            }
         }
         __syncwarp();
 
         for (int tt = 0; tt < R_TPW; ++tt) {
-            const int t = t0 + tt;
+            const int t = t_tile + warp * R_TPW + tt;
             if (t >= a.T) break;
             float* z = zs[tt];
             for (int e = lane; e < a.E_r; e += 32) {
@@ -179,7 +281,6 @@ __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a
             }
             __syncwarp();
         }
-        __syncwarp();
     }
 }
 
@@ -308,10 +409,15 @@ __global__ void pk_prep_keys_kernel(const __nv_bfloat16* kr, const __nv_bfloat16
 moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
-    const int tgroups = cdiv(a.T, R_TPW);
-    const int grid = std::max(1, std::min(cdiv(tgroups, R_WARPS), num_sms() * 8));
-    if (dtype == MOE_BF16) router_kernel<__nv_bfloat16><<<grid, R_WARPS * 32, 0, st>>>(a);
-    else router_kernel<float><<<grid, R_WARPS * 32, 0, st>>>(a);
+    const int grid = std::max(1, std::min(cdiv(a.T, R_TILE), num_sms()));
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM);
+        cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM);
+        attr_done = true;
+    }
+    if (dtype == MOE_BF16) router_kernel<__nv_bfloat16><<<grid, R_WARPS * 32, R_SMEM, st>>>(a);
+    else router_kernel<float><<<grid, R_WARPS * 32, R_SMEM, st>>>(a);
     count_launch();
     return cuda_status(cudaGetLastError());
 }

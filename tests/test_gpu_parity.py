@@ -72,6 +72,20 @@ def test_atomic_small_grid():
     check_atomic_layer(cfg, make_inputs(cfg))
 
 
+@pytest.mark.parametrize("E,T", [(2, 600), (4, 1100), (2, 513)])
+def test_cta_pair_gemm_ragged_groups(E, T):
+    """>= 512 rows per expert on average: the grouped GEMMs run on CTA pairs
+    (256-row tiles); group sizes are not multiples of 256."""
+    cfg = scaled(get_config("mixtral"), T=T, d=512, hidden=1024, n_ffn=E)
+    check_swiglu_layer(cfg, make_inputs(cfg))
+
+
+def test_atomic_cta_pair_router():
+    cfg = scaled(get_config("atomic"), T=600, d=256, pk_rows=64, pk_cols=64, pk_topk_half=16,
+                 top_k=32, d_query=128)
+    check_atomic_layer(cfg, make_inputs(cfg))
+
+
 @pytest.mark.parametrize("T", [1, 2, 127, 129])
 def test_bf16_token_counts_across_tile_edges(T):
     cfg = scaled(get_config("mixtral"), T=T, d=256, hidden=384, n_ffn=4)
@@ -124,6 +138,23 @@ def test_invalid_expert_id_sets_bounds_status():
     idx[5, 1] = 1
     moe.moe_permute(desc, idx, inp["x"], b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace)
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait on a barrier nothing arrives on gives up after its limit: the
+    kernel returns, the status reads MOE_ERR_TIMEOUT, and the next layer call
+    on the same context runs and is correct."""
+    import time
+    ok = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    moe.moe_selftest_wait_timeout(50_000_000, ok)          # 50 ms
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 1.5
+    assert int(ok.item()) == 0
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_ERR_TIMEOUT
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+    cfg = scaled(get_config("mixtral"), T=40, d=256, hidden=256, n_ffn=4)
+    check_swiglu_layer(cfg, make_inputs(cfg))
 
 
 def test_argument_errors_return_before_launch():
