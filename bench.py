@@ -183,6 +183,24 @@ def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
                       f"{el:.1f} s"}
 
 
+# ------------------------------------------------------------------- ranks
+
+def reduce_max_over_ranks(dist, values, device) -> list:
+    """Time-like values of this rank -> their maximum over all ranks (every
+    rank takes part; a single process returns its own values)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the tokens of all ranks per second of the
+    slowest rank's step time (weak scaling: every rank has its own batch)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------- ours
 
 def stage_names(cfg) -> list:
@@ -333,12 +351,8 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         cublas = library_reference(cfg, R_total, dev)
 
     mean = {n: sum(v) / K for n, v in per.items()}
-    res = {"total_ms": total_ms, "e2e_ms": e2e_ms / KE, "mean": mean}
-    if dist:   # max over ranks
-        t = torch.tensor([total_ms, res["e2e_ms"]] + [mean[n] for n in names], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        res["total_ms"], res["e2e_ms"] = float(t[0]), float(t[1])
-        res["mean"] = {n: float(t[2 + j]) for j, n in enumerate(names)}
+    red = reduce_max_over_ranks(dist, [total_ms, e2e_ms / KE] + [mean[n] for n in names], dev)
+    res = {"total_ms": red[0], "e2e_ms": red[1], "mean": {n: red[2 + j] for j, n in enumerate(names)}}
     if rank != 0:
         return None
 
@@ -356,7 +370,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     hbm = hbm or 6650.0
     work = work_model(cfg, R_total, R_ffn, touched)
     ms_step = res["total_ms"] / K
-    value = world * cfg.T / (ms_step / 1e3)
+    value = job_value(world, cfg.T, ms_step)
     kern = {}
     for n in names:
         ms = res["mean"][n]
@@ -393,7 +407,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         "kernels": kern,
         "step_tflops": round(flops / (ms_step / 1e3) / 1e12, 1),
         "rows": {"grouped": R_total, "ffn": R_ffn, "touched_experts": touched},
-        "e2e": {"value": round(world * cfg.T / (res["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_value(world, cfg.T, res["e2e_ms"]), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "moe_layer_forward, x from pinned host, y to pinned host"},
         "gpu_launches": launches,

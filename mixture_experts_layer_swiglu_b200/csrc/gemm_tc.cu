@@ -33,6 +33,10 @@ namespace moe {
 
 namespace {
 
+#ifndef MOE_KB_FENCE
+#define MOE_KB_FENCE 0            // tcgen05 fence after every stage wait (TMA -> MMA needs none)
+#endif
+
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int BN_MMA = 256;
@@ -320,7 +324,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (*abort_flag || !mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+#if MOE_KB_FENCE
                     tc_fence_after();
+#endif
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * TILE_A));
                     const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * TILE_B));
 #pragma unroll
@@ -374,15 +380,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // No multicast loads.
 
 constexpr int P_BM = 256;
+// K per stage = 64 * MOE_P_KH: one issuing thread drives the tensor cores of
+// both SMs and pays a wait / commit / loop per stage, so wider stages (more
+// MMAs each) keep it ahead of the tensor pipe.
+#ifndef MOE_P_KH
+#define MOE_P_KH 2
+#endif
 #ifndef MOE_P_STAGES
-#define MOE_P_STAGES 6
+#define MOE_P_STAGES (6 / MOE_P_KH)
 #endif
-#ifndef MOE_TMA_HINTS
-#define MOE_TMA_HINTS 0
-#endif
+constexpr int P_KH = MOE_P_KH;
+
 constexpr int P_STAGES = MOE_P_STAGES;
-constexpr int P_TILE_A = 128 * BK * 2;       // 16 KB
-constexpr int P_TILE_B = 128 * BK * 2;       // 16 KB
+constexpr int P_HALF = 128 * BK * 2;         // one 128-row x 64-K box: 16 KB
+constexpr int P_TILE_A = P_KH * P_HALF;      // A: 128 rows x 64*KH of K
+constexpr int P_TILE_B = P_KH * P_HALF;
 constexpr int P_STAGE_BYTES = P_TILE_A + P_TILE_B;
 constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + SMEM_TABLE_INTS * 4;
 
@@ -433,7 +445,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 
     const uint32_t tmem_base = *tmem_slot;
     const int total = tile_start[a.n_groups];
-    const int nk = cdiv(a.K, BK);
+    const int pnk = cdiv(a.K, BK * P_KH);          // stages of K per tile
     const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     const uint32_t full_leader = mapa_shared(smem_u32(&full[0]), 0);
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
@@ -444,10 +456,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             int s = 0;
             uint32_t ph = 0;
             bool bad = false;
-#if MOE_TMA_HINTS
-            const uint64_t pol_a = l2_policy_evict_last();
-            const uint64_t pol_b = l2_policy_evict_first();
-#endif
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
                 const TileInfo ti = decode_tile<P_BM>(tile, tile_start, g_lo, g_cnt, a.n_groups);
                 const bool first = ti.g < a.n_first;
@@ -462,18 +470,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     brow = gb * a.N + ti.n * 256 + (int)rank * 128;
                 }
                 const int arow = ti.row0 + (int)rank * 128;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
+                if (*abort_flag) { bad = true; break; }
+                for (int kb = 0; kb < pnk; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
                     if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
-#if MOE_TMA_HINTS
-                    // A rows (tokens) serve every n-tile of the group; each B
-                    // tile serves only the group's few m-tiles
-                    tma_load_2d_pair_hint(sA + s * P_TILE_A, &tmA, full_leader + 8 * s, kb * BK, arow, pol_a);
-                    tma_load_2d_pair_hint(sB + s * P_TILE_B, mb, full_leader + 8 * s, kb * BK, brow, pol_b);
-#else
-                    tma_load_2d_pair(sA + s * P_TILE_A, &tmA, full_leader + 8 * s, kb * BK, arow);
-                    tma_load_2d_pair(sB + s * P_TILE_B, mb, full_leader + 8 * s, kb * BK, brow);
-#endif
+#pragma unroll
+                    for (int h = 0; h < P_KH; ++h) {
+                        const int k0 = (kb * P_KH + h) * BK;      // past K: zero fill
+                        tma_load_2d_pair(sA + s * P_TILE_A + h * P_HALF, &tmA, full_leader + 8 * s, k0, arow);
+                        tma_load_2d_pair(sB + s * P_TILE_B + h * P_HALF, mb, full_leader + 8 * s, k0, brow);
+                    }
                     if (++s == P_STAGES) { s = 0; ph ^= 1; }
                 }
             }
@@ -489,18 +495,26 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             int s = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             bool bad = false;
+            const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
+            const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
                 if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (*abort_flag || !mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+                for (int kb = 0; kb < pnk; ++kb) {
+                    if (!mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+#if MOE_KB_FENCE
                     tc_fence_after();
-                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * P_TILE_A));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * P_TILE_B));
+#endif
+                    // descriptor start addresses advance in 16-byte units
+                    const uint64_t ad = ad0 + (uint64_t)((s * P_TILE_A) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)((s * P_TILE_B) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        tc_mma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    for (int h = 0; h < P_KH; ++h)
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma_bf16_pair(d_tmem, ad + (h * P_HALF >> 4) + 2 * kk, bd + (h * P_HALF >> 4) + 2 * kk,
+                                             idesc, (kb | h | kk) != 0);
                     tc_commit_pair(&empty[s], 0x3);
                     if (++s == P_STAGES) { s = 0; ph ^= 1; }
                 }
