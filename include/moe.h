@@ -183,8 +183,10 @@ MOE_API moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_i
  *   kept in fp32.  y_sorted [row capacity, d_model] fp32.  token_of, x,
  *   topk_gate unused.
  * Atomic: c[s] = topk_gate[s] * GELU(u_e . x_t) for each task s = t*K + j of
- *   expert e, computed expert by expert (each u_e read once); y_sorted is
- *   float c[T*K] in slot order.  x_sorted unused.
+ *   expert e, over the expert-sorted task order in units of 16 tasks whose
+ *   dot products are one tensor-core tile (each touched u_e read once per
+ *   unit); y_sorted is float c[T*K] in slot order.  x_sorted unused.  The
+ *   workspace holds the expert of each task (T*top_k int32).
  */
 MOE_API moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_layer_weights* w,
                            const void* x_sorted, const int32_t* expert_offsets,

@@ -12,9 +12,9 @@
 //
 // Atomic experts ("OmniMoE" 2.1 Atomic Experts E_i(x) = sigma(x . u_i) v_i,
 // Dynamic Expert Assembly; 2.2 Expert-Centric Scheduling):
-//   phase A, expert by expert: each touched u_e is read once from HBM and
-//     dotted with the x rows of its tasks (x stays in L2):
-//     c[s] = g[s] * GELU(u_e . x_t);
+//   phase A, over the expert-sorted tasks: the dot products u_e . x_t of 16
+//     consecutive tasks are one m16n8k16 tile sequence (x stays in L2, each
+//     touched u_e is read once): c[s] = g[s] * GELU(u_e . x_t);
 //   phase B, token by token: y_t = sum_j c[t, j] v_{e_tj}, fp32 in slot order.
 
 #include <cuda_bf16.h>
@@ -203,43 +203,132 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
 
 // ---------------------------------------------------------------- atomic
 
-// phase A: one warp per expert; u_e kept in registers (NV uint4 per lane).
-template <int NV>
-__global__ void __launch_bounds__(256) atomic_phase_a_kernel(const AtomicArgs a)
+// Expert of every task: task_expert[p] = e for p in [offsets[e], offsets[e+1]).
+__global__ void atomic_task_expert_kernel(const int32_t* offsets, int N, long long cap, int32_t* te)
 {
-    const int lane = threadIdx.x & 31;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < N;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int lo = offsets[e], hi = offsets[e + 1];
+        if (lo < 0 || hi > cap || lo > hi) {
+            set_status(MOE_ERR_DEVICE_BOUNDS);
+            continue;
+        }
+        for (int p = lo; p < hi; ++p) te[p] = (int)e;
+    }
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int AT_M = 16;       // tasks per warp unit
+constexpr int AT_UNROLL = 4;   // 32-element chunks of d whose loads are issued together
+
+// D[i][j] += x_{t_i} . u_{e_j} over d for the 16 task rows i and NT*8 expert
+// columns j.  Chunk c covers elements [32c, 32c + 32); lane (g, q) loads the
+// 16 bytes at 32c + 8q of its A rows (tasks g, g + 8) and B rows (columns g,
+// g + 8) and feeds them to two k16 steps, so A and B agree on the k order.
+template <int NT>
+__device__ __forceinline__ void atomic_dot_tiles(const uint4* xr0, const uint4* xr1, const uint4* ur0,
+                                                 const uint4* ur1, int chunks, int q, float (&d0)[4],
+                                                 float (&d1)[4])
+{
+    for (int c0 = 0; c0 < chunks; c0 += AT_UNROLL) {
+        uint4 xa[AT_UNROLL], xb[AT_UNROLL], ua[AT_UNROLL], ub[AT_UNROLL];
+#pragma unroll
+        for (int c = 0; c < AT_UNROLL; ++c) {
+            const int o = (c0 + c) * 4 + q;
+            xa[c] = __ldg(xr0 + o);
+            xb[c] = __ldg(xr1 + o);
+            ua[c] = __ldg(ur0 + o);
+            if (NT == 2) ub[c] = __ldg(ur1 + o);
+        }
+#pragma unroll
+        for (int c = 0; c < AT_UNROLL; ++c) {
+            mma_16816(d0, xa[c].x, xb[c].x, xa[c].y, xb[c].y, ua[c].x, ua[c].y);
+            mma_16816(d0, xa[c].z, xb[c].z, xa[c].w, xb[c].w, ua[c].z, ua[c].w);
+            if (NT == 2) {
+                mma_16816(d1, xa[c].x, xb[c].x, xa[c].y, xb[c].y, ub[c].x, ub[c].y);
+                mma_16816(d1, xa[c].z, xb[c].z, xa[c].w, xb[c].w, ub[c].z, ub[c].w);
+            }
+        }
+    }
+}
+
+// phase A: c[s] = g[s] * GELU(u_e . x_t) for every task (s = slot t*K + j,
+// e its expert).  A warp takes 16 consecutive tasks of the expert-sorted
+// order; their distinct experts (at most 16, about 7 at 2.4 tasks per
+// expert) are the columns of one or two m16n8 tiles, and task i keeps
+// D[i][column of its expert].  Each touched u_e is read once per unit it
+// appears in (x stays in L2); the tensor cores do the dot products.
+__global__ void __launch_bounds__(256, 2) atomic_phase_a_kernel(const AtomicArgs a)
+{
+    __shared__ int col_expert[8][AT_M];
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int wib = threadIdx.x >> 5;
+    const long long cap = (long long)a.T * a.K;
+    const int R = (int)min((long long)a.offsets[a.N], cap);
+    const int units = (R + AT_M - 1) / AT_M;
+    const int vecs = a.d >> 3;
+    const int chunks = a.d >> 5;
     const uint4* x = reinterpret_cast<const uint4*>(a.x);
     const uint4* u = reinterpret_cast<const uint4*>(a.u);
-    const int vecs = a.d / 8;
-    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long e = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); e < a.N; e += nw) {
-        const int lo = a.offsets[e], hi = a.offsets[e + 1];
-        if (lo >= hi) continue;
-        float ue[NV][8];
-#pragma unroll
-        for (int q = 0; q < NV; ++q) {
-            const uint4 w = __ldg(u + e * vecs + q * 32 + lane);
-            ue[q][0] = bf16_lo(w.x); ue[q][1] = bf16_hi(w.x); ue[q][2] = bf16_lo(w.y); ue[q][3] = bf16_hi(w.y);
-            ue[q][4] = bf16_lo(w.z); ue[q][5] = bf16_hi(w.z); ue[q][6] = bf16_lo(w.w); ue[q][7] = bf16_hi(w.w);
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    for (int un = blockIdx.x * (blockDim.x >> 5) + wib; un < units; un += nw) {
+        const int p = un * AT_M + (lane & (AT_M - 1));
+        int s = -1, e = -1;
+        float gt = 0.f;
+        if (lane < AT_M && p < R) {
+            s = a.token_of[p];
+            e = a.task_expert[p];
+            if (s < 0 || s >= cap || e < 0 || e >= a.N) {
+                set_status(MOE_ERR_DEVICE_BOUNDS);
+                s = -1;
+                e = -1;
+            } else {
+                gt = a.gate[s];
+            }
         }
-        for (int p = lo; p < hi; ++p) {
-            const int s = a.token_of[p];
-            const int t = s / a.K;
-            float dot = 0.f;
+        const int eprev = __shfl_up_sync(FULL, e, 1);
+        const bool fresh = lane < AT_M && e >= 0 && (lane == 0 || e != eprev);
+        const unsigned nm = __ballot_sync(FULL, fresh);
+        const int ndist = __popc(nm);
+        if (ndist == 0) continue;
+        const int col = __popc(nm & ((2u << (lane & (AT_M - 1))) - 1u)) - 1;   // tasks: own column
+        if (fresh) col_expert[wib][col] = e;
+        __syncwarp();
+        const int s0 = __shfl_sync(FULL, s, g), s1 = __shfl_sync(FULL, s, g + 8);
+        const int k0 = __shfl_sync(FULL, col, g), k1 = __shfl_sync(FULL, col, g + 8);
+        const float g0 = __shfl_sync(FULL, gt, g), g1 = __shfl_sync(FULL, gt, g + 8);
+        const uint4* xr0 = x + (long long)(s0 >= 0 ? s0 / a.K : 0) * vecs;
+        const uint4* xr1 = x + (long long)(s1 >= 0 ? s1 / a.K : 0) * vecs;
+        const uint4* ur0 = u + (long long)col_expert[wib][min(g, ndist - 1)] * vecs;
+        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ndist <= 8) {
+            atomic_dot_tiles<1>(xr0, xr1, ur0, ur0, chunks, q, d0, d1);
+        } else {
+            const uint4* ur1 = u + (long long)col_expert[wib][min(g + 8, ndist - 1)] * vecs;
+            atomic_dot_tiles<2>(xr0, xr1, ur0, ur1, chunks, q, d0, d1);
+        }
+        __syncwarp();
+        // D fragment: d[0], d[1] = row g, columns 2q, 2q+1; d[2], d[3] = row g+8.
 #pragma unroll
-            for (int q = 0; q < NV; ++q) {
-                const uint4 w = __ldg(x + (long long)t * vecs + q * 32 + lane);
-                dot = fmaf(ue[q][0], bf16_lo(w.x), dot); dot = fmaf(ue[q][1], bf16_hi(w.x), dot);
-                dot = fmaf(ue[q][2], bf16_lo(w.y), dot); dot = fmaf(ue[q][3], bf16_hi(w.y), dot);
-                dot = fmaf(ue[q][4], bf16_lo(w.z), dot); dot = fmaf(ue[q][5], bf16_hi(w.z), dot);
-                dot = fmaf(ue[q][6], bf16_lo(w.w), dot); dot = fmaf(ue[q][7], bf16_hi(w.w), dot);
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(FULL, dot, o);
-            if (lane == 0) {
-                const float gel = 0.5f * dot * (1.0f + erff(dot * 0.70710678118654752f));
-                a.c[s] = a.gate[s] * gel;
-            }
+        for (int h = 0; h < 2; ++h) {
+            const int sr = h ? s1 : s0, kr = h ? k1 : k0;
+            if (sr < 0) continue;
+            const int tile = kr >> 3, cc = kr & 7;
+            if ((cc >> 1) != q) continue;
+            const float lo = tile ? d1[2 * h] : d0[2 * h];
+            const float hi = tile ? d1[2 * h + 1] : d0[2 * h + 1];
+            const float dot = (cc & 1) ? hi : lo;
+            const float gel = 0.5f * dot * (1.0f + erff(dot * 0.70710678118654752f));
+            a.c[sr] = (h ? g1 : g0) * gel;
         }
     }
 }
@@ -310,12 +399,6 @@ moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
     return cuda_status(cudaGetLastError());
 }
 
-template <int NV> struct PhaseA {
-    static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
-    {
-        atomic_phase_a_kernel<NV><<<grid, 256, 0, st>>>(a);
-    }
-};
 template <int NV> struct PhaseB {
     static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
     {
@@ -339,8 +422,17 @@ moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st)
 
 moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st)
 {
-    const int grid = std::max(1, std::min(cdiv(a.N, 8), num_sms() * 16));
-    return launch_nv<PhaseA>(a.d / 256, grid, st, a);
+    const long long cap = (long long)a.T * a.K;
+    if (cap == 0) return MOE_OK;
+    if (a.d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    const int g0 = (int)std::min<long long>((a.N + 255) / 256, num_sms() * 8);
+    atomic_task_expert_kernel<<<std::max(1, g0), 256, 0, st>>>(a.offsets, a.N, cap, a.task_expert);
+    count_launch();
+    const long long units = (cap + AT_M - 1) / AT_M;
+    const int grid = (int)std::max(1LL, std::min<long long>((units + 7) / 8, num_sms() * 2));
+    atomic_phase_a_kernel<<<grid, 256, 0, st>>>(a);
+    count_launch();
+    return cuda_status(cudaGetLastError());
 }
 
 moe_status launch_atomic_phase_b(const AtomicArgs& a, cudaStream_t st)

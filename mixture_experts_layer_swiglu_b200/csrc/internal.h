@@ -117,6 +117,7 @@ struct AtomicArgs {
     const void* v;        // [N, d]
     const int32_t* offsets;
     const int32_t* token_of;   // task -> slot id
+    int32_t* task_expert;      // task -> expert (scratch, written by phase A's first kernel)
     const int32_t* idx;        // [T, K]
     const float* gate;         // [T, K]
     float* c;                  // [T*K]

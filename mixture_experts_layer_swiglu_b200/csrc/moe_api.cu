@@ -105,6 +105,7 @@ Scratch scratch_sizes(const moe_layer_desc* d)
                   al((size_t)2 * d->T * d->pk_rows * 4);
         const size_t N = (size_t)d->pk_rows * d->pk_cols;
         s.permute = al(N * 4) * 2 + al((size_t)atomic_scan_blocks((int)N) * 4);
+        s.ffn = al((size_t)d->T * d->top_k * 4);
     }
     return s;
 }
@@ -366,8 +367,11 @@ moe_status ffn_impl(const moe_layer_desc* d, const moe_layer_weights* w, const v
         return ffn_phase_impl(d, w, 2, xs, offsets, ys, ws, ws_bytes, st);
     }
     if (!w->u || !aligned16(w->u) || !x || !aligned16(x) || !gate || !token_of) return MOE_ERR_INVALID_ARG;
+    const Scratch sc = scratch_sizes(d);
+    if (!ws || ws_bytes < sc.ffn || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     AtomicArgs a{};
     a.x = x;
+    a.task_expert = static_cast<int32_t*>(ws);
     a.u = w->u;
     a.v = w->v;
     a.offsets = offsets;

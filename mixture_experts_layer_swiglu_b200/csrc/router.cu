@@ -285,45 +285,105 @@ __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a
 }
 
 // ------------------------------------------------------- product-key selection
+//
+// Every candidate gets one unsigned 64-bit key whose order is the selection
+// order (descending score, ties to the lower index): the high word maps the
+// score to an unsigned integer with the same order, the low word is the
+// complement of the index.  The best of 32 lane keys is then two (three for
+// the merge, whose scores are fp64) __reduce_max_sync steps, with no
+// shuffles.
 
-// Best kh of n scores (per lane: elements lane + 32 i, i < MAXV); lane j < kh
-// receives the j-th best value and its index.
-template <int MAXV>
-__device__ __forceinline__ void top_half(const float* s, int n, int kh, int lane, float& out_v,
-                                         int& out_i)
+__device__ __forceinline__ uint32_t order_key32(float v)
 {
-    float vals[MAXV];
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;                    // -0 orders as +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key32_value(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ unsigned long long order_key64(double v)
+{
+    unsigned long long b = (unsigned long long)__double_as_longlong(v);
+    if (b == 0x8000000000000000ull) b = 0ull;
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// Bitonic sort of a lane's keys, descending.
+template <int MAXV>
+__device__ __forceinline__ void sort_desc(unsigned long long (&c)[MAXV])
+{
+#pragma unroll
+    for (int k = 2; k <= MAXV; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < MAXV; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const unsigned long long a = c[i], b = c[l];
+                    const bool sw = ((i & k) == 0) ? (a < b) : (a > b);
+                    c[i] = sw ? b : a;
+                    c[l] = sw ? a : b;
+                }
+            }
+}
+
+// Best kh of the n scores s[0..n) (kh <= n), best first, into out_v / out_i.
+// Lane l owns elements l + 32 i, sorts them, and keeps all but its current
+// head in `list` ([MAXV][32], this warp's); each step the warp takes the
+// best head and only the winning lane advances.
+template <int MAXV>
+__device__ __forceinline__ void select_half(const float* s, int n, int kh, int lane,
+                                            unsigned long long* list, float* out_v, int* out_i)
+{
+    unsigned long long c[MAXV];
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
         const int e = lane + 32 * i;
-        vals[i] = e < n ? s[e] : -INFINITY;
+        c[i] = e < n ? ((unsigned long long)order_key32(__ldg(s + e)) << 32) | (uint32_t)~e : 0ull;
     }
-    uint32_t taken = 0;
-    out_v = -INFINITY;
-    out_i = -1;
+    sort_desc<MAXV>(c);
+#pragma unroll
+    for (int i = 1; i < MAXV; ++i) list[i * 32 + lane] = c[i];
+    __syncwarp();
+    unsigned long long head = c[0];
+    int h = 0;
     for (int j = 0; j < kh; ++j) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
-#pragma unroll
-        for (int i = 0; i < MAXV; ++i) {
-            const int e = lane + 32 * i;
-            if (e < n && !((taken >> i) & 1u) && better(vals[i], e, bv, bi)) { bv = vals[i]; bi = e; }
+        const uint32_t hi = (uint32_t)(head >> 32), lo = (uint32_t)head;
+        const uint32_t m1 = __reduce_max_sync(FULL, hi);
+        const uint32_t m2 = __reduce_max_sync(FULL, hi == m1 ? lo : 0u);
+        if (hi == m1 && lo == m2) {
+            out_v[j] = key32_value(hi);
+            out_i[j] = (int)~lo;
+            ++h;
+            head = h < MAXV ? list[h * 32 + lane] : 0ull;
         }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(FULL, bv, o);
-            const int oi = __shfl_xor_sync(FULL, bi, o);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == j) { out_v = bv; out_i = (bi == INT_MAX) ? -1 : bi; }
     }
+    __syncwarp();
 }
 
+template <int MAXV> struct PkWarpSmem {
+    unsigned long long list[MAXV * 32];
+    double sel_v[128];
+    int sel_i[128];
+    float rv[32], cv[32];
+    int ri[32], ci[32];
+};
+
+// One warp per token.  The merge relies on both halves being sorted: lane
+// i < kh walks row candidate i along the sorted columns, so its next
+// candidate is always its best remaining one, and the best of the lanes'
+// heads is the best remaining pair.
 template <int MAXV>
 __global__ void __launch_bounds__(256) pk_select_kernel(const PkSelectArgs a)
 {
+    extern __shared__ __align__(16) unsigned char pk_smem[];
     const int lane = threadIdx.x & 31;
+    PkWarpSmem<MAXV>& w = reinterpret_cast<PkWarpSmem<MAXV>*>(pk_smem)[threadIdx.x >> 5];
     const int warps = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += warps) {
         const float* sr = a.s_row + (long long)t * a.rows;
@@ -333,61 +393,59 @@ __global__ void __launch_bounds__(256) pk_select_kernel(const PkSelectArgs a)
             for (int e = lane; e < a.rows; e += 32) lo[e] = sr[e];
             for (int e = lane; e < a.cols; e += 32) lo[a.rows + e] = sc[e];
         }
-        float rv, cv;
-        int ri, ci;
-        top_half<MAXV>(sr, a.rows, a.kh, lane, rv, ri);
-        top_half<MAXV>(sc, a.cols, a.kh, lane, cv, ci);
+        select_half<MAXV>(sr, a.rows, a.kh, lane, w.list, w.rv, w.ri);
+        select_half<MAXV>(sc, a.cols, a.kh, lane, w.list, w.cv, w.ci);
 
-        // merge: lane i < kh walks row candidate i along its sorted columns
+        const bool rowl = lane < a.kh;
+        const double my_r = rowl ? (double)w.rv[lane] : 0.0;
+        const int my_base = rowl ? w.ri[lane] * a.cols : 0;
         int p = 0;
-        double v0 = 0.0;
-        double selv[4];
-        int selid[4];
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-            selv[blk] = -INFINITY;
-            selid[blk] = -1;
-            for (int jj = 0; jj < 32; ++jj) {
-                const int j = blk * 32 + jj;
-                if (j >= a.K) break;
-                const float cvp = __shfl_sync(FULL, cv, p & 31);
-                const int cip = __shfl_sync(FULL, ci, p & 31);
-                double hv = -INFINITY;
-                int hid = INT_MAX, wl = lane;
-                if (lane < a.kh && p < a.kh && ri >= 0 && cip >= 0) {
-                    hv = (double)rv + (double)cvp;
-                    hid = ri * a.cols + cip;
+        double sum = my_r + (double)w.cv[0];
+        unsigned long long key = rowl ? order_key64(sum) : 0ull;
+        uint32_t id = (uint32_t)(my_base + w.ci[0]);
+        for (int j = 0; j < a.K; ++j) {
+            const uint32_t hi = (uint32_t)(key >> 32), lo = (uint32_t)key;
+            const uint32_t m1 = __reduce_max_sync(FULL, hi);
+            bool win = hi == m1;
+            if (__popc(__ballot_sync(FULL, win)) > 1) {        // equal high words: rare
+                const uint32_t m2 = __reduce_max_sync(FULL, win ? lo : 0u);
+                win = win && lo == m2;
+                const uint32_t m3 = __reduce_max_sync(FULL, win ? ~id : 0u);
+                win = win && ~id == m3;
+            }
+            if (win) {
+                w.sel_v[j] = sum;
+                w.sel_i[j] = (int)id;
+                if (++p < a.kh) {
+                    sum = my_r + (double)w.cv[p];
+                    key = order_key64(sum);
+                    id = (uint32_t)(my_base + w.ci[p]);
+                } else {
+                    key = 0ull;
                 }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    const double ov = __shfl_xor_sync(FULL, hv, o);
-                    const int oi = __shfl_xor_sync(FULL, hid, o);
-                    const int ol = __shfl_xor_sync(FULL, wl, o);
-                    if (ov > hv || (ov == hv && oi < hid)) { hv = ov; hid = oi; wl = ol; }
-                }
-                if (lane == wl) ++p;
-                if (j == 0) v0 = hv;
-                if (jj == lane) { selv[blk] = hv; selid[blk] = (hid == INT_MAX) ? -1 : hid; }
             }
         }
+        __syncwarp();
+        const double v0 = w.sel_v[0];
         float ex[4];
-        float sum = 0.f;
+        float tot = 0.f;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             const int j = blk * 32 + lane;
-            ex[blk] = (j < a.K) ? expf((float)(selv[blk] - v0)) : 0.f;
-            sum += ex[blk];
+            ex[blk] = (j < a.K) ? expf((float)(w.sel_v[j] - v0)) : 0.f;
+            tot += ex[blk];
         }
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+        for (int o = 16; o >= 1; o >>= 1) tot += __shfl_xor_sync(FULL, tot, o);
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             const int j = blk * 32 + lane;
             if (j < a.K) {
-                a.idx[(long long)t * a.K + j] = selid[blk];
-                a.gate[(long long)t * a.K + j] = ex[blk] / sum;
+                a.idx[(long long)t * a.K + j] = w.sel_i[j];
+                a.gate[(long long)t * a.K + j] = ex[blk] / tot;
             }
         }
+        __syncwarp();
     }
 }
 
@@ -425,10 +483,19 @@ moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
 moe_status launch_pk_select(const PkSelectArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
-    const int grid = std::max(1, std::min(cdiv(a.T, 8), num_sms() * 8));
+    constexpr int warps = 8;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaFuncSetAttribute(pk_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             warps * (int)sizeof(PkWarpSmem<16>));
+        cudaFuncSetAttribute(pk_select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             warps * (int)sizeof(PkWarpSmem<32>));
+        attr_done = true;
+    }
+    const int grid = std::max(1, std::min(cdiv(a.T, warps), num_sms() * 4));
     const int n = std::max(a.rows, a.cols);
-    if (n <= 512) pk_select_kernel<16><<<grid, 256, 0, st>>>(a);
-    else pk_select_kernel<32><<<grid, 256, 0, st>>>(a);
+    if (n <= 512) pk_select_kernel<16><<<grid, warps * 32, warps * sizeof(PkWarpSmem<16>), st>>>(a);
+    else pk_select_kernel<32><<<grid, warps * 32, warps * sizeof(PkWarpSmem<32>), st>>>(a);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
