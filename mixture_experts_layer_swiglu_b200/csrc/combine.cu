@@ -16,6 +16,9 @@
 //     consecutive tasks are one m16n8k16 tile sequence (x stays in L2, each
 //     touched u_e is read once): c[s] = g[s] * GELU(u_e . x_t);
 //   phase B, token by token: y_t = sum_j c[t, j] v_{e_tj}, fp32 in slot order.
+// Phase A loads its operands straight into registers with 32-byte loads;
+// phase B streams whole v rows through a warp-private ring of shared-memory
+// stages filled by bulk copies.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -203,124 +206,172 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
 
 // ---------------------------------------------------------------- atomic
 
-// Expert of every task: task_expert[p] = e for p in [offsets[e], offsets[e+1]).
-__global__ void atomic_task_expert_kernel(const int32_t* offsets, int N, long long cap, int32_t* te)
+// Per task p of the expert-sorted order: its expert (task_expert[p] = e for
+// p in [offsets[e], offsets[e+1])) and its gate (task_gate[p] = gate[slot]).
+__global__ void atomic_task_meta_kernel(const AtomicArgs a)
 {
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < N;
-         e += (long long)gridDim.x * blockDim.x) {
-        const int lo = offsets[e], hi = offsets[e + 1];
-        if (lo < 0 || hi > cap || lo > hi) {
-            set_status(MOE_ERR_DEVICE_BOUNDS);
-            continue;
+    const long long cap = (long long)a.T * a.K;
+    const int R = (int)min((long long)a.offsets[a.N], cap);
+    const long long n = max((long long)a.N, (long long)R);
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        if (i < a.N) {
+            const int lo = a.offsets[i], hi = a.offsets[i + 1];
+            if (lo < 0 || hi > cap || lo > hi) set_status(MOE_ERR_DEVICE_BOUNDS);
+            else
+                for (int p = lo; p < hi; ++p) a.task_expert[p] = (int)i;
         }
-        for (int p = lo; p < hi; ++p) te[p] = (int)e;
+        if (i < R) {
+            const int s = a.token_of[i];
+            a.task_gate[i] = (s >= 0 && s < cap) ? a.gate[s] : 0.f;
+        }
     }
 }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int AT_M = 16;       // tasks per warp unit
-constexpr int AT_UNROLL = 4;   // 32-element chunks of d whose loads are issued together
+// ---- phase A: c[s] = g[s] * GELU(u_e . x_t) for every task.
+//
+// A warp takes units of 16 consecutive tasks of the expert-sorted order.
+// The unit's distinct experts (at most 16, about 7 at 2.4 tasks per expert)
+// are the columns of one or two m16n8 tiles; D[i][j] = x_{t_i} . u_{e_j}
+// accumulates over d on the tensor cores and task i keeps D[i][its column].
+// Operands come straight from global memory into registers with 32-byte
+// loads: for each 64-element slice of d, lane (g, q) loads bytes
+// [32q, 32q + 32) of its A rows (tasks g, g+8) and B rows (columns g, g+8),
+// so one warp instruction reads 8 whole 128-byte lines, and those 16
+// elements feed four k16 steps.  The k order this implies (step s takes
+// elements 16q + 4s + {0,1} as k = 2q, 2q+1 and 16q + 4s + {2,3} as k = 2q+8,
+// 2q+9) is the same for A and B, so the sums are the dot products.  x rows
+// come from L2, each touched u row from HBM once per unit it appears in;
+// occupancy (16 warps per SM, each with up to 12 KiB of loads in flight)
+// hides the latency.
+constexpr int AT_M = 16;
+constexpr int PA_WARPS = 4;
+#ifndef MOE_PA_U1
+#define MOE_PA_U1 4      // 64-element slices loaded together, one-tile units
+#endif
+#ifndef MOE_PA_U2
+#define MOE_PA_U2 2      // the same, two-tile units
+#endif
+#ifndef MOE_PA_MINB
+#define MOE_PA_MINB 4    // resident blocks per SM
+#endif
+static_assert(4 % MOE_PA_U1 == 0 && 4 % MOE_PA_U2 == 0, "slice groups must divide d / 64 for d = 256");
 
-// D[i][j] += x_{t_i} . u_{e_j} over d for the 16 task rows i and NT*8 expert
-// columns j.  Chunk c covers elements [32c, 32c + 32); lane (g, q) loads the
-// 16 bytes at 32c + 8q of its A rows (tasks g, g + 8) and B rows (columns g,
-// g + 8) and feeds them to two k16 steps, so A and B agree on the k order.
-template <int NT>
-__device__ __forceinline__ void atomic_dot_tiles(const uint4* xr0, const uint4* xr1, const uint4* ur0,
-                                                 const uint4* ur1, int chunks, int q, float (&d0)[4],
-                                                 float (&d1)[4])
+struct PaRaw {       // lane i < 16: task i of a unit
+    int s, e;
+    float g;
+};
+
+__device__ __forceinline__ PaRaw pa_load(const AtomicArgs& a, int un, int units, int R, long long cap, int lane)
 {
-    for (int c0 = 0; c0 < chunks; c0 += AT_UNROLL) {
-        uint4 xa[AT_UNROLL], xb[AT_UNROLL], ua[AT_UNROLL], ub[AT_UNROLL];
+    PaRaw r{-1, -1, 0.f};
+    const int p = un * AT_M + lane;
+    if (un < units && lane < AT_M && p < R) {
+        const int s = a.token_of[p], e = a.task_expert[p];
+        if (s < 0 || s >= cap || e < 0 || e >= a.N) {
+            set_status(MOE_ERR_DEVICE_BOUNDS);
+        } else {
+            r.s = s;
+            r.e = e;
+            r.g = a.task_gate[p];
+        }
+    }
+    return r;
+}
+
+__device__ __forceinline__ void ld256(const unsigned char* p, uint32_t (&r)[8])
+{
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+
+// D += the products of the 64-element slices of d, in groups of U slices
+// whose loads are issued together (one tile: U * 3 KiB per warp in flight,
+// two tiles: U * 4 KiB).  Measured on B200 for d = 1024, groups of 4 / 2
+// slices at 16 warps per SM beat both smaller groups at higher occupancy and
+// double-buffered groups.  U divides the slice count for every supported d.
+template <int NT>
+__device__ __forceinline__ void pa_dot(const unsigned char* xr0, const unsigned char* xr1, const unsigned char* ur0,
+                                       const unsigned char* ur1, int nsc, int q, float (&d0)[4], float (&d1)[4])
+{
+    constexpr int U = NT == 1 ? MOE_PA_U1 : MOE_PA_U2;
+#pragma unroll 1
+    for (int sc = 0; sc < nsc; sc += U) {
+        uint32_t xa[U][8], xb[U][8], ua[U][8], ub[NT == 2 ? U : 1][8];
 #pragma unroll
-        for (int c = 0; c < AT_UNROLL; ++c) {
-            const int o = (c0 + c) * 4 + q;
-            xa[c] = __ldg(xr0 + o);
-            xb[c] = __ldg(xr1 + o);
-            ua[c] = __ldg(ur0 + o);
-            if (NT == 2) ub[c] = __ldg(ur1 + o);
+        for (int u = 0; u < U; ++u) {
+            const int off = (sc + u) * 128 + q * 32;
+            ld256(xr0 + off, xa[u]);
+            ld256(xr1 + off, xb[u]);
+            ld256(ur0 + off, ua[u]);
+            if constexpr (NT == 2) ld256(ur1 + off, ub[u]);
         }
 #pragma unroll
-        for (int c = 0; c < AT_UNROLL; ++c) {
-            mma_16816(d0, xa[c].x, xb[c].x, xa[c].y, xb[c].y, ua[c].x, ua[c].y);
-            mma_16816(d0, xa[c].z, xb[c].z, xa[c].w, xb[c].w, ua[c].z, ua[c].w);
-            if (NT == 2) {
-                mma_16816(d1, xa[c].x, xb[c].x, xa[c].y, xb[c].y, ub[c].x, ub[c].y);
-                mma_16816(d1, xa[c].z, xb[c].z, xa[c].w, xb[c].w, ub[c].z, ub[c].w);
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int st = 0; st < 4; ++st) {
+                mma_16816(d0, xa[u][2 * st], xb[u][2 * st], xa[u][2 * st + 1], xb[u][2 * st + 1], ua[u][2 * st],
+                          ua[u][2 * st + 1]);
+                if constexpr (NT == 2)
+                    mma_16816(d1, xa[u][2 * st], xb[u][2 * st], xa[u][2 * st + 1], xb[u][2 * st + 1], ub[u][2 * st],
+                              ub[u][2 * st + 1]);
             }
-        }
     }
 }
 
-// phase A: c[s] = g[s] * GELU(u_e . x_t) for every task (s = slot t*K + j,
-// e its expert).  A warp takes 16 consecutive tasks of the expert-sorted
-// order; their distinct experts (at most 16, about 7 at 2.4 tasks per
-// expert) are the columns of one or two m16n8 tiles, and task i keeps
-// D[i][column of its expert].  Each touched u_e is read once per unit it
-// appears in (x stays in L2); the tensor cores do the dot products.
-__global__ void __launch_bounds__(256, 2) atomic_phase_a_kernel(const AtomicArgs a)
+__global__ void __launch_bounds__(PA_WARPS * 32, MOE_PA_MINB) atomic_phase_a_kernel(const AtomicArgs a)
 {
-    __shared__ int col_expert[8][AT_M];
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int wib = threadIdx.x >> 5;
+    __shared__ int col_expert[PA_WARPS][AT_M];
+    __shared__ int task_slot[PA_WARPS][AT_M], task_col[PA_WARPS][AT_M];
+    __shared__ float task_g[PA_WARPS][AT_M];
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, wib = threadIdx.x >> 5;
     const long long cap = (long long)a.T * a.K;
     const int R = (int)min((long long)a.offsets[a.N], cap);
     const int units = (R + AT_M - 1) / AT_M;
-    const int vecs = a.d >> 3;
-    const int chunks = a.d >> 5;
-    const uint4* x = reinterpret_cast<const uint4*>(a.x);
-    const uint4* u = reinterpret_cast<const uint4*>(a.u);
-    const int nw = gridDim.x * (blockDim.x >> 5);
-    for (int un = blockIdx.x * (blockDim.x >> 5) + wib; un < units; un += nw) {
-        const int p = un * AT_M + (lane & (AT_M - 1));
-        int s = -1, e = -1;
-        float gt = 0.f;
-        if (lane < AT_M && p < R) {
-            s = a.token_of[p];
-            e = a.task_expert[p];
-            if (s < 0 || s >= cap || e < 0 || e >= a.N) {
-                set_status(MOE_ERR_DEVICE_BOUNDS);
-                s = -1;
-                e = -1;
-            } else {
-                gt = a.gate[s];
-            }
-        }
-        const int eprev = __shfl_up_sync(FULL, e, 1);
-        const bool fresh = lane < AT_M && e >= 0 && (lane == 0 || e != eprev);
+    const int nsc = a.d / 64;
+    const size_t rowb = (size_t)a.d * 2;
+    const unsigned char* xb = static_cast<const unsigned char*>(a.x);
+    const unsigned char* ub = static_cast<const unsigned char*>(a.u);
+    const int nw = gridDim.x * PA_WARPS;
+    int un = blockIdx.x * PA_WARPS + wib;
+    PaRaw r = pa_load(a, un, units, R, cap, lane);
+    for (; un < units; un += nw) {
+        const int eprev = __shfl_up_sync(FULL, r.e, 1);
+        const bool fresh = r.e >= 0 && (lane == 0 || r.e != eprev);
         const unsigned nm = __ballot_sync(FULL, fresh);
         const int ndist = __popc(nm);
-        if (ndist == 0) continue;
-        const int col = __popc(nm & ((2u << (lane & (AT_M - 1))) - 1u)) - 1;   // tasks: own column
-        if (fresh) col_expert[wib][col] = e;
-        __syncwarp();
-        const int s0 = __shfl_sync(FULL, s, g), s1 = __shfl_sync(FULL, s, g + 8);
-        const int k0 = __shfl_sync(FULL, col, g), k1 = __shfl_sync(FULL, col, g + 8);
-        const float g0 = __shfl_sync(FULL, gt, g), g1 = __shfl_sync(FULL, gt, g + 8);
-        const uint4* xr0 = x + (long long)(s0 >= 0 ? s0 / a.K : 0) * vecs;
-        const uint4* xr1 = x + (long long)(s1 >= 0 ? s1 / a.K : 0) * vecs;
-        const uint4* ur0 = u + (long long)col_expert[wib][min(g, ndist - 1)] * vecs;
-        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-        if (ndist <= 8) {
-            atomic_dot_tiles<1>(xr0, xr1, ur0, ur0, chunks, q, d0, d1);
-        } else {
-            const uint4* ur1 = u + (long long)col_expert[wib][min(g + 8, ndist - 1)] * vecs;
-            atomic_dot_tiles<2>(xr0, xr1, ur0, ur1, chunks, q, d0, d1);
+        const int col = __popc(nm & ((2u << (lane & (AT_M - 1))) - 1u)) - 1;
+        if (fresh) col_expert[wib][col] = r.e;
+        if (lane < AT_M) {
+            task_slot[wib][lane] = r.s;
+            task_col[wib][lane] = col;
+            task_g[wib][lane] = r.g;
         }
         __syncwarp();
+        const int s0 = task_slot[wib][g], s1 = task_slot[wib][g + 8];
+        const int last = max(ndist - 1, 0);
+        const unsigned char* xr0 = xb + (size_t)(s0 >= 0 ? s0 / a.K : 0) * rowb;
+        const unsigned char* xr1 = xb + (size_t)(s1 >= 0 ? s1 / a.K : 0) * rowb;
+        const unsigned char* ur0 = ub + (size_t)(ndist ? col_expert[wib][min(g, last)] : 0) * rowb;
+        const unsigned char* ur1 = ub + (size_t)(ndist ? col_expert[wib][min(g + 8, last)] : 0) * rowb;
+        r = pa_load(a, un + nw, units, R, cap, lane);   // next unit, in flight meanwhile
+        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ndist > 8) pa_dot<2>(xr0, xr1, ur0, ur1, nsc, q, d0, d1);
+        else pa_dot<1>(xr0, xr1, ur0, ur1, nsc, q, d0, d1);
         // D fragment: d[0], d[1] = row g, columns 2q, 2q+1; d[2], d[3] = row g+8.
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int sr = h ? s1 : s0, kr = h ? k1 : k0;
+            const int sr = task_slot[wib][g + 8 * h], kr = task_col[wib][g + 8 * h];
             if (sr < 0) continue;
             const int tile = kr >> 3, cc = kr & 7;
             if ((cc >> 1) != q) continue;
@@ -328,59 +379,176 @@ __global__ void __launch_bounds__(256, 2) atomic_phase_a_kernel(const AtomicArgs
             const float hi = tile ? d1[2 * h + 1] : d0[2 * h + 1];
             const float dot = (cc & 1) ? hi : lo;
             const float gel = 0.5f * dot * (1.0f + erff(dot * 0.70710678118654752f));
-            a.c[sr] = (h ? g1 : g0) * gel;
+            a.c[sr] = task_g[wib][g + 8 * h] * gel;
         }
     }
 }
 
-// phase B: one warp per token; 4 v rows in flight per lane.
-template <int NV>
-__global__ void __launch_bounds__(256) atomic_phase_b_kernel(const AtomicArgs a)
+// Waits (bounded) for every stage still being filled; used on the way out
+// after a failed wait, so that no copy into this block's shared memory is
+// in flight when it exits.
+template <int NST>
+__device__ __forceinline__ void drain_stages(uint64_t* full, uint32_t pend, uint32_t ph)
 {
+    for (int st = 0; st < NST; ++st)
+        if ((pend >> st) & 1u) mbar_wait(&full[st], (ph >> st) & 1u);
+}
+
+// ---- phase B: y_t = sum_j c[t, j] v_{e_tj}, one warp per token, fp32 in slot order.
+//
+// The token's v rows stream through a warp-private ring of 4 KiB stages
+// (8/NV rows each, one bulk copy per row), three stages ahead and across
+// tokens; lane l accumulates the 16-byte vectors l + 32 i of the row with
+// packed fp32x2 FMAs.
+constexpr int PB_WARPS = 12;
+constexpr int PB_STAGES = 4;
+constexpr int PB_STAGE = 4096;
+
+template <int NV>
+__global__ void __launch_bounds__(PB_WARPS * 32, 1) atomic_phase_b_kernel(const AtomicArgs a)
+{
+    extern __shared__ __align__(16) unsigned char pb_smem[];
+    constexpr int RPS = 8 / NV;          // rows per stage
+    constexpr int ROWB = NV * 512;       // bytes per row
+    const int wib = threadIdx.x >> 5;
+    unsigned char* ring = pb_smem + wib * (PB_STAGES * PB_STAGE);
+    uint64_t* full = reinterpret_cast<uint64_t*>(pb_smem + PB_WARPS * PB_STAGES * PB_STAGE) + wib * PB_STAGES;
     const int lane = threadIdx.x & 31;
-    const uint4* v = reinterpret_cast<const uint4*>(a.v);
-    const int vecs = a.d / 8;
-    const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long t = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += nw) {
-        float acc[NV][8];
+    const int ns = (a.K + RPS - 1) / RPS;
+    const int nw = gridDim.x * PB_WARPS;
+    const int t0 = blockIdx.x * PB_WARPS + wib;
+    if (t0 >= a.T) return;
+    if (lane == 0) {
+        for (int st = 0; st < PB_STAGES; ++st) mbar_init(&full[st], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    const unsigned char* vb = static_cast<const unsigned char*>(a.v);
+
+    auto pick = [](const int (&r)[4], int j) { return j < 32 ? r[0] : j < 64 ? r[1] : j < 96 ? r[2] : r[3]; };
+    auto pickf = [](const float (&r)[4], int j) { return j < 32 ? r[0] : j < 64 ? r[1] : j < 96 ? r[2] : r[3]; };
+    // expert ids of token t (lane + 32 i); an invalid id reads row 0 with weight 0
+    auto load_e = [&](int t, int (&E)[4]) {
 #pragma unroll
-        for (int q = 0; q < NV; ++q)
+        for (int i = 0; i < 4; ++i) {
+            const int j = lane + 32 * i;
+            int e = 0;
+            if (t < a.T && j < a.K) {
+                e = a.idx[(long long)t * a.K + j];
+                if (e < 0 || e >= a.N) e = 0;
+            }
+            E[i] = e;
+        }
+    };
+    auto load_c = [&](int t, float (&C)[4]) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[q][i] = 0.f;
-        for (int j0 = 0; j0 < a.K; j0 += 32) {
-            const int my_e = (j0 + lane < a.K) ? a.idx[t * a.K + j0 + lane] : -1;
-            const float my_c = (j0 + lane < a.K) ? a.c[t * a.K + j0 + lane] : 0.f;
-            const int jn = min(32, a.K - j0);
-            for (int jj = 0; jj < jn; ++jj) {
-                const int e = __shfl_sync(FULL, my_e, jj);
-                const float c = __shfl_sync(FULL, my_c, jj);
-                if (e < 0 || e >= a.N) { if (lane == 0) set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
-                uint4 w[NV];
+        for (int i = 0; i < 4; ++i) {
+            const int j = lane + 32 * i;
+            float c = 0.f;
+            if (t < a.T && j < a.K) {
+                const int e = a.idx[(long long)t * a.K + j];
+                if (e < 0 || e >= a.N) set_status(MOE_ERR_DEVICE_BOUNDS);
+                else c = a.c[(long long)t * a.K + j];
+            }
+            C[i] = c;
+        }
+    };
+
+    uint32_t ph = 0, pend = 0;
+    int ti = t0, ki = 0;
+    int Ei[4], Ep[4];
+    load_e(ti, Ei);
+    load_e(ti + nw, Ep);
+    auto issue = [&](int st) {
+        if (ti >= a.T) return;
+        const int j0 = ki * RPS;
+        const int rows = min(RPS, a.K - j0);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], rows * ROWB);
+        __syncwarp();
+        // lane rr < rows copies row rr of the stage
+        int e = 0;
 #pragma unroll
-                for (int q = 0; q < NV; ++q) w[q] = __ldg(v + (long long)e * vecs + q * 32 + lane);
+        for (int rr = 0; rr < RPS; ++rr) {
+            const int j = min(j0 + rr, a.K - 1);
+            const int er = __shfl_sync(FULL, pick(Ei, j), j & 31);
+            if (lane == rr) e = er;
+        }
+        if (lane < rows) bulk_g2s(ring + st * PB_STAGE + lane * ROWB, vb + (size_t)e * ROWB, ROWB, &full[st]);
+        pend |= 1u << st;
+        if (++ki == ns) {
+            ki = 0;
+            ti += nw;
 #pragma unroll
-                for (int q = 0; q < NV; ++q) {
-                    acc[q][0] = fmaf(c, bf16_lo(w[q].x), acc[q][0]); acc[q][1] = fmaf(c, bf16_hi(w[q].x), acc[q][1]);
-                    acc[q][2] = fmaf(c, bf16_lo(w[q].y), acc[q][2]); acc[q][3] = fmaf(c, bf16_hi(w[q].y), acc[q][3]);
-                    acc[q][4] = fmaf(c, bf16_lo(w[q].z), acc[q][4]); acc[q][5] = fmaf(c, bf16_hi(w[q].z), acc[q][5]);
-                    acc[q][6] = fmaf(c, bf16_lo(w[q].w), acc[q][6]); acc[q][7] = fmaf(c, bf16_hi(w[q].w), acc[q][7]);
+            for (int i = 0; i < 4; ++i) Ei[i] = Ep[i];
+            load_e(ti + nw, Ep);
+        }
+    };
+
+    int tc = t0, kc = 0;
+    float Cc[4], Cp[4];
+    load_c(tc, Cc);
+    load_c(tc + nw, Cp);
+    float acc[NV][8];
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
+    for (int s = 0; s < PB_STAGES - 1; ++s) issue(s);
+    int cons = 0;
+    while (tc < a.T) {
+        const int cst = cons % PB_STAGES;
+        if (!__all_sync(FULL, mbar_wait(&full[cst], (ph >> cst) & 1u))) {
+            drain_stages<PB_STAGES>(full, pend & ~(1u << cst), ph);
+            return;
+        }
+        ph ^= 1u << cst;
+        pend &= ~(1u << cst);
+        const unsigned char* st = ring + cst * PB_STAGE;
+#pragma unroll
+        for (int rr = 0; rr < RPS; ++rr) {
+            const int j = kc * RPS + rr;
+            if (j < a.K) {
+                const float c = __shfl_sync(FULL, pickf(Cc, j), j & 31);
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(st + rr * ROWB + (lane + 32 * v) * 16);
+                    fma2(acc[v][0], acc[v][1], c, bf16_lo(w.x), bf16_hi(w.x));
+                    fma2(acc[v][2], acc[v][3], c, bf16_lo(w.y), bf16_hi(w.y));
+                    fma2(acc[v][4], acc[v][5], c, bf16_lo(w.z), bf16_hi(w.z));
+                    fma2(acc[v][6], acc[v][7], c, bf16_lo(w.w), bf16_hi(w.w));
                 }
             }
         }
-        if (a.out_f32) {
-            float4* y = reinterpret_cast<float4*>(a.y);
+        __syncwarp();
+        issue((cons + PB_STAGES - 1) % PB_STAGES);
+        ++cons;
+        if (++kc == ns) {
+            const int vecs = a.d / 8;
+            if (a.out_f32) {
+                float4* y = reinterpret_cast<float4*>(a.y);
 #pragma unroll
-            for (int q = 0; q < NV; ++q) {
-                const long long o = (t * vecs + q * 32 + lane) * 2;
-                y[o] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
-                y[o + 1] = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
+                for (int v = 0; v < NV; ++v) {
+                    const long long o = ((long long)tc * vecs + v * 32 + lane) * 2;
+                    y[o] = make_float4(acc[v][0], acc[v][1], acc[v][2], acc[v][3]);
+                    y[o + 1] = make_float4(acc[v][4], acc[v][5], acc[v][6], acc[v][7]);
+                }
+            } else {
+                uint4* y = reinterpret_cast<uint4*>(a.y);
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+                    y[(long long)tc * vecs + v * 32 + lane] =
+                        make_uint4(pack_bf16(acc[v][0], acc[v][1]), pack_bf16(acc[v][2], acc[v][3]),
+                                   pack_bf16(acc[v][4], acc[v][5]), pack_bf16(acc[v][6], acc[v][7]));
             }
-        } else {
-            uint4* y = reinterpret_cast<uint4*>(a.y);
 #pragma unroll
-            for (int q = 0; q < NV; ++q)
-                y[t * vecs + q * 32 + lane] = make_uint4(pack_bf16(acc[q][0], acc[q][1]), pack_bf16(acc[q][2], acc[q][3]),
-                                                         pack_bf16(acc[q][4], acc[q][5]), pack_bf16(acc[q][6], acc[q][7]));
+            for (int v = 0; v < NV; ++v)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
+            kc = 0;
+            tc += nw;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) Cc[i] = Cp[i];
+            load_c(tc + nw, Cp);
         }
     }
 }
@@ -399,10 +567,17 @@ moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
     return cuda_status(cudaGetLastError());
 }
 
+constexpr int kPbSmem = PB_WARPS * PB_STAGES * (PB_STAGE + 8);
+
 template <int NV> struct PhaseB {
     static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
     {
-        atomic_phase_b_kernel<NV><<<grid, 256, 0, st>>>(a);
+        static bool attr_done = false;
+        if (!attr_done) {
+            cudaFuncSetAttribute(atomic_phase_b_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPbSmem);
+            attr_done = true;
+        }
+        atomic_phase_b_kernel<NV><<<grid, PB_WARPS * 32, kPbSmem, st>>>(a);
     }
 };
 
@@ -425,12 +600,13 @@ moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st)
     const long long cap = (long long)a.T * a.K;
     if (cap == 0) return MOE_OK;
     if (a.d % 256 != 0) return MOE_ERR_UNSUPPORTED;
-    const int g0 = (int)std::min<long long>((a.N + 255) / 256, num_sms() * 8);
-    atomic_task_expert_kernel<<<std::max(1, g0), 256, 0, st>>>(a.offsets, a.N, cap, a.task_expert);
+    const long long n = std::max((long long)a.N, cap);
+    const int g0 = (int)std::max(1LL, std::min<long long>((n + 255) / 256, num_sms() * 8));
+    atomic_task_meta_kernel<<<g0, 256, 0, st>>>(a);
     count_launch();
     const long long units = (cap + AT_M - 1) / AT_M;
-    const int grid = (int)std::max(1LL, std::min<long long>((units + 7) / 8, num_sms() * 2));
-    atomic_phase_a_kernel<<<grid, 256, 0, st>>>(a);
+    const int grid = (int)std::max(1LL, std::min<long long>((units + PA_WARPS - 1) / PA_WARPS, num_sms() * MOE_PA_MINB));
+    atomic_phase_a_kernel<<<grid, PA_WARPS * 32, 0, st>>>(a);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
@@ -438,7 +614,8 @@ moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st)
 moe_status launch_atomic_phase_b(const AtomicArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
-    const int grid = std::max(1, std::min(cdiv(a.T, 8), num_sms() * 16));
+    if (a.K > 128) return MOE_ERR_UNSUPPORTED;
+    const int grid = std::max(1, std::min(cdiv(a.T, PB_WARPS), num_sms()));
     return launch_nv<PhaseB>(a.d / 256, grid, st, a);
 }
 

@@ -42,6 +42,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only), and its groups.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer()
 {
     uint64_t t;
@@ -104,6 +113,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 }
 
 // ------------------------------------------------------------ TMA
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, counted on
+// `bar` in bytes.  No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// acc[0..1] += c * (w0, w1) with one packed fp32x2 FMA.
+__device__ __forceinline__ void fma2(float& a0, float& a1, float c, float w0, float w1)
+{
+    asm("{\n\t.reg .b64 d, x, y;\n\t"
+        "mov.b64 x, {%2, %2};\n\t"
+        "mov.b64 y, {%3, %4};\n\t"
+        "mov.b64 d, {%0, %1};\n\t"
+        "fma.rn.f32x2 d, x, y, d;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(c), "f"(w0), "f"(w1));
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

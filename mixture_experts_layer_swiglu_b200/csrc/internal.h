@@ -118,6 +118,7 @@ struct AtomicArgs {
     const int32_t* offsets;
     const int32_t* token_of;   // task -> slot id
     int32_t* task_expert;      // task -> expert (scratch, written by phase A's first kernel)
+    float* task_gate;          // task -> gate of its slot (scratch, same kernel)
     const int32_t* idx;        // [T, K]
     const float* gate;         // [T, K]
     float* c;                  // [T*K]

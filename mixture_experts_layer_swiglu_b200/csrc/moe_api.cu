@@ -105,7 +105,7 @@ Scratch scratch_sizes(const moe_layer_desc* d)
                   al((size_t)2 * d->T * d->pk_rows * 4);
         const size_t N = (size_t)d->pk_rows * d->pk_cols;
         s.permute = al(N * 4) * 2 + al((size_t)atomic_scan_blocks((int)N) * 4);
-        s.ffn = al((size_t)d->T * d->top_k * 4);
+        s.ffn = 2 * al((size_t)d->T * d->top_k * 4);
     }
     return s;
 }
@@ -372,6 +372,7 @@ moe_status ffn_impl(const moe_layer_desc* d, const moe_layer_weights* w, const v
     AtomicArgs a{};
     a.x = x;
     a.task_expert = static_cast<int32_t*>(ws);
+    a.task_gate = reinterpret_cast<float*>(static_cast<char*>(ws) + al((size_t)d->T * d->top_k * 4));
     a.u = w->u;
     a.v = w->v;
     a.offsets = offsets;

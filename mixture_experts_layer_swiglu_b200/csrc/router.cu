@@ -90,13 +90,6 @@ constexpr int R_STAGES = 4;
 constexpr int R_W_BYTES = 8 * 4096;          // 8 router rows of <= 4 KiB (resident tiles)
 constexpr int R_SMEM = R_STAGES * R_TILE * R_CHUNK_BYTES + 2 * R_W_BYTES + R_WARPS * R_TPW * R_MAXROWS * 4;
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <typename Tin>
 __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a)
