@@ -254,20 +254,20 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     stream = torch.cuda.current_stream(dev)
     atomic = cfg.kind == "atomic"
 
-    def calls():
-        c = [lambda: moe.moe_route(desc, ws, x, zp, None, b.idx, b.gate, cm, b.workspace, stream),
+    def calls(st=stream):
+        c = [lambda: moe.moe_route(desc, ws, x, zp, None, b.idx, b.gate, cm, b.workspace, st),
              lambda: moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace,
-                                     stream)]
+                                     st)]
         if atomic:
             c.append(lambda: moe.moe_grouped_ffn(desc, ws, None, b.offsets, b.token_of, x, b.gate, b.y_sorted,
-                                                 b.workspace, stream))
+                                                 b.workspace, st))
         else:
             c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 1, b.x_sorted, b.offsets, b.y_sorted,
-                                                       b.workspace, stream))
+                                                       b.workspace, st))
             c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 2, b.x_sorted, b.offsets, b.y_sorted,
-                                                       b.workspace, stream))
+                                                       b.workspace, st))
         c.append(lambda: moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, cm, x, b.y,
-                                         stream))
+                                         st))
         return c
 
     stage_calls = calls()
@@ -319,6 +319,9 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     R_ffn = int(off[cfg.n_ffn].item()) if not atomic else R_total
     touched = int((off[1:] > off[:-1]).sum().item()) if atomic else 0
 
+    graph_ms = graph_step_ms(calls, stream, flush, sleep_cycles, K)
+    assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+
     # end to end through the public call with host buffers
     x_host = a_cpu["x"].pin_memory()
     y_host = torch.empty(x_host.shape, dtype=x_host.dtype).pin_memory()
@@ -351,8 +354,9 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         cublas = library_reference(cfg, R_total, dev)
 
     mean = {n: sum(v) / K for n, v in per.items()}
-    red = reduce_max_over_ranks(dist, [total_ms, e2e_ms / KE] + [mean[n] for n in names], dev)
-    res = {"total_ms": red[0], "e2e_ms": red[1], "mean": {n: red[2 + j] for j, n in enumerate(names)}}
+    red = reduce_max_over_ranks(dist, [total_ms, e2e_ms / KE, graph_ms] + [mean[n] for n in names], dev)
+    res = {"total_ms": red[0], "e2e_ms": red[1], "graph_ms": red[2],
+           "mean": {n: red[3 + j] for j, n in enumerate(names)}}
     if rank != 0:
         return None
 
@@ -410,6 +414,9 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         "e2e": {"value": round(job_value(world, cfg.T, res["e2e_ms"]), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "moe_layer_forward, x from pinned host, y to pinned host"},
+        "graph": {"ms_per_step": round(res["graph_ms"], 4),
+                  "value": round(job_value(world, cfg.T, res["graph_ms"]), 1), "unit": "tokens/s",
+                  "how": "the same step captured once in a CUDA graph and replayed; L2 flushed before each replay"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
@@ -419,6 +426,35 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         w_cpu.update(a_cpu)
         out["cpu_baseline"] = cpu_oracle_leg(cfg, w_cpu, args.oracle_tokens)
     return out
+
+
+def graph_step_ms(calls, stream, flush, sleep_cycles: int, K: int) -> float:
+    """Mean device time of one step replayed from a CUDA graph (the step's
+    launches captured once), timed like the eager steps: L2 flush and a GPU
+    sleep before each replay, CUDA events around it."""
+    side = torch.cuda.Stream(device=stream.device)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for f in calls(side):      # warm the capture stream's path once
+            f()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for f in calls(side):
+            f()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        torch.cuda._sleep(sleep_cycles)
+        evs[i][0].record(stream)
+        g.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    del g
+    return ms
 
 
 def library_reference(cfg, R_total: int, dev) -> dict:

@@ -122,6 +122,36 @@ def test_layer_forward_equals_stages():
     assert torch.equal(y, r["bufs"].y)
 
 
+@pytest.mark.parametrize("name,T,changes", [("moepp", 700, {"hidden": 640}), ("atomic", 300, {})])
+def test_cuda_graph_replay_matches_eager(name, T, changes):
+    """The layer's launches captured once in a CUDA graph and replayed give
+    the eager result bit for bit, also after the input changes in place."""
+    cfg = scaled(get_config(name), T=T, **changes)
+    inp = to_device(make_inputs(cfg))
+    layer = moe.MoELayer(moe.desc_from(cfg), inp)
+    x, zp = inp["x"], inp.get("z_prev")
+    y = layer.forward(x, prev_logits=zp)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.forward(x, prev_logits=zp, y=y)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, prev_logits=zp, y=y)
+    for trial in range(2):
+        if trial:
+            x.copy_(torch.roll(x, shifts=1, dims=0))
+        ref = layer.forward(x, prev_logits=zp).clone()
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref)
+    del g
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
 def test_invalid_expert_id_sets_bounds_status():
     cfg = scaled(get_config("mixtral"), T=64, d=256, hidden=256, n_ffn=4)
     inp = to_device(make_inputs(cfg))
