@@ -48,7 +48,13 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 192;
 constexpr int SMEM_TABLE_INTS = 3 * kMaxGemmGroups + 1;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + SMEM_TABLE_INTS * 4;
+constexpr int EPI_STAGE_BYTES = 32 * 128;      // one 32-row x 128-byte output box per epilogue warp
+constexpr int EPI_WARPS = 4;
+__host__ __device__ constexpr int epi_stage_offset(int stage_bytes)
+{
+    return ((stage_bytes + 256 + SMEM_TABLE_INTS * 4) + 1023) / 1024 * 1024;
+}
+constexpr int SMEM_BYTES = 1024 + epi_stage_offset(STAGES * STAGE_BYTES) + EPI_WARPS * EPI_STAGE_BYTES;
 
 struct DevArgs {
     const int32_t* offsets;
@@ -192,6 +198,97 @@ __device__ __forceinline__ void epilogue_tile(const DevArgs& a, uint32_t tacc, c
     }
 }
 
+// The epilogue of one warp's 32 rows when all of them are valid: each
+// 128-byte column chunk of the 32 rows (32 fp32 or 64 bf16 values per row)
+// is written into the warp's 4 KiB staging box in the 128-byte swizzled
+// layout (16-byte unit j of row r at unit j ^ (r & 7): conflict-free) and
+// stored with one TMA store, so global memory sees whole lines instead of
+// one 16-byte piece per row per instruction.  The next chunk's TMEM load
+// overlaps the wait for the previous store to finish reading the box.
+// Blocks with invalid rows (the end of a group) take epilogue_tile.
+template <int EPI>
+__device__ __forceinline__ void epilogue_block_tma(const DevArgs& a, const CUtensorMap* tm_out, uint32_t tacc,
+                                                   const TileInfo& ti, int q, int lane, uint8_t* box)
+{
+    if (ti.rows < q * 32 + 32) {
+        epilogue_tile<EPI>(a, tacc, ti, q * 32 + lane);
+        return;
+    }
+    const int row = ti.row0 + q * 32;
+    uint4* mine = reinterpret_cast<uint4*>(box + lane * 128);
+    auto put = [&](const uint32_t (&w)[32], int col) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mine[j ^ (lane & 7)] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tm_out, box, col, row);
+            bulk_commit();
+        }
+    };
+    if constexpr (EPI == EPI_SWIGLU) {
+        const int col0 = ti.n * 128;
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t w[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c = 2 * c2 + hh;
+                uint32_t g[32], u[32];
+                tmem_ld32(tacc + c * 32, g);
+                tmem_ld32(tacc + 128 + c * 32, u);
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                    const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                    w[16 * hh + i] = pack_bf16(g0 / (1.0f + __expf(-g0)) * u0, g1 / (1.0f + __expf(-g1)) * u1);
+                }
+            }
+            put(w, col0 + c2 * 64);
+        }
+    } else if constexpr (EPI == EPI_BF16) {
+        const int col0 = ti.n * 256;
+#pragma unroll 1
+        for (int c2 = 0; c2 < 4; ++c2) {
+            if (col0 + c2 * 64 >= a.N) break;
+            uint32_t w[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v[32];
+                tmem_ld32(tacc + (2 * c2 + hh) * 32, v);
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[16 * hh + i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            put(w, col0 + c2 * 64);
+        }
+    } else {   // EPI_F32
+        const int col0 = ti.n * 256;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+            if (col0 + c * 32 >= a.N) break;
+            uint32_t v[32];
+            tmem_ld32(tacc + c * 32, v);
+            tc_wait_ld();
+            put(v, col0 + c * 32);
+        }
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_any(const DevArgs& a, const CUtensorMap* tm_out, uint32_t tacc,
+                                             const TileInfo& ti, int q, int lane, uint8_t* box)
+{
+    // the split query keeps direct stores: its three parts per chunk would
+    // serialise on the one staging box (measured slower)
+    if constexpr (EPI == EPI_PK_SPLIT) epilogue_tile<EPI>(a, tacc, ti, q * 32 + lane);
+    else epilogue_block_tma<EPI>(a, tm_out, tacc, ti, q, lane, box);
+}
+
 // Warp 0 builds, for every group, its first row, its row count and the index
 // of its first output tile (tiles of TBM rows x one n-tile).
 template <int TBM>
@@ -230,7 +327,8 @@ template <int EPI>
 __global__ void __launch_bounds__(NTHREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-                    const __grid_constant__ CUtensorMap tmB3, const DevArgs a)
+                    const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmOut,
+                    const DevArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -343,7 +441,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;            // row of the tile
+        uint8_t* epi_box = smem + epi_stage_offset(STAGES * STAGE_BYTES) + (warp - 2) * EPI_STAGE_BYTES;
         int acc = 0;
         uint32_t aph = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -351,11 +449,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (*abort_flag || !mbar_wait(&acc_full[acc], aph)) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
-            epilogue_tile<EPI>(a, tacc, ti, r);
+            epilogue_any<EPI>(a, &tmOut, tacc, ti, q, lane, epi_box);
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
             if (++acc == 2) { acc = 0; aph ^= 1; }
         }
+        if (lane == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -396,13 +495,15 @@ constexpr int P_HALF = 128 * BK * 2;         // one 128-row x 64-K box: 16 KB
 constexpr int P_TILE_A = P_KH * P_HALF;      // A: 128 rows x 64*KH of K
 constexpr int P_TILE_B = P_KH * P_HALF;
 constexpr int P_STAGE_BYTES = P_TILE_A + P_TILE_B;
-constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + SMEM_TABLE_INTS * 4;
+constexpr int P_SMEM_BYTES = 1024 + epi_stage_offset(P_STAGES * P_STAGE_BYTES) + EPI_WARPS * EPI_STAGE_BYTES;
+static_assert(SMEM_BYTES <= 232448 && P_SMEM_BYTES <= 232448, "shared memory per block");
 
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-                         const __grid_constant__ CUtensorMap tmB3, const DevArgs a)
+                         const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmOut,
+                         const DevArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -529,7 +630,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
-        const int r = q * 32 + lane;
+        uint8_t* epi_box = smem + epi_stage_offset(P_STAGES * P_STAGE_BYTES) + (warp - 2) * EPI_STAGE_BYTES;
         int acc = 0;
         uint32_t aph = 0;
         for (int tile = cluster; tile < total; tile += n_clusters) {
@@ -539,12 +640,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             if (*abort_flag || !mbar_wait(&acc_full[acc], aph)) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
-            epilogue_tile<EPI>(a, tacc, ti, r);
+            epilogue_any<EPI>(a, &tmOut, tacc, ti, q, lane, epi_box);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8 * acc);
             if (++acc == 2) { acc = 0; aph ^= 1; }
         }
+        if (lane == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -594,10 +696,27 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int K)
     return r == CUDA_SUCCESS;
 }
 
+// Output [rows, N] (row stride ldo elements) as boxes of 32 rows x 128 bytes,
+// 128-byte swizzle, for the TMA-store epilogues.
+bool make_out_map(CUtensorMap* m, void* base, long long rows, int N, long long ldo, bool f32)
+{
+    EncodeTiledFn enc = get_encode();
+    if (!enc || !base || rows <= 0) return false;
+    const int elt = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ldo * elt};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elt), 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int EPI>
 moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
 {
-    CUtensorMap mA, m0, m1, m2, m3;
+    CUtensorMap mA, m0, m1, m2, m3, mo;
     const void* b1 = p.B1 ? p.B1 : p.B0;
     const void* b2 = p.B2 ? p.B2 : p.B0;
     const void* b3 = p.B3 ? p.B3 : (p.B2 ? p.B2 : b1);
@@ -605,6 +724,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, p.K) ||
         !make_map(&m1, b1, p.b01_rows, p.K) || !make_map(&m2, b2, r23, p.K) ||
         !make_map(&m3, b3, r23, p.K))
+        return MOE_ERR_CUDA;
+    if (EPI == EPI_PK_SPLIT) mo = mA;   // direct stores; the map is unused
+    else if (!make_out_map(&mo, p.out, std::min<long long>(p.rows_cap, 1ll << 31), p.N, p.ldo, EPI == EPI_F32))
         return MOE_ERR_CUDA;
     static bool attr_done = false, attr_pair_done = false;
     DevArgs a;
@@ -630,7 +752,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
         }
         const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
         const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
-        grouped_gemm_pair_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+        grouped_gemm_pair_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, mo, a);
     } else {
         if (!attr_done) {
             cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
@@ -640,7 +762,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
         }
         const long long tiles_ub = (long long)(cdiv((int)rows, BM) + p.n_groups) * ntn;
         const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms()));
-        grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+        grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, mo, a);
     }
     count_launch();
     return cuda_status(cudaGetLastError());

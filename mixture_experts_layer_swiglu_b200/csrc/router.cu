@@ -371,8 +371,12 @@ template <int MAXV> struct PkWarpSmem {
 // i < kh walks row candidate i along the sorted columns, so its next
 // candidate is always its best remaining one, and the best of the lanes'
 // heads is the best remaining pair.
+#ifndef MOE_PK_MINB
+#define MOE_PK_MINB 3     // resident blocks of 8 warps per SM
+#endif
+
 template <int MAXV>
-__global__ void __launch_bounds__(256) pk_select_kernel(const PkSelectArgs a)
+__global__ void __launch_bounds__(256, MOE_PK_MINB) pk_select_kernel(const PkSelectArgs a)
 {
     extern __shared__ __align__(16) unsigned char pk_smem[];
     const int lane = threadIdx.x & 31;
@@ -485,7 +489,7 @@ moe_status launch_pk_select(const PkSelectArgs& a, cudaStream_t st)
                              warps * (int)sizeof(PkWarpSmem<32>));
         attr_done = true;
     }
-    const int grid = std::max(1, std::min(cdiv(a.T, warps), num_sms() * 4));
+    const int grid = std::max(1, std::min(cdiv(a.T, warps), num_sms() * MOE_PK_MINB));
     const int n = std::max(a.rows, a.cols);
     if (n <= 512) pk_select_kernel<16><<<grid, warps * 32, warps * sizeof(PkWarpSmem<16>), st>>>(a);
     else pk_select_kernel<32><<<grid, warps * 32, warps * sizeof(PkWarpSmem<32>), st>>>(a);
