@@ -217,8 +217,11 @@ def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
         return {
             "router": ("tensor", 2.0 * T * d * dq + 2.0 * (2 * T) * (1.5 * dq) * cfg.pk_rows),
             "permute": ("hbm", T * k * 4 * 6 + N * 4 * 5),
-            "expert_dot": ("hbm", touched * d * e + T * k * 12),
-            "expert_combine": ("hbm", T * k * d * e + T * k * 8 + T * d * e),
+            # each touched expert's u (phase A) and v (phase B) row once, x read
+            # once, y written once (the token-centric phase B moves more: it
+            # gathers a v row per slot, with L2 hits for rows shared in time)
+            "expert_dot": ("hbm", touched * d * e + T * d * e + T * k * 12),
+            "expert_combine": ("hbm", touched * d * e + T * d * e + T * k * 8),
         }
     H = cfg.hidden
     E_r = cfg.n_routed

@@ -59,6 +59,7 @@ constexpr int SMEM_BYTES = 1024 + epi_stage_offset(STAGES * STAGE_BYTES) + EPI_W
 struct DevArgs {
     const int32_t* offsets;
     int n_groups, n_first, group_rows, N, K;
+    int b_kmod;                 // > 0: B's k coordinate is k mod b_kmod
     void* out;
     long long ldo;
     long long rows_cap;
@@ -397,8 +398,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     armed &= ~(1u << s);
                     mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
                     tma_load_2d(sA + s * TILE_A, &tmA, &full[s], kb * BK, ti.row0);
-                    tma_load_2d(sB + s * TILE_B, mlo, &full[s], kb * BK, brow_lo);
-                    tma_load_2d(sB + s * TILE_B + TILE_B / 2, mhi, &full[s], kb * BK, brow_hi);
+                    const int kbb = a.b_kmod ? (kb * BK) % a.b_kmod : kb * BK;
+                    tma_load_2d(sB + s * TILE_B, mlo, &full[s], kbb, brow_lo);
+                    tma_load_2d(sB + s * TILE_B + TILE_B / 2, mhi, &full[s], kbb, brow_hi);
                     armed |= 1u << s;
                     arm_par = (arm_par & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -579,7 +581,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     for (int h = 0; h < P_KH; ++h) {
                         const int k0 = (kb * P_KH + h) * BK;      // past K: zero fill
                         tma_load_2d_pair(sA + s * P_TILE_A + h * P_HALF, &tmA, full_leader + 8 * s, k0, arow);
-                        tma_load_2d_pair(sB + s * P_TILE_B + h * P_HALF, mb, full_leader + 8 * s, k0, brow);
+                        tma_load_2d_pair(sB + s * P_TILE_B + h * P_HALF, mb, full_leader + 8 * s,
+                                         a.b_kmod ? k0 % a.b_kmod : k0, brow);
                     }
                     if (++s == P_STAGES) { s = 0; ph ^= 1; }
                 }
@@ -721,9 +724,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     const void* b2 = p.B2 ? p.B2 : p.B0;
     const void* b3 = p.B3 ? p.B3 : (p.B2 ? p.B2 : b1);
     const long long r23 = p.B2 ? p.b23_rows : p.b01_rows;
-    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, p.K) ||
-        !make_map(&m1, b1, p.b01_rows, p.K) || !make_map(&m2, b2, r23, p.K) ||
-        !make_map(&m3, b3, r23, p.K))
+    const int kb = p.b_kmod > 0 ? p.b_kmod : p.K;   // B's own K extent
+    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, kb) ||
+        !make_map(&m1, b1, p.b01_rows, kb) || !make_map(&m2, b2, r23, kb) || !make_map(&m3, b3, r23, kb))
         return MOE_ERR_CUDA;
     if (EPI == EPI_PK_SPLIT) mo = mA;   // direct stores; the map is unused
     else if (!make_out_map(&mo, p.out, std::min<long long>(p.rows_cap, 1ll << 31), p.N, p.ldo, EPI == EPI_F32))
@@ -736,6 +739,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     a.group_rows = p.group_rows;
     a.N = p.N;
     a.K = p.K;
+    a.b_kmod = p.b_kmod;
     a.out = p.out;
     a.ldo = p.ldo;
     a.rows_cap = p.rows_cap;

@@ -49,6 +49,7 @@ struct GemmProblem {
     int pk_T;             // EPI_PK_SPLIT: tokens
     int pk_dq;            // EPI_PK_SPLIT: query width
     int pair;             // 1: 256-row tiles on CTA pairs (cta_group::2); 0: 128-row tiles per CTA
+    int b_kmod;           // > 0: B has b_kmod columns and is repeated along K (B k = k mod b_kmod)
 };
 
 moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st);
@@ -89,7 +90,6 @@ struct PermuteArgs {
     int32_t* token_of;
     void* x_sorted;
     int32_t* ws_counts;   // [n_blocks, n_ffn] (SwiGLU) or [N] (atomic)
-    int32_t* ws_cursor;   // atomic: [N]
     int32_t* ws_blocksum; // atomic scan: [scan blocks]
     int T, k, d, n_ffn, n_shared, n_ids, elt_bytes;
 };

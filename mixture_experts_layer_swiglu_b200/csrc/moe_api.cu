@@ -104,7 +104,7 @@ Scratch scratch_sizes(const moe_layer_desc* d)
         s.route = al((size_t)2 * d->T * 3 * half * 2) + al((size_t)(d->pk_rows + d->pk_cols) * 3 * half * 2) +
                   al((size_t)2 * d->T * d->pk_rows * 4);
         const size_t N = (size_t)d->pk_rows * d->pk_cols;
-        s.permute = al(N * 4) * 2 + al((size_t)atomic_scan_blocks((int)N) * 4);
+        s.permute = al(N * 4) + al((size_t)atomic_scan_blocks((int)N) * 4);
         s.ffn = 2 * al((size_t)d->T * d->top_k * 4);
     }
     return s;
@@ -198,8 +198,15 @@ moe_status route_impl(const moe_layer_desc* d, const moe_layer_weights* w, const
     void* w3 = p;
     p += al((size_t)(d->pk_rows + d->pk_cols) * 3 * half * 2);
     float* scores = reinterpret_cast<float*>(p);
-    moe_status s = launch_pk_prep_keys(w->subkeys_row, w->subkeys_col, w3, d->pk_rows, d->pk_cols, half, st);
-    if (s != MOE_OK) return s;
+    // The score GEMM's B operand is [K|K|K] along k (one copy per bf16 part
+    // of q).  When a copy spans whole 64-wide k blocks the GEMM reads the
+    // sub-keys directly with k taken mod half; otherwise it reads a tripled
+    // copy built here.
+    const bool kmod = half % 64 == 0;
+    moe_status s = MOE_OK;
+    if (!kmod && (s = launch_pk_prep_keys(w->subkeys_row, w->subkeys_col, w3, d->pk_rows, d->pk_cols, half, st)) !=
+                     MOE_OK)
+        return s;
     GemmProblem q{};
     q.epi = EPI_PK_SPLIT;
     q.A = x;
@@ -224,11 +231,20 @@ moe_status route_impl(const moe_layer_desc* d, const moe_layer_weights* w, const
     g.A = a3;
     g.a_rows = 2ll * d->T;
     g.K = 3 * half;
-    g.B0 = w3;
-    g.b01_rows = d->pk_rows + d->pk_cols;
+    if (kmod) {                 // group 0: row sub-keys, group 1: column sub-keys
+        g.B0 = w->subkeys_row;
+        g.b01_rows = d->pk_rows;
+        g.B2 = w->subkeys_col;
+        g.b23_rows = d->pk_cols;
+        g.n_first = 1;
+        g.b_kmod = half;
+    } else {
+        g.B0 = w3;
+        g.b01_rows = d->pk_rows + d->pk_cols;
+        g.n_first = 2;
+    }
     g.offsets = nullptr;
     g.n_groups = 2;
-    g.n_first = 2;
     g.group_rows = d->T;
     g.N = d->pk_rows;
     g.out = scores;
@@ -278,8 +294,7 @@ moe_status permute_impl(const moe_layer_desc* d, const int32_t* idx, const void*
     const size_t N = (size_t)d->pk_rows * d->pk_cols;
     char* p = static_cast<char*>(ws);
     a.ws_counts = reinterpret_cast<int32_t*>(p);
-    a.ws_cursor = reinterpret_cast<int32_t*>(p + al(N * 4));
-    a.ws_blocksum = reinterpret_cast<int32_t*>(p + 2 * al(N * 4));
+    a.ws_blocksum = reinterpret_cast<int32_t*>(p + al(N * 4));
     a.n_ffn = 0;
     a.n_shared = 0;
     a.n_ids = (int)N;

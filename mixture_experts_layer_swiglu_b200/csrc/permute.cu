@@ -175,7 +175,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int32_t* __restr
 
 __global__ void zero_i32_kernel(int32_t* p, long long n)
 {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+    const long long n4 = n / 4;   // p is 16-byte aligned
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x)
+        reinterpret_cast<int4*>(p)[i] = make_int4(0, 0, 0, 0);
+    for (long long i = n4 * 4 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x)
         p[i] = 0;
 }
@@ -232,31 +236,23 @@ __global__ void __launch_bounds__(1024) atomic_scan1_kernel(const int32_t* count
     if (threadIdx.x == 0) blocksum[blockIdx.x] = tot;
 }
 
-// pass 2: exclusive scan of the block totals (one block; nb <= 1024 * 4)
-__global__ void __launch_bounds__(1024) atomic_scan2_kernel(int32_t* blocksum, int nb)
-{
-    __shared__ int wt[32];
-    __shared__ int tot;
-    const int base = threadIdx.x * 4;
-    int v[4], s = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) { v[i] = (base + i < nb) ? blocksum[base + i] : 0; s += v[i]; }
-    int run = block_excl_scan_1024(s, wt, &tot);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) if (base + i < nb) { blocksum[base + i] = run; run += v[i]; }
-}
-
-// pass 3: offsets[e] = block base + exclusive scan inside the block
-__global__ void __launch_bounds__(1024) atomic_scan3_kernel(const int32_t* counts, int N,
+// pass 2: offsets[e] = (sum of the totals of the blocks before this one) +
+// exclusive scan inside the block; each block sums the preceding totals
+// itself (nb <= 4096), so no third pass is needed.
+__global__ void __launch_bounds__(1024) atomic_scan2_kernel(const int32_t* counts, int N,
                                                             const int32_t* blocksum, int32_t* offsets)
 {
     __shared__ int wt[32];
     __shared__ int tot;
+    int pre = 0;
+    for (int i = threadIdx.x; i < (int)blockIdx.x; i += blockDim.x) pre += blocksum[i];
+    block_excl_scan_1024(pre, wt, &tot);
+    const int base_sum = tot;                  // sum of all preceding block totals
     const long long base = (long long)blockIdx.x * SCAN_ELEMS + threadIdx.x * 4;
     int v[4], s = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) { v[i] = (base + i < N) ? counts[base + i] : 0; s += v[i]; }
-    int run = blocksum[blockIdx.x] + block_excl_scan_1024(s, wt, &tot);
+    int run = base_sum + block_excl_scan_1024(s, wt, &tot);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         if (base + i < N) offsets[base + i] = run;
@@ -272,7 +268,7 @@ __global__ void atomic_place_kernel(const PermuteArgs a)
          s += (long long)gridDim.x * blockDim.x) {
         const int e = a.idx[s];
         if (e < 0 || e >= a.n_ids) { a.row_of[s] = -1; continue; }
-        const int pos = a.offsets[e] + atomicAdd(&a.ws_cursor[e], 1);
+        const int pos = a.offsets[e] + atomicSub(&a.ws_counts[e], 1) - 1;   // any order; sorted next
         a.token_of[pos] = (int)s;
     }
 }
@@ -328,17 +324,14 @@ moe_status launch_permute_atomic(const PermuteArgs& a, cudaStream_t st)
 {
     const int N = a.n_ids;
     const int grid_n = std::max(1, std::min(cdiv(N, 256), num_sms() * 8));
-    zero_i32_kernel<<<grid_n, 256, 0, st>>>(a.ws_counts, N);
-    zero_i32_kernel<<<grid_n, 256, 0, st>>>(a.ws_cursor, N);
-    count_launch(2);
+    zero_i32_kernel<<<std::max(1, std::min(cdiv(N, 1024), num_sms() * 4)), 256, 0, st>>>(a.ws_counts, N);
     const long long n = (long long)a.T * a.k;
     const int grid_t = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, num_sms() * 8));
     atomic_count_kernel<<<grid_t, 256, 0, st>>>(a);
     const int nb = atomic_scan_blocks(N);
     if (nb > 4096) return MOE_ERR_UNSUPPORTED;
     atomic_scan1_kernel<<<nb, 1024, 0, st>>>(a.ws_counts, N, a.ws_blocksum);
-    atomic_scan2_kernel<<<1, 1024, 0, st>>>(a.ws_blocksum, nb);
-    atomic_scan3_kernel<<<nb, 1024, 0, st>>>(a.ws_counts, N, a.ws_blocksum, a.offsets);
+    atomic_scan2_kernel<<<nb, 1024, 0, st>>>(a.ws_counts, N, a.ws_blocksum, a.offsets);
     atomic_place_kernel<<<grid_t, 256, 0, st>>>(a);
     atomic_sort_kernel<<<grid_n, 256, 0, st>>>(a);
     count_launch(6);

@@ -325,43 +325,75 @@ __device__ __forceinline__ void sort_desc(unsigned long long (&c)[MAXV])
             }
 }
 
-// Best kh of the n scores s[0..n) (kh <= n), best first, into out_v / out_i.
-// Lane l owns elements l + 32 i, sorts them, and keeps all but its current
-// head in `list` ([MAXV][32], this warp's); each step the warp takes the
-// best head and only the winning lane advances.
-template <int MAXV>
-__device__ __forceinline__ void select_half(const float* s, int n, int kh, int lane,
-                                            unsigned long long* list, float* out_v, int* out_i)
+// Walk of the candidates list[0..C): lane l sorts candidates l + 32 j
+// (j < SZ) in registers; each step the warp takes the best lane head (two
+// __reduce_max_sync on the 64-bit key) and the winning lane shifts its list
+// by one (compile-time register indices, no shared-memory round trip).
+template <int SZ>
+__device__ __forceinline__ void walk_half(const unsigned long long* list, int C, int kh, int lane, float* out_v,
+                                          int* out_i)
 {
-    unsigned long long c[MAXV];
+    unsigned long long c[SZ];
 #pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-        const int e = lane + 32 * i;
-        c[i] = e < n ? ((unsigned long long)order_key32(__ldg(s + e)) << 32) | (uint32_t)~e : 0ull;
-    }
-    sort_desc<MAXV>(c);
-#pragma unroll
-    for (int i = 1; i < MAXV; ++i) list[i * 32 + lane] = c[i];
-    __syncwarp();
-    unsigned long long head = c[0];
-    int h = 0;
+    for (int j = 0; j < SZ; ++j) c[j] = (j * 32 + lane < C) ? list[j * 32 + lane] : 0ull;
+    sort_desc<SZ>(c);
     for (int j = 0; j < kh; ++j) {
-        const uint32_t hi = (uint32_t)(head >> 32), lo = (uint32_t)head;
+        const uint32_t hi = (uint32_t)(c[0] >> 32), lo = (uint32_t)c[0];
         const uint32_t m1 = __reduce_max_sync(FULL, hi);
         const uint32_t m2 = __reduce_max_sync(FULL, hi == m1 ? lo : 0u);
         if (hi == m1 && lo == m2) {
             out_v[j] = key32_value(hi);
             out_i[j] = (int)~lo;
-            ++h;
-            head = h < MAXV ? list[h * 32 + lane] : 0ull;
+#pragma unroll
+            for (int q = 0; q + 1 < SZ; ++q) c[q] = c[q + 1];
+            c[SZ - 1] = 0ull;
         }
     }
     __syncwarp();
 }
 
+// Best kh of the n scores s[0..n) (32 <= n, kh <= 32), best first, into
+// out_v / out_i.  Prefilter: each lane's maximum is one score, so at least
+// 32 scores are >= tau = the smallest lane maximum, and the kh-th best score
+// is >= tau; only scores >= tau (about 110 of 512 for random scores) are
+// sorted and walked.
+template <int MAXV>
+__device__ __forceinline__ void select_half(const float* s, int n, int kh, int lane,
+                                            unsigned long long* list, float* out_v, int* out_i)
+{
+    uint32_t k[MAXV];
+    uint32_t mx = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int e = lane + 32 * i;
+        k[i] = e < n ? order_key32(__ldg(s + e)) : 0u;   // valid keys are > 0
+        mx = max(mx, k[i]);
+    }
+    const uint32_t tau = __reduce_min_sync(FULL, mx);
+    const unsigned lt = (1u << lane) - 1u;
+    int C = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const bool take = k[i] >= tau;
+        const unsigned b = __ballot_sync(FULL, take);
+        if (take) list[C + __popc(b & lt)] = ((unsigned long long)k[i] << 32) | (uint32_t)~(lane + 32 * i);
+        C += __popc(b);
+    }
+    __syncwarp();
+    if (C <= 128) walk_half<4>(list, C, kh, lane, out_v, out_i);
+    else if (C <= 256) walk_half<8>(list, C, kh, lane, out_v, out_i);
+    else if (C <= 512) walk_half<16>(list, C, kh, lane, out_v, out_i);
+    else walk_half<32>(list, C, kh, lane, out_v, out_i);
+}
+
+__device__ __forceinline__ double key64_value(unsigned long long k)
+{
+    return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
 template <int MAXV> struct PkWarpSmem {
-    unsigned long long list[MAXV * 32];
-    double sel_v[128];
+    unsigned long long list[MAXV * 32];   // half candidates; then each row's merge candidates
+    unsigned long long sel_k[128];
     int sel_i[128];
     float rv[32], cv[32];
     int ri[32], ci[32];
@@ -370,7 +402,11 @@ template <int MAXV> struct PkWarpSmem {
 // One warp per token.  The merge relies on both halves being sorted: lane
 // i < kh walks row candidate i along the sorted columns, so its next
 // candidate is always its best remaining one, and the best of the lanes'
-// heads is the best remaining pair.
+// heads is the best remaining pair.  A pair (i, j) (ranks in the sorted
+// halves) is dominated by the (i+1)(j+1) pairs (i' <= i, j' <= j), none of
+// which ranks after it (sums of the sorted scores are monotone and the ids
+// order ties the same way), so only pairs with (i+1)(j+1) <= K can be
+// selected: lane i precomputes the keys of its first min(kh, K/(i+1)) pairs.
 #ifndef MOE_PK_MINB
 #define MOE_PK_MINB 3     // resident blocks of 8 warps per SM
 #endif
@@ -393,17 +429,27 @@ __global__ void __launch_bounds__(256, MOE_PK_MINB) pk_select_kernel(const PkSel
         select_half<MAXV>(sr, a.rows, a.kh, lane, w.list, w.rv, w.ri);
         select_half<MAXV>(sc, a.cols, a.kh, lane, w.list, w.cv, w.ci);
 
+        // merge candidates: lane i < kh owns list[off, off + np)
         const bool rowl = lane < a.kh;
+        const int np = rowl ? min(a.kh, a.K / (lane + 1)) : 0;
+        int off = np;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(FULL, off, o);
+            if (lane >= o) off += u;
+        }
+        off -= np;
         const double my_r = rowl ? (double)w.rv[lane] : 0.0;
         const int my_base = rowl ? w.ri[lane] * a.cols : 0;
+        for (int pp = 0; pp < np; ++pp) w.list[off + pp] = order_key64(my_r + (double)w.cv[pp]);
+        __syncwarp();
         int p = 0;
-        double sum = my_r + (double)w.cv[0];
-        unsigned long long key = rowl ? order_key64(sum) : 0ull;
-        uint32_t id = (uint32_t)(my_base + w.ci[0]);
+        unsigned long long key = np > 0 ? w.list[off] : 0ull;
         for (int j = 0; j < a.K; ++j) {
             const uint32_t hi = (uint32_t)(key >> 32), lo = (uint32_t)key;
             const uint32_t m1 = __reduce_max_sync(FULL, hi);
             bool win = hi == m1;
+            const uint32_t id = (uint32_t)(my_base + w.ci[p < a.kh ? p : 0]);
             if (__popc(__ballot_sync(FULL, win)) > 1) {        // equal high words: rare
                 const uint32_t m2 = __reduce_max_sync(FULL, win ? lo : 0u);
                 win = win && lo == m2;
@@ -411,25 +457,20 @@ __global__ void __launch_bounds__(256, MOE_PK_MINB) pk_select_kernel(const PkSel
                 win = win && ~id == m3;
             }
             if (win) {
-                w.sel_v[j] = sum;
+                w.sel_k[j] = key;
                 w.sel_i[j] = (int)id;
-                if (++p < a.kh) {
-                    sum = my_r + (double)w.cv[p];
-                    key = order_key64(sum);
-                    id = (uint32_t)(my_base + w.ci[p]);
-                } else {
-                    key = 0ull;
-                }
+                ++p;
+                key = p < np ? w.list[off + p] : 0ull;
             }
         }
         __syncwarp();
-        const double v0 = w.sel_v[0];
+        const double v0 = key64_value(w.sel_k[0]);
         float ex[4];
         float tot = 0.f;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             const int j = blk * 32 + lane;
-            ex[blk] = (j < a.K) ? expf((float)(w.sel_v[j] - v0)) : 0.f;
+            ex[blk] = (j < a.K) ? expf((float)(key64_value(w.sel_k[j]) - v0)) : 0.f;
             tot += ex[blk];
         }
 #pragma unroll
