@@ -234,6 +234,30 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
                              moe_stream_t stream);
 
 /*
+ * The whole layer from host memory to host memory, for a caller whose tokens
+ * arrive on the host (a serving loop).  The T tokens are processed in
+ * `chunks` consecutive token ranges (0: automatic, 4 for T >= 8192, 2 for
+ * T >= 4096, else 1; at most 8); the host->device copy of range c + 1 and the
+ * device->host copy of range c - 1 run on two internal copy streams while
+ * range c is computed on `stream`, so PCIe transfers overlap the layer.  Every
+ * token's result equals moe_layer_forward's bit for bit (tokens are
+ * independent).  The pages (OmniMoE's serving scenario) name no such call.
+ * x_host [T, d_model] (dtype), prev_logits_host [T, rows of w_router] fp32
+ * (nullable), y_host [T, d_model] (dtype, or fp32 if desc->out_f32): host
+ * memory, page-locked for the copies to overlap (pageable memory works but
+ * serialises).  workspace: device, moe_layer_host_workspace_size bytes.
+ * Asynchronous on `stream`: y_host is complete when `stream` reaches this
+ * point (the internal streams are joined back into `stream`, so the call can
+ * be captured in a CUDA graph).  Calls from several host threads on one
+ * device share the internal streams (correct, but not concurrent).
+ */
+MOE_API int64_t moe_layer_host_workspace_size(const moe_layer_desc* desc, int chunks);
+MOE_API moe_status moe_layer_forward_host(const moe_layer_desc* desc, const moe_layer_weights* w,
+                                          const void* x_host, const float* prev_logits_host,
+                                          void* y_host, int chunks, void* workspace,
+                                          size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute without a workspace, for callers that cannot allocate device
  * memory: for example a plugin inside a host framework that owns all device
  * memory and offers the plugin no allocator, or a service whose device

@@ -10,9 +10,9 @@ from ._abi import (  # noqa: F401
     EXPORTED, MOE_BF16, MOE_ERR_CUDA, MOE_ERR_DEVICE_BOUNDS, MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT,
     MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_EXPERT_ATOMIC_GELU, MOE_EXPERT_SWIGLU, MOE_F32, MOE_OK,
     MoEError, MoELayerDesc, MoELayerWeights, moe_combine, moe_get_device_status, moe_grouped_ffn,
-    moe_grouped_ffn_phase, moe_last_launch_count, moe_layer_forward, moe_layer_workspace_size,
-    moe_num_groups, moe_permute, moe_permute_static, moe_route, moe_selftest_wait_timeout, moe_row_capacity, moe_workspace_size, status_string,
-    weights_struct)
+    moe_grouped_ffn_phase, moe_last_launch_count, moe_layer_forward, moe_layer_forward_host,
+    moe_layer_host_workspace_size, moe_layer_workspace_size, moe_num_groups, moe_permute, moe_permute_static,
+    moe_route, moe_row_capacity, moe_selftest_wait_timeout, moe_workspace_size, status_string, weights_struct)
 from .layer import (MoELayer, StageBuffers, desc_from, make_desc, out_dtype, run_stages,  # noqa: F401
                     torch_dtype)
 

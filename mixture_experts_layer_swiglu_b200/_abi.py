@@ -23,7 +23,8 @@ MOE_EXPERT_SWIGLU, MOE_EXPERT_ATOMIC_GELU = 0, 1
 EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_layer_workspace_size",
             "moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
             "moe_layer_forward", "moe_get_device_status", "moe_status_string",
-            "moe_last_launch_count", "moe_permute_static", "moe_selftest_wait_timeout")
+            "moe_last_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
+            "moe_layer_host_workspace_size", "moe_layer_forward_host")
 
 
 class MoEError(RuntimeError):
@@ -70,13 +71,16 @@ def load(path: Path | str | None = None):
     L.moe_grouped_ffn_phase.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, SZ, VP]
     L.moe_combine.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, VP, VP]
     L.moe_layer_forward.argtypes = [D, W, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_layer_host_workspace_size.argtypes = [D, ctypes.c_int]
+    L.moe_layer_host_workspace_size.restype = I64
+    L.moe_layer_forward_host.argtypes = [D, W, VP, VP, VP, ctypes.c_int, VP, SZ, VP]
     L.moe_get_device_status.argtypes = [P(ctypes.c_int), ctypes.c_int, VP]
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_launch_count.restype = I32
     for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
                  "moe_layer_forward", "moe_get_device_status", "moe_permute_static",
-                 "moe_selftest_wait_timeout"):
+                 "moe_selftest_wait_timeout", "moe_layer_forward_host"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -94,6 +98,17 @@ def _p(t):
         return t
     if not t.is_cuda:
         raise ValueError("libmoe takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _hp(t):
+    """Host pointer of a CPU tensor (None -> NULL); page-locked memory lets the copies overlap."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("moe_layer_forward_host takes host tensors")
     if not t.is_contiguous():
         raise ValueError("libmoe takes contiguous tensors")
     return t.data_ptr()
@@ -195,6 +210,18 @@ def moe_layer_forward(desc, weights, x, prev_logits, y, logits_out, workspace, s
     _check("moe_layer_forward", load().moe_layer_forward(ctypes.byref(desc), ctypes.byref(ws), _p(x),
                                                          _p(prev_logits), _p(y), _p(logits_out),
                                                          _p(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def moe_layer_host_workspace_size(desc: MoELayerDesc, chunks: int = 0) -> int:
+    return int(load().moe_layer_host_workspace_size(ctypes.byref(desc), int(chunks)))
+
+
+def moe_layer_forward_host(desc, weights, x_host, prev_logits_host, y_host, chunks, workspace, stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_layer_forward_host",
+           load().moe_layer_forward_host(ctypes.byref(desc), ctypes.byref(ws), _hp(x_host), _hp(prev_logits_host),
+                                         _hp(y_host), int(chunks), _p(workspace), _nbytes(workspace),
+                                         _stream(stream)))
 
 
 def moe_get_device_status(reset: bool = True, stream=None) -> int:

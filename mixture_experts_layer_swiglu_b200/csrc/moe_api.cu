@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -455,6 +456,67 @@ moe_status validate_desc(const moe_layer_desc* d) { return check_desc(d); }
 
 using namespace moe;
 
+// ----------------------------------------------------- host-to-host layer
+
+namespace {
+
+constexpr int kMaxHostChunks = 8;
+
+struct HostPipe {                       // per device: two copy streams and their events
+    bool ok = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t fork = nullptr;
+    cudaEvent_t in_done[kMaxHostChunks], comp_done[kMaxHostChunks], out_done[kMaxHostChunks];
+};
+
+HostPipe* host_pipe()
+{
+    static std::mutex mu;
+    static HostPipe pipes[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    HostPipe& p = pipes[dev];
+    if (!p.ok) {
+        bool good = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int c = 0; good && c < kMaxHostChunks; ++c)
+            good = cudaEventCreateWithFlags(&p.in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&p.comp_done[c], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&p.out_done[c], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) return nullptr;
+        p.ok = true;
+    }
+    return &p;
+}
+
+int host_chunks(const moe_layer_desc* d, int chunks)
+{
+    if (chunks <= 0) chunks = d->T >= 8192 ? 4 : (d->T >= 4096 ? 2 : 1);
+    return std::max(1, std::min(std::min(chunks, kMaxHostChunks), std::max(d->T, 1)));
+}
+
+struct HostLayout {
+    moe_layer_desc dc;                  // one token range (the largest)
+    size_t layer_bytes, x_bytes, y_bytes, z_bytes, total;
+};
+
+HostLayout host_layout(const moe_layer_desc* d, int nch)
+{
+    HostLayout h;
+    h.dc = *d;
+    h.dc.T = cdiv(std::max(d->T, 1), nch);
+    h.layer_bytes = al((size_t)moe_layer_workspace_size(&h.dc));
+    h.x_bytes = al((size_t)h.dc.T * d->d_model * elt(d));
+    h.y_bytes = al((size_t)h.dc.T * d->d_model * (d->out_f32 ? 4 : elt(d)));
+    h.z_bytes = d->kind == MOE_EXPERT_SWIGLU ? al((size_t)h.dc.T * n_router_rows(d) * 4) : 0;
+    h.total = h.layer_bytes + 2 * (h.x_bytes + h.y_bytes + h.z_bytes);
+    return h;
+}
+
+}  // namespace
+
 extern "C" {
 
 int64_t moe_num_groups(const moe_layer_desc* d)
@@ -572,6 +634,80 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const moe_layer_weights* w
     if ((s = ffn_impl(d, w, b.xs, b.offsets, b.token_of, x, b.gate, b.ys, b.scratch, b.scratch_bytes, st)) != MOE_OK)
         return s;
     return combine_impl(d, w, b.ys, b.offsets, b.row_of, b.idx, b.gate, b.cmix, x, y, st);
+}
+
+int64_t moe_layer_host_workspace_size(const moe_layer_desc* d, int chunks)
+{
+    if (check_desc(d) != MOE_OK) return -1;
+    return (int64_t)host_layout(d, host_chunks(d, chunks)).total;
+}
+
+moe_status moe_layer_forward_host(const moe_layer_desc* d, const moe_layer_weights* w, const void* x_host,
+                                  const float* prev_logits_host, void* y_host, int chunks, void* workspace,
+                                  size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || (d->T > 0 && (!x_host || !y_host))) return MOE_ERR_INVALID_ARG;
+    if (prev_logits_host && d->kind != MOE_EXPERT_SWIGLU) return MOE_ERR_INVALID_ARG;
+    const int nch = host_chunks(d, chunks);
+    const HostLayout h = host_layout(d, nch);
+    if (!workspace || ws_bytes < h.total || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
+    if (d->T == 0) return MOE_OK;
+    HostPipe* pp = host_pipe();
+    if (!pp) return MOE_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(workspace);
+    void* layer_ws = base;
+    char* xb[2] = {base + h.layer_bytes, base + h.layer_bytes + h.x_bytes};
+    char* yb[2] = {xb[1] + h.x_bytes, xb[1] + h.x_bytes + h.y_bytes};
+    char* zb[2] = {yb[1] + h.y_bytes, yb[1] + h.y_bytes + h.z_bytes};
+    const size_t xrow = (size_t)d->d_model * elt(d);
+    const size_t yrow = (size_t)d->d_model * (d->out_f32 ? 4 : elt(d));
+    const size_t zrow = (size_t)n_router_rows(d) * 4;
+    cudaError_t e;
+#define MOE_CU(call)                                    \
+    do {                                                \
+        if ((e = (call)) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+    MOE_CU(cudaEventRecord(pp->fork, st));              // the copy streams join `stream`'s work
+    MOE_CU(cudaStreamWaitEvent(pp->in, pp->fork, 0));
+    MOE_CU(cudaStreamWaitEvent(pp->out, pp->fork, 0));
+    int launches = 0;
+    for (int c = 0; c < nch; ++c) {
+        const int t0 = c * h.dc.T;
+        const int tc = std::min(h.dc.T, d->T - t0);
+        if (tc <= 0) break;
+        const int b = c & 1;
+        if (c >= 2) MOE_CU(cudaStreamWaitEvent(pp->in, pp->comp_done[c - 2], 0));   // staging b read
+        MOE_CU(cudaMemcpyAsync(xb[b], static_cast<const char*>(x_host) + (size_t)t0 * xrow, (size_t)tc * xrow,
+                               cudaMemcpyHostToDevice, pp->in));
+        if (prev_logits_host)
+            MOE_CU(cudaMemcpyAsync(zb[b], reinterpret_cast<const char*>(prev_logits_host) + (size_t)t0 * zrow,
+                                   (size_t)tc * zrow, cudaMemcpyHostToDevice, pp->in));
+        MOE_CU(cudaEventRecord(pp->in_done[c], pp->in));
+        MOE_CU(cudaStreamWaitEvent(st, pp->in_done[c], 0));
+        if (c >= 2) MOE_CU(cudaStreamWaitEvent(st, pp->out_done[c - 2], 0));     // output b copied out
+        moe_layer_desc dcc = h.dc;
+        dcc.T = tc;
+        s = moe_layer_forward(&dcc, w, xb[b], prev_logits_host ? reinterpret_cast<const float*>(zb[b]) : nullptr,
+                              yb[b], nullptr, layer_ws, h.layer_bytes, stream);
+        launches += t_launches;
+        if (s != MOE_OK) return s;
+        MOE_CU(cudaEventRecord(pp->comp_done[c], st));
+        MOE_CU(cudaStreamWaitEvent(pp->out, pp->comp_done[c], 0));
+        MOE_CU(cudaMemcpyAsync(static_cast<char*>(y_host) + (size_t)t0 * yrow, yb[b], (size_t)tc * yrow,
+                               cudaMemcpyDeviceToHost, pp->out));
+        MOE_CU(cudaEventRecord(pp->out_done[c], pp->out));
+        if (c == nch - 1 || (c + 1) * h.dc.T >= d->T) {   // join both copy streams back into `stream`
+            MOE_CU(cudaStreamWaitEvent(st, pp->out_done[c], 0));
+            MOE_CU(cudaStreamWaitEvent(st, pp->in_done[c], 0));
+        }
+    }
+#undef MOE_CU
+    t_launches = launches;
+    return MOE_OK;
 }
 
 moe_status moe_get_device_status(moe_status* out, int reset, moe_stream_t stream)

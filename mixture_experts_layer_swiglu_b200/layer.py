@@ -116,4 +116,21 @@ class MoELayer:
                               self.workspace(x.device), stream)
         return y
 
+    def forward_host(self, x_host: torch.Tensor, prev_logits=None, y_host=None, chunks: int = 0, stream=None,
+                     device=None):
+        """moe_layer_forward_host: x from host memory, y to host memory, the
+        copies pipelined against the layer in token ranges.  Returns y_host
+        (complete once `stream` reaches this point)."""
+        device = torch.device(device or "cuda")
+        if y_host is None:
+            y_host = torch.empty(x_host.shape, dtype=out_dtype(self.desc), pin_memory=True)
+        need = abi.moe_layer_host_workspace_size(self.desc, chunks)
+        if need < 0:
+            raise abi.MoEError("moe_layer_host_workspace_size", abi.MOE_ERR_INVALID_ARG)
+        if getattr(self, "_host_ws", None) is None or self._host_ws.numel() < need or self._host_ws.device != device:
+            self._host_ws = torch.empty((need,), dtype=torch.uint8, device=device)
+        abi.moe_layer_forward_host(self.desc, self._ws_struct, x_host, prev_logits, y_host, chunks, self._host_ws,
+                                   stream)
+        return y_host
+
     __call__ = forward

@@ -68,6 +68,19 @@ def test_rejected_descriptors(abi, bad):
     d = _desc(abi, **bad)
     assert abi.moe_workspace_size(d) == -1
     assert abi.moe_layer_workspace_size(d) == -1
+    assert abi.moe_layer_host_workspace_size(d, 0) == -1
+
+
+def test_host_call_workspace_follows_the_token_ranges(abi):
+    d = _desc(abi, T=4096, d_model=4096, top_k=2, n_ffn=8, hidden=14336)
+    one = _desc(abi, T=2048, d_model=4096, top_k=2, n_ffn=8, hidden=14336)
+    two = abi.moe_layer_host_workspace_size(d, 0)           # automatic: 2 ranges of 2048 tokens
+    assert two == abi.moe_layer_host_workspace_size(d, 2)
+    # one range's layer workspace plus double-buffered x, y and router-logit staging
+    staging = 2 * (2048 * 4096 * 2 * 2 + 2048 * 8 * 4)
+    assert two >= abi.moe_layer_workspace_size(one) + staging
+    assert abi.moe_layer_host_workspace_size(d, 1) > two     # one range holds the whole batch
+    assert abi.moe_layer_host_workspace_size(d, 100) == abi.moe_layer_host_workspace_size(d, 8)
 
 
 def test_argument_errors_without_a_device(abi):
@@ -80,5 +93,9 @@ def test_argument_errors_without_a_device(abi):
                          None) == 1
     assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), 16, None, 16, None, None, 0, None) == 3
     assert lib.moe_grouped_ffn_phase(ctypes.byref(d), ctypes.byref(w), 3, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert lib.moe_layer_forward_host(ctypes.byref(d), ctypes.byref(w), None, None, None, 0, None, 0, None) == 1
+    assert lib.moe_layer_forward_host(ctypes.byref(d), ctypes.byref(w), 16, None, 16, 0, 16, 0, None) == 3
+    a = _desc(abi, T=8, d_model=256, top_k=4, kind="atomic", pk_rows=32, pk_cols=32, pk_topk_half=4, d_query=64)
+    assert lib.moe_layer_forward_host(ctypes.byref(a), ctypes.byref(w), 16, 16, 16, 0, 16, 1 << 30, None) == 1
     assert lib.moe_last_launch_count() == 0
     assert abi.status_string(3) == "workspace too small"

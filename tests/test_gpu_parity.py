@@ -152,6 +152,28 @@ def test_cuda_graph_replay_matches_eager(name, T, changes):
     assert moe.moe_get_device_status() == moe.MOE_OK
 
 
+@pytest.mark.parametrize("name,T,changes,chunks", [
+    ("moepp", 700, {"hidden": 640}, 3),        # gating residual from host memory, ragged last range
+    ("atomic", 1000, {}, 4),
+    ("mixtral", 600, {"d": 512, "hidden": 512}, 0),
+    ("tiny_f32", 64, {}, 2),
+])
+def test_host_call_equals_device_call(name, T, changes, chunks):
+    """moe_layer_forward_host (host buffers, copies pipelined over token
+    ranges) gives moe_layer_forward's output bit for bit."""
+    cfg = scaled(get_config(name), T=T, **changes)
+    inp = make_inputs(cfg)
+    dev = to_device(inp)
+    layer = moe.MoELayer(moe.desc_from(cfg), dev)
+    ref = layer.forward(dev["x"], prev_logits=dev.get("z_prev"))
+    x_host = inp["x"].contiguous().pin_memory()
+    zp_host = inp["z_prev"].contiguous().pin_memory() if "z_prev" in inp else None
+    y_host = layer.forward_host(x_host, prev_logits=zp_host, chunks=chunks)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, ref.cpu())
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
 def test_invalid_expert_id_sets_bounds_status():
     cfg = scaled(get_config("mixtral"), T=64, d=256, hidden=256, n_ffn=4)
     inp = to_device(make_inputs(cfg))
