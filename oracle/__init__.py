@@ -64,6 +64,8 @@ def lib():
         L.orc_pk_select.argtypes = [ctypes.c_int] * 5 + [_F64P, _F64P, _I32P, _F64P, _F64P]
         L.orc_atomic_tokens.argtypes = [ctypes.c_int] * 3 + [_VP] * 3 + [
             ctypes.c_int, _I32P, _I32P, _F64P, _F64P]
+        L.orc_omni_tokens.argtypes = [ctypes.c_int] * 3 + [_VP] * 3 + [ctypes.c_int] * 2 + [_VP] * 3 + [
+            ctypes.c_int, _I32P, _I32P, _F64P, _F64P]
         _lib = L
     return _lib
 
@@ -235,8 +237,10 @@ def pk_select(s_row, s_col, kh: int, K: int):
     return idx, gate, mg
 
 
-def atomic_tokens(x, u, v, tokens, idx, gate) -> np.ndarray:
-    """y_t = sum_j g_j GELU(u_e . x_t) v_e for the listed tokens (fp64)."""
+def atomic_tokens(x, u, v, tokens, idx, gate, shared=None) -> np.ndarray:
+    """y_t = sum_j g_j GELU(u_e . x_t) v_e for the listed tokens (fp64); with
+    ``shared`` = dict(ws_gate, ws_up, ws_down) the shared dense SwiGLU
+    branches are added (the full OmniMoE layer)."""
     x, u, v = _cpu(x), _cpu(u), _cpu(v)
     tokens = _np_i32(tokens).reshape(-1)
     n = tokens.shape[0]
@@ -245,6 +249,12 @@ def atomic_tokens(x, u, v, tokens, idx, gate) -> np.ndarray:
     gate = _np_f64(gate).reshape(n, K)
     d = x.shape[1]
     y = np.empty((n, d), np.float64)
-    lib().orc_atomic_tokens(d, K, _dt(x, u, v), _vp(x), _vp(u), _vp(v), n, _i32(tokens),
-                            _i32(idx), _f64(gate), _f64(y))
+    if shared is None:
+        lib().orc_atomic_tokens(d, K, _dt(x, u, v), _vp(x), _vp(u), _vp(v), n, _i32(tokens),
+                                _i32(idx), _f64(gate), _f64(y))
+    else:
+        sg, su, sd = (_cpu(shared[k_]) for k_ in ("ws_gate", "ws_up", "ws_down"))
+        S, Hs = sg.shape[0], sg.shape[1]
+        lib().orc_omni_tokens(d, K, _dt(x, u, v, sg, su, sd), _vp(x), _vp(u), _vp(v), S, Hs, _vp(sg), _vp(su),
+                              _vp(sd), n, _i32(tokens), _i32(idx), _f64(gate), _f64(y))
     return y

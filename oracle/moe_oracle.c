@@ -430,3 +430,31 @@ void orc_atomic_tokens(int d, int K, int dt, const void* x, const void* u, const
         free(xt);
     }
 }
+
+/*
+ * The full OmniMoE layer ("OmniMoE" 2.1: a shared dense MLP branch, always
+ * active, beside the routed atomic experts) for the listed tokens:
+ *   y_t = sum_s SwiGLU_s(x_t) + sum_j g_j * GELU(u_e . x_t) * v_e
+ * with the shared branches in the layer's SwiGLU form (ws_gate, ws_up
+ * [n_shared, Hs, d], ws_down [n_shared, d, Hs]) and weight 1.
+ */
+void orc_omni_tokens(int d, int K, int dt, const void* x, const void* u, const void* v,
+                     int n_shared, int Hs, const void* ws_gate, const void* ws_up, const void* ws_down,
+                     int n_tok, const int32_t* tokens, const int32_t* idx, const double* gate, double* y)
+{
+    orc_atomic_tokens(d, K, dt, x, u, v, n_tok, tokens, idx, gate, y);
+    const size_t eb = dt == ORC_F32 ? 4 : 2;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < n_tok; ++n) {
+        double* xt = (double*)malloc(sizeof(double) * (size_t)d);
+        double* h = (double*)malloc(sizeof(double) * (size_t)(Hs > 0 ? Hs : 1));
+        widen_row(x, (size_t)tokens[n], d, dt, xt);
+        for (int sh = 0; sh < n_shared; ++sh) {
+            const size_t off = (size_t)sh * Hs * d * eb;
+            swiglu_acc(d, Hs, dt, (const char*)ws_gate + off, (const char*)ws_up + off,
+                       (const char*)ws_down + off, xt, 1.0, y + (size_t)n * d, h);
+        }
+        free(xt);
+        free(h);
+    }
+}

@@ -364,3 +364,31 @@ def test_atomic_layer_dense_masked_bruteforce():
     ref = (torch.from_numpy(G) * act) @ v.double()
     np.testing.assert_allclose(y, ref.numpy(), atol=1e-13)
     np.testing.assert_allclose(gate.sum(1), 1.0, atol=1e-14)
+
+
+def test_full_omnimoe_layer_is_atomic_plus_shared_swiglu():
+    """The full OmniMoE layer (shared dense branch beside the atomic experts)
+    minus the atomic-only layer equals the shared SwiGLU branch, computed two
+    other ways: by the SwiGLU-kind layer whose one routed expert has a zero
+    down projection, and densely with torch."""
+    x, wq, kr, kc = _pk_inputs(5, T=5, d=16, dq=8, rows=8, cols=8)
+    g = torch.Generator().manual_seed(11)
+    u = torch.randn(64, 16, generator=g) * 0.25
+    v = torch.randn(64, 16, generator=g) * 0.25
+    Hs = 24
+    sh = {"ws_gate": torch.randn(1, Hs, 16, generator=g) * 0.25, "ws_up": torch.randn(1, Hs, 16, generator=g) * 0.25,
+          "ws_down": torch.randn(1, 16, Hs, generator=g) * 0.2}
+    sr, sc = oracle.pk_scores(x, wq, kr, kc)
+    idx, gate, _ = oracle.pk_select(sr, sc, kh=6, K=5)
+    y_full = oracle.atomic_tokens(x, u, v, np.arange(5), idx, gate, shared=sh)
+    y_atom = oracle.atomic_tokens(x, u, v, np.arange(5), idx, gate)
+    cfg = _cfg(T=5, d=16, top_k=1, n_ffn=1, hidden=4, n_shared=1, hidden_shared=Hs)
+    inp = {"x": x, "w_router": torch.ones(1, 16), "w_gate": torch.randn(1, 4, 16, generator=g),
+           "w_up": torch.randn(1, 4, 16, generator=g), "w_down": torch.zeros(1, 16, 4), **sh}
+    y_sh = oracle.moe_tokens(cfg, inp, np.arange(5))[0]
+    np.testing.assert_allclose(y_full - y_atom, y_sh, rtol=0, atol=1e-13)
+    xd = x.double()
+    a = xd @ sh["ws_gate"][0].double().T
+    dense = ((a * torch.sigmoid(a)) * (xd @ sh["ws_up"][0].double().T)) @ sh["ws_down"][0].double().T
+    np.testing.assert_allclose(y_full - y_atom, dense.numpy(), rtol=0, atol=1e-13)
+    assert np.abs(dense.numpy()).max() > 0.05          # the branch is not negligible here
