@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
     p.add_argument("--experts", type=int, default=0, help="override the expert count (profiling)")
     p.add_argument("--workload", default=WORKLOAD,
-                   help="tiny_f32 | mixtral | longtail | moepp | atomic (default: the Mixtral-shaped layer)")
+                   help="tiny_f32 | mixtral | longtail | moepp | atomic | omnimoe (default: the Mixtral-shaped layer)")
     p.add_argument("--no-library-ref", action="store_true", help="skip the cuBLAS same-shape reference")
     return p.parse_args()
 
@@ -73,6 +73,9 @@ def workload_config(cfg) -> dict:
     if cfg.kind == "atomic":
         name = f"{cfg.name}_T{cfg.T}_d{cfg.d}_N{cfg.pk_rows}x{cfg.pk_cols}_K{cfg.top_k}_half{cfg.pk_topk_half}"
         shape = {"experts": cfg.n_atomic, "d_query": cfg.d_query, "router": "Cartesian product, top-K of top-half^2"}
+        if cfg.n_shared:
+            name += f"_shared{cfg.hidden_shared}"
+            shape["shared_dense_hidden"] = cfg.hidden_shared
     else:
         name = f"{cfg.name}_T{cfg.T}_d{cfg.d}_E{cfg.n_ffn}_H{cfg.hidden}_k{cfg.top_k}"
         if cfg.n_shared:
@@ -153,7 +156,8 @@ def oracle_sample(cfg, inp, toks) -> None:
         xs = inp["x"][torch.from_numpy(toks).long()]
         sr, sc = oracle.pk_scores(xs, inp["w_query"], inp["subkeys_row"], inp["subkeys_col"])
         idx, gate, _ = oracle.pk_select(sr, sc, cfg.pk_topk_half, cfg.top_k)
-        oracle.atomic_tokens(inp["x"], inp["u"], inp["v"], toks, idx, gate)
+        shared = {k_: inp[k_] for k_ in ("ws_gate", "ws_up", "ws_down")} if cfg.n_shared else None
+        oracle.atomic_tokens(inp["x"], inp["u"], inp["v"], toks, idx, gate, shared=shared)
     else:
         oracle.moe_tokens(cfg, inp, toks)
 
@@ -205,7 +209,8 @@ def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
 
 def stage_names(cfg) -> list:
     if cfg.kind == "atomic":
-        return ["router", "permute", "expert_dot", "expert_combine"]
+        shared = ["shared_gate_up_gemm", "shared_down_gemm"] if cfg.n_shared else []
+        return ["router", "permute", "expert_dot"] + shared + ["expert_combine"]
     return ["router", "permute", "gate_up_gemm", "down_gemm", "combine"]
 
 
@@ -221,7 +226,9 @@ def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
             # once, y written once (the token-centric phase B moves more: it
             # gathers a v row per slot, with L2 hits for rows shared in time)
             "expert_dot": ("hbm", touched * d * e + T * d * e + T * k * 12),
-            "expert_combine": ("hbm", touched * d * e + T * d * e + T * k * 8),
+            "expert_combine": ("hbm", touched * d * e + T * d * e + T * k * 8 + cfg.n_shared * T * d * 4),
+            "shared_gate_up_gemm": ("tensor", 4.0 * T * d * cfg.hidden_shared),
+            "shared_down_gemm": ("tensor", 2.0 * T * d * cfg.hidden_shared),
         }
     H = cfg.hidden
     E_r = cfg.n_routed
@@ -250,6 +257,8 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     x = a_cpu["x"].to(dev)
     zp = a_cpu["z_prev"].to(dev) if "z_prev" in a_cpu else None
     desc = moe.desc_from(cfg)
+    desc_atomic = moe.desc_from(cfg)          # the same layer without its shared branch
+    desc_atomic.n_shared, desc_atomic.hidden_shared = 0, 0
     ws = moe.weights_struct(w)
     b = moe.StageBuffers(desc, device=dev)
     cm = b.const_mix if cfg.n_const else None
@@ -261,9 +270,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         c = [lambda: moe.moe_route(desc, ws, x, zp, None, b.idx, b.gate, cm, b.workspace, st),
              lambda: moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace,
                                      st)]
-        if atomic:
-            c.append(lambda: moe.moe_grouped_ffn(desc, ws, None, b.offsets, b.token_of, x, b.gate, b.y_sorted,
-                                                 b.workspace, st))
+        if atomic:   # the atomic step alone, then the shared dense branch's two GEMMs (if any)
+            c.append(lambda: moe.moe_grouped_ffn(desc_atomic, ws, None, b.offsets, b.token_of, x, b.gate,
+                                                 b.y_sorted, b.workspace, st))
+            if cfg.n_shared:
+                c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 1, x, b.offsets, b.y_sorted, b.workspace, st))
+                c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 2, x, b.offsets, b.y_sorted, b.workspace, st))
         else:
             c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 1, b.x_sorted, b.offsets, b.y_sorted,
                                                        b.workspace, st))

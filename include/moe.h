@@ -83,8 +83,10 @@ typedef struct moe_layer_desc {
     int32_t kind;          /* moe_expert_kind                                     */
     int32_t n_ffn;         /* routed SwiGLU experts                               */
     int32_t hidden;        /* their hidden width H                                */
-    int32_t n_shared;      /* always-on SwiGLU experts (weight 1)                 */
-    int32_t hidden_shared; /* their hidden width (must equal hidden if n_shared)  */
+    int32_t n_shared;      /* always-on SwiGLU experts (weight 1); atomic kind:   *
+                            * 0 or 1 shared dense branch (the full OmniMoE layer) */
+    int32_t hidden_shared; /* their hidden width (SwiGLU kind: equal to hidden;   *
+                            * atomic kind: a multiple of 128)                     */
     int32_t n_zero;        /* MoE++ zero experts                                  */
     int32_t n_copy;        /* MoE++ copy experts                                  */
     int32_t n_const;       /* MoE++ constant experts                              */
@@ -186,7 +188,12 @@ MOE_API moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_i
  *   expert e, over the expert-sorted task order in units of 16 tasks whose
  *   dot products are one tensor-core tile (each touched u_e read once per
  *   unit); y_sorted is float c[T*K] in slot order.  x_sorted unused.  The
- *   workspace holds the expert of each task (T*top_k int32).
+ *   workspace holds the expert of each task (T*top_k int32).  With a shared
+ *   dense branch ("OmniMoE" 2.1, Shared Dense MLP; n_shared = 1) the call
+ *   also computes ys = Ws_down (silu(Ws_gate x_t) * (Ws_up x_t)) for every
+ *   token (two grouped GEMMs, the hidden activation rounded to bf16 in the
+ *   workspace) into y_sorted after c, at byte offset align256(T*K*4), as
+ *   [T, d_model] fp32.
  */
 MOE_API moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_layer_weights* w,
                            const void* x_sorted, const int32_t* expert_offsets,
@@ -198,7 +205,10 @@ MOE_API moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_layer_w
  * The two grouped GEMMs of the SwiGLU step, one per call (same arguments as
  * moe_grouped_ffn): phase 1 writes the hidden activation h into the
  * workspace, phase 2 reads it and writes y_sorted.  Calling phase 1 then
- * phase 2 on the same workspace equals moe_grouped_ffn.  SwiGLU kind only.
+ * phase 2 on the same workspace equals moe_grouped_ffn.  Atomic kind with a
+ * shared dense branch: phase 1 and 2 are that branch's two GEMMs (x_sorted
+ * is x itself, expert_offsets unused); moe_grouped_ffn = the atomic step
+ * followed by both.
  */
 MOE_API moe_status moe_grouped_ffn_phase(const moe_layer_desc* desc, const moe_layer_weights* w,
                                  int phase, const void* x_sorted,
@@ -214,7 +224,8 @@ MOE_API moe_status moe_grouped_ffn_phase(const moe_layer_desc* desc, const moe_l
  *   for an FFN expert, 0 for a zero expert, x_t for a copy expert and
  *   a1 x_t + a2 v_c for constant expert c (const_mix, w->const_vec);
  *   accumulated in fp32 in slot order, rounded once to dtype.
- * Atomic: y_t = sum_j c[t*K + j] * v_{topk_idx[t, j]} (y_sorted = c).
+ * Atomic: y_t = sum_j c[t*K + j] * v_{topk_idx[t, j]} (+ the shared branch's
+ *   row of y_sorted when n_shared = 1), fp32, rounded once.
  * y [T, d_model] in dtype, or fp32 if desc->out_f32.
  */
 MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weights* w,

@@ -524,6 +524,16 @@ __global__ void __launch_bounds__(PB_WARPS * 32, 1) atomic_phase_b_kernel(const 
         ++cons;
         if (++kc == ns) {
             const int vecs = a.d / 8;
+            if (a.shared_out) {   // the shared dense branch, added before the one rounding
+                const float4* sp = reinterpret_cast<const float4*>(a.shared_out);
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    const long long o = ((long long)tc * vecs + v * 32 + lane) * 2;
+                    const float4 s0 = sp[o], s1 = sp[o + 1];
+                    acc[v][0] += s0.x; acc[v][1] += s0.y; acc[v][2] += s0.z; acc[v][3] += s0.w;
+                    acc[v][4] += s1.x; acc[v][5] += s1.y; acc[v][6] += s1.z; acc[v][7] += s1.w;
+                }
+            }
             if (a.out_f32) {
                 float4* y = reinterpret_cast<float4*>(a.y);
 #pragma unroll

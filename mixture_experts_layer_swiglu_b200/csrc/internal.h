@@ -122,6 +122,7 @@ struct AtomicArgs {
     const int32_t* idx;        // [T, K]
     const float* gate;         // [T, K]
     float* c;                  // [T*K]
+    const float* shared_out;   // [T, d] fp32 output of the shared dense branch, nullable
     void* y;                   // [T, d] bf16, or fp32 if out_f32
     int T, d, K, N;
     int out_f32;

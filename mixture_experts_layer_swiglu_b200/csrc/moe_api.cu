@@ -69,8 +69,11 @@ moe_status check_desc(const moe_layer_desc* d)
     }
     if (d->kind == MOE_EXPERT_ATOMIC_GELU) {
         if (d->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-        if (d->n_ffn || d->n_shared || d->n_zero || d->n_copy || d->n_const || d->hidden)
+        if (d->n_ffn || d->n_zero || d->n_copy || d->n_const || d->hidden) return MOE_ERR_INVALID_ARG;
+        // one shared dense SwiGLU branch beside the atomic experts (the full OmniMoE layer)
+        if (d->n_shared < 0 || d->n_shared > 1 || (d->n_shared == 0 && d->hidden_shared != 0))
             return MOE_ERR_INVALID_ARG;
+        if (d->n_shared == 1 && (d->hidden_shared <= 0 || d->hidden_shared % 128 != 0)) return MOE_ERR_UNSUPPORTED;
         if (d->pk_rows <= 0 || d->pk_cols <= 0 || d->pk_topk_half <= 0 || d->d_query <= 0)
             return MOE_ERR_INVALID_ARG;
         if (d->pk_topk_half > d->pk_rows || d->pk_topk_half > d->pk_cols) return MOE_ERR_INVALID_ARG;
@@ -106,7 +109,7 @@ Scratch scratch_sizes(const moe_layer_desc* d)
                   al((size_t)2 * d->T * d->pk_rows * 4);
         const size_t N = (size_t)d->pk_rows * d->pk_cols;
         s.permute = al(N * 4) + al((size_t)atomic_scan_blocks((int)N) * 4);
-        s.ffn = 2 * al((size_t)d->T * d->top_k * 4);
+        s.ffn = 2 * al((size_t)d->T * d->top_k * 4) + (d->n_shared ? al((size_t)d->T * d->hidden_shared * 2) : 0);
     }
     return s;
 }
@@ -150,7 +153,7 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
         b.ys = take((size_t)cap * d->d_model * 4);
     } else {
         b.xs = nullptr;
-        b.ys = take((size_t)Tk * 4);
+        b.ys = take(al((size_t)Tk * 4) + (size_t)d->n_shared * d->T * d->d_model * 4);
     }
     b.scratch_bytes = scratch_max(d);
     b.scratch = take(b.scratch_bytes);
@@ -303,6 +306,54 @@ moe_status permute_impl(const moe_layer_desc* d, const int32_t* idx, const void*
     return launch_permute_atomic(a, st);
 }
 
+// The shared dense SwiGLU branch of the atomic kind: phase 1 h = silu(x Ws_gate^T) * (x Ws_up^T)
+// (bf16, after the task metadata in the workspace), phase 2 ys_shared = h Ws_down^T (fp32, after c
+// in y_sorted).  One group of all T tokens on the grouped tcgen05 GEMM, A read straight from x.
+moe_status atomic_shared_phase(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* x,
+                               void* ys, void* ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (d->n_shared == 0 || d->T == 0) return MOE_OK;
+    const Scratch sc = scratch_sizes(d);
+    if (!ws || ws_bytes < sc.ffn || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (!w->ws_gate || !w->ws_up || !w->ws_down || !ys || !aligned16(ys)) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[4] = {w->ws_gate, w->ws_up, w->ws_down, x};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const size_t Tk4 = al((size_t)d->T * d->top_k * 4);
+    void* h = static_cast<char*>(ws) + 2 * Tk4;
+    GemmProblem g{};
+    g.offsets = nullptr;
+    g.n_groups = 1;
+    g.n_first = 1;
+    g.group_rows = d->T;
+    g.rows_cap = d->T;
+    g.pair = d->T >= 512 ? 1 : 0;
+    if (phase == 1) {
+        if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+        g.epi = EPI_SWIGLU;
+        g.A = x;
+        g.a_rows = d->T;
+        g.K = d->d_model;
+        g.B0 = w->ws_gate;
+        g.B1 = w->ws_up;
+        g.b01_rows = d->hidden_shared;
+        g.N = d->hidden_shared;
+        g.out = h;
+        g.ldo = d->hidden_shared;
+    } else {
+        g.epi = EPI_F32;
+        g.A = h;
+        g.a_rows = d->T;
+        g.K = d->hidden_shared;
+        g.B0 = w->ws_down;
+        g.b01_rows = d->d_model;
+        g.N = d->d_model;
+        g.out = static_cast<char*>(ys) + Tk4;
+        g.ldo = d->d_model;
+    }
+    return launch_grouped_gemm(g, st);
+}
+
 moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* xs,
                           const int32_t* offsets, void* ys, void* ws, size_t ws_bytes, cudaStream_t st)
 {
@@ -399,7 +450,10 @@ moe_status ffn_impl(const moe_layer_desc* d, const moe_layer_weights* w, const v
     a.d = d->d_model;
     a.K = d->top_k;
     a.N = d->pk_rows * d->pk_cols;
-    return launch_atomic_phase_a(a, st);
+    moe_status s = launch_atomic_phase_a(a, st);
+    if (s != MOE_OK || d->n_shared == 0) return s;
+    if ((s = atomic_shared_phase(d, w, 1, x, ys, ws, ws_bytes, st)) != MOE_OK) return s;
+    return atomic_shared_phase(d, w, 2, x, ys, ws, ws_bytes, st);
 }
 
 moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, const void* ys,
@@ -414,6 +468,9 @@ moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, con
         a.v = w->v;
         a.idx = idx;
         a.c = const_cast<float*>(static_cast<const float*>(ys));
+        a.shared_out = d->n_shared ? reinterpret_cast<const float*>(static_cast<const char*>(ys) +
+                                                                     al((size_t)d->T * d->top_k * 4))
+                                   : nullptr;
         a.y = y;
         a.T = d->T;
         a.d = d->d_model;
@@ -596,7 +653,12 @@ moe_status moe_grouped_ffn_phase(const moe_layer_desc* d, const moe_layer_weight
     t_launches = 0;
     moe_status s = check_desc(d);
     if (s != MOE_OK) return s;
-    if (d->kind != MOE_EXPERT_SWIGLU || (phase != 1 && phase != 2)) return MOE_ERR_INVALID_ARG;
+    if (phase != 1 && phase != 2) return MOE_ERR_INVALID_ARG;
+    if (d->kind == MOE_EXPERT_ATOMIC_GELU) {   // the shared dense branch; x_sorted is x itself
+        if (!w || d->n_shared == 0 || (d->T > 0 && (!x_sorted || !y_sorted))) return MOE_ERR_INVALID_ARG;
+        return atomic_shared_phase(d, w, phase, x_sorted, y_sorted, workspace, ws_bytes,
+                                   static_cast<cudaStream_t>(stream));
+    }
     if (!w || !expert_offsets || (d->T > 0 && (!x_sorted || !y_sorted))) return MOE_ERR_INVALID_ARG;
     return ffn_phase_impl(d, w, phase, x_sorted, expert_offsets, y_sorted, workspace, ws_bytes,
                           static_cast<cudaStream_t>(stream));

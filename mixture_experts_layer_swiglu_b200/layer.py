@@ -73,7 +73,9 @@ class StageBuffers:
             self.y_sorted = torch.empty((max(cap, 1), d), dtype=f32, device=device)
         else:
             self.x_sorted = None
-            self.y_sorted = torch.empty((max(T * k, 1),), dtype=f32, device=device)
+            # c [T*k] fp32, then (full OmniMoE layer) the shared branch's [T, d] fp32 at a 256-byte boundary
+            c_floats = (T * k * 4 + 255) // 256 * 64
+            self.y_sorted = torch.empty((max(c_floats + desc.n_shared * T * d, 1),), dtype=f32, device=device)
         self.workspace = torch.empty((abi.moe_workspace_size(desc),), dtype=torch.uint8, device=device)
         self.y = torch.empty((T, d), dtype=out_dtype(desc), device=device)
 

@@ -18,6 +18,11 @@ shapes and distributions follow the workloads the pages study:
 * ``atomic``        : OmniMoE atomic experts, T=8192, d=1024, N=512x512 vector
                       experts, Cartesian-product router with top-32 per half and
                       top-64 overall (OmniMoE page, 2.1 and 2.2).
+* ``omnimoe``       : the full OmniMoE layer: the ``atomic`` workload plus the
+                      shared dense branch every token passes through (OmniMoE
+                      page, 2.1 "Shared Dense MLP"), a SwiGLU FFN of hidden
+                      width 2816 (8/3 d rounded up to a multiple of 128; the
+                      page gives no size).
 """
 
 from __future__ import annotations
@@ -82,9 +87,12 @@ CONFIGS: dict[str, MoEConfig] = {
     "atomic": MoEConfig(
         name="atomic", T=8192, d=1024, top_k=64, dtype="bf16", kind="atomic",
         pk_rows=512, pk_cols=512, pk_topk_half=32, d_query=1024),
+    "omnimoe": MoEConfig(
+        name="omnimoe", T=8192, d=1024, top_k=64, dtype="bf16", kind="atomic",
+        pk_rows=512, pk_cols=512, pk_topk_half=32, d_query=1024, n_shared=1, hidden_shared=2816),
 }
 
-ORDER = ["tiny_f32", "mixtral", "longtail", "moepp", "atomic"]
+ORDER = ["tiny_f32", "mixtral", "longtail", "moepp", "atomic", "omnimoe"]
 
 
 def get_config(name: str) -> MoEConfig:

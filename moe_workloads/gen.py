@@ -109,6 +109,23 @@ def make_router_weight(cfg: MoEConfig, seed: int = 0) -> torch.Tensor:
     return _normal((cfg.n_routed, cfg.d), cfg.d ** -0.5, seed, _WR, _dt(cfg))
 
 
+def _shared_jobs(cfg: MoEConfig, w: dict, dt) -> list:
+    """Allocate the always-on SwiGLU experts' weights in ``w``; their draws."""
+    if not cfg.n_shared:
+        return []
+    d, S, Hs = cfg.d, cfg.n_shared, cfg.hidden_shared
+    sg = torch.empty((S, Hs, d), dtype=dt)
+    su = torch.empty((S, Hs, d), dtype=dt)
+    sd = torch.empty((S, d, Hs), dtype=dt)
+    jobs = []
+    for s in range(S):
+        base = _SHARED + s * 4 * 64
+        jobs += [(sg, s, (Hs, d), d ** -0.5, base + 0), (su, s, (Hs, d), d ** -0.5, base + 64),
+                 (sd, s, (d, Hs), Hs ** -0.5, base + 128)]
+    w["ws_gate"], w["ws_up"], w["ws_down"] = sg, su, sd
+    return jobs
+
+
 def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
     dt = _dt(cfg)
     d = cfg.d
@@ -126,6 +143,7 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
             for c, r0 in enumerate(range(0, cfg.n_atomic, _CHUNK_ROWS)):
                 r1 = min(cfg.n_atomic, r0 + _CHUNK_ROWS)
                 jobs.append((w[name], slice(r0, r1), (r1 - r0, d), 1024 ** -0.5, stream + c * 65536))
+        jobs += _shared_jobs(cfg, w, dt)
         _fill_parallel(jobs, seed, dt)
         return w
     H = cfg.hidden
@@ -140,16 +158,7 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
         base = _EXPERT + e * 4 * 64
         jobs += [(wg, e, (H, d), d ** -0.5, base + 0), (wu, e, (H, d), d ** -0.5, base + 64),
                  (wd, e, (d, H), H ** -0.5, base + 128)]
-    if cfg.n_shared:
-        S, Hs = cfg.n_shared, cfg.hidden_shared
-        sg = torch.empty((S, Hs, d), dtype=dt)
-        su = torch.empty((S, Hs, d), dtype=dt)
-        sd = torch.empty((S, d, Hs), dtype=dt)
-        for s in range(S):
-            base = _SHARED + s * 4 * 64
-            jobs += [(sg, s, (Hs, d), d ** -0.5, base + 0), (su, s, (Hs, d), d ** -0.5, base + 64),
-                     (sd, s, (d, Hs), Hs ** -0.5, base + 128)]
-        w["ws_gate"], w["ws_up"], w["ws_down"] = sg, su, sd
+    jobs += _shared_jobs(cfg, w, dt)
     _fill_parallel(jobs, seed, dt)
     w["w_gate"], w["w_up"], w["w_down"] = wg, wu, wd
     if cfg.n_const:

@@ -228,7 +228,8 @@ def check_atomic_layer(cfg, inp: dict, tokens=None) -> dict:
     tokens = np.asarray(tokens, dtype=np.int32)
     # outputs: oracle on the GPU's routing with gates from the fp64 scores of those experts
     g_ref = _pk_gates_for(sr, sc, idx[tokens], tokens, cfg.pk_cols)
-    y_ref = oracle.atomic_tokens(inp["x"], inp["u"], inp["v"], tokens, idx[tokens], g_ref)
+    shared = {k_: inp[k_] for k_ in ("ws_gate", "ws_up", "ws_down")} if cfg.n_shared else None
+    y_ref = oracle.atomic_tokens(inp["x"], inp["u"], inp["v"], tokens, idx[tokens], g_ref, shared=shared)
     y_gpu = b.y.float().cpu().numpy()[tokens].astype(np.float64)
     rel = assert_close(y_gpu, y_ref, "bf16")
     return rep | {"rel_err": rel, "rel_err_out": _out_err(r, tokens, y_ref)}

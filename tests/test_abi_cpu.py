@@ -50,6 +50,11 @@ def test_sizes_and_groups(abi):
     a = _desc(abi, T=8192, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512,
               pk_topk_half=32, d_query=1024)
     assert abi.moe_num_groups(a) == 512 * 512 and abi.moe_row_capacity(a) == 8192 * 64
+    o = _desc(abi, T=8192, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512,
+              pk_topk_half=32, d_query=1024, n_shared=1, hidden_shared=2816)
+    # the full layer: the shared branch's fp32 output after the task coefficients
+    assert abi.moe_num_groups(o) == 512 * 512
+    assert abi.moe_layer_workspace_size(o) >= abi.moe_layer_workspace_size(a) + 8192 * 1024 * 4
 
 
 @pytest.mark.parametrize("bad", [
@@ -63,6 +68,12 @@ def test_sizes_and_groups(abi):
          d_query=1024),                                                   # rows != cols
     dict(T=8, d_model=1024, top_k=2000, kind="atomic", pk_rows=512, pk_cols=512, pk_topk_half=32,
          d_query=1024),                                                   # K > kh^2
+    dict(T=8, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512, pk_topk_half=32,
+         d_query=1024, n_shared=2, hidden_shared=1024),                   # one shared branch at most
+    dict(T=8, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512, pk_topk_half=32,
+         d_query=1024, n_shared=1, hidden_shared=1000),                   # shared width not a multiple of 128
+    dict(T=8, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512, pk_topk_half=32,
+         d_query=1024, n_shared=0, hidden_shared=1024),                   # width without a branch
 ])
 def test_rejected_descriptors(abi, bad):
     d = _desc(abi, **bad)

@@ -72,6 +72,14 @@ def test_atomic_small_grid():
     check_atomic_layer(cfg, make_inputs(cfg))
 
 
+@pytest.mark.parametrize("T", [100, 700])      # single-CTA and CTA-pair shared GEMMs
+def test_full_omnimoe_layer_small(T):
+    """Atomic experts plus the shared dense SwiGLU branch."""
+    cfg = scaled(get_config("omnimoe"), T=T, d=256, pk_rows=64, pk_cols=64, pk_topk_half=16,
+                 top_k=32, d_query=128, hidden_shared=384)
+    check_atomic_layer(cfg, make_inputs(cfg))
+
+
 @pytest.mark.parametrize("E,T", [(2, 600), (4, 1100), (2, 513)])
 def test_cta_pair_gemm_ragged_groups(E, T):
     """>= 512 rows per expert on average: the grouped GEMMs run on CTA pairs
@@ -245,3 +253,9 @@ def test_atomic_full_size_sampled():
     cfg = get_config("atomic")
     rep = check_atomic_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 48))
     _report("atomic", rep)
+
+
+def test_omnimoe_full_size_sampled():
+    cfg = get_config("omnimoe")
+    rep = check_atomic_layer(cfg, make_inputs(cfg), tokens=_sample(cfg.T, 48))
+    _report("omnimoe", rep)
