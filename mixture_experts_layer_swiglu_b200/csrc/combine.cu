@@ -228,14 +228,6 @@ __global__ void atomic_task_meta_kernel(const AtomicArgs a)
     }
 }
 
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // ---- phase A: c[s] = g[s] * GELU(u_e . x_t) for every task.
 //
@@ -288,12 +280,6 @@ __device__ __forceinline__ PaRaw pa_load(const AtomicArgs& a, int un, int units,
     return r;
 }
 
-__device__ __forceinline__ void ld256(const unsigned char* p, uint32_t (&r)[8])
-{
-    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "l"(p));
-}
 
 // D += the products of the 64-element slices of d, in groups of U slices
 // whose loads are issued together (one tile: U * 3 KiB per warp in flight,

@@ -141,6 +141,26 @@ __device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_g
 // async-proxy (TMA) reads.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// D += A B for one m16n8k16 bf16 tile (fp32 accumulators), the legacy
+// warp-level tensor-core path: A regs {row g k 2q.., row g+8 k 2q.., row g
+// k 2q+8.., row g+8 k 2q+8..}, B regs {k 2q.., k 2q+8..} of column g.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 32-byte read-only global load (8 words), no L1 allocation.
+__device__ __forceinline__ void ld256(const unsigned char* p, uint32_t (&r)[8])
+{
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+
 // acc[0..1] += c * (w0, w1) with one packed fp32x2 FMA.
 __device__ __forceinline__ void fma2(float& a0, float& a1, float c, float w0, float w1)
 {

@@ -91,6 +91,61 @@ constexpr int R_W_BYTES = 8 * 4096;          // 8 router rows of <= 4 KiB (resid
 constexpr int R_SMEM = R_STAGES * R_TILE * R_CHUNK_BYTES + 2 * R_W_BYTES + R_WARPS * R_TPW * R_MAXROWS * 4;
 
 
+// One token's routing from its raw router logits z[0, E_r) (and the constant
+// experts' mixing logits z[E_r, E_r + 2 n_const)), in shared memory: adds the
+// bias and the previous layer's logits, writes logits_out, selects the k
+// largest (value desc, ties to the lower id) with a warp argmax, softmax gates
+// over the selected, and the constant experts' (a1, a2).
+__device__ __forceinline__ void route_token(const RouterArgs& a, int t, float* z, int lane)
+{
+    for (int e = lane; e < a.E_r; e += 32) {
+        float v = z[e];
+        if (a.bias) v += a.bias[e];
+        if (a.prev) v += a.prev[(long long)t * a.E_r + e];
+        z[e] = v;
+        if (a.logits_out) a.logits_out[(long long)t * a.E_r + e] = v;
+    }
+    __syncwarp();
+    uint32_t taken = 0;   // bit i: expert lane + 32 i already selected
+    float zsel = 0.f, z0 = 0.f;
+    int isel = -1;
+    for (int j = 0; j < a.k; ++j) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+        for (int i = 0; lane + 32 * i < a.E_r; ++i) {
+            if ((taken >> i) & 1u) continue;
+            const int e = lane + 32 * i;
+            const float v = z[e];
+            if (better(v, e, bv, bi)) { bv = v; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(FULL, bv, o);
+            const int oi = __shfl_xor_sync(FULL, bi, o);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+        if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) { zsel = bv; isel = (bi == INT_MAX) ? -1 : bi; }
+        if (j == 0) z0 = bv;
+    }
+    const float ex = (lane < a.k) ? expf(zsel - z0) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+    if (lane < a.k) {
+        a.idx[(long long)t * a.k + lane] = isel;
+        a.gate[(long long)t * a.k + lane] = ex / sum;
+    }
+    for (int c = lane; c < a.n_const; c += 32) {
+        const float l0 = z[a.E_r + 2 * c], l1 = z[a.E_r + 2 * c + 1];
+        const float m = fmaxf(l0, l1);
+        const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+        a.const_mix[((long long)t * a.n_const + c) * 2 + 0] = e0 / (e0 + e1);
+        a.const_mix[((long long)t * a.n_const + c) * 2 + 1] = e1 / (e0 + e1);
+    }
+    __syncwarp();
+}
+
 template <typename Tin>
 __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a)
 {
@@ -226,54 +281,97 @@ __global__ void __launch_bounds__(R_WARPS * 32) router_kernel(const RouterArgs a
         for (int tt = 0; tt < R_TPW; ++tt) {
             const int t = t_tile + warp * R_TPW + tt;
             if (t >= a.T) break;
-            float* z = zs[tt];
-            for (int e = lane; e < a.E_r; e += 32) {
-                float v = z[e];
-                if (a.bias) v += a.bias[e];
-                if (a.prev) v += a.prev[(long long)t * a.E_r + e];
-                z[e] = v;
-                if (a.logits_out) a.logits_out[(long long)t * a.E_r + e] = v;
-            }
-            __syncwarp();
-            uint32_t taken = 0;   // bit i: expert lane + 32 i already selected
-            float zsel = 0.f, z0 = 0.f;
-            int isel = -1;
-            for (int j = 0; j < a.k; ++j) {
-                float bv = -INFINITY;
-                int bi = INT_MAX;
-                for (int i = 0; lane + 32 * i < a.E_r; ++i) {
-                    if ((taken >> i) & 1u) continue;
-                    const int e = lane + 32 * i;
-                    const float v = z[e];
-                    if (better(v, e, bv, bi)) { bv = v; bi = e; }
-                }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    const float ov = __shfl_xor_sync(FULL, bv, o);
-                    const int oi = __shfl_xor_sync(FULL, bi, o);
-                    if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-                }
-                if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-                if (lane == j) { zsel = bv; isel = (bi == INT_MAX) ? -1 : bi; }
-                if (j == 0) z0 = bv;
-            }
-            const float ex = (lane < a.k) ? expf(zsel - z0) : 0.f;
-            float sum = ex;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-            if (lane < a.k) {
-                a.idx[(long long)t * a.k + lane] = isel;
-                a.gate[(long long)t * a.k + lane] = ex / sum;
-            }
-            for (int c = lane; c < a.n_const; c += 32) {
-                const float l0 = z[a.E_r + 2 * c], l1 = z[a.E_r + 2 * c + 1];
-                const float m = fmaxf(l0, l1);
-                const float e0 = expf(l0 - m), e1 = expf(l1 - m);
-                a.const_mix[((long long)t * a.n_const + c) * 2 + 0] = e0 / (e0 + e1);
-                a.const_mix[((long long)t * a.n_const + c) * 2 + 1] = e1 / (e0 + e1);
-            }
-            __syncwarp();
+            route_token(a, t, zs[tt], lane);
         }
+    }
+}
+
+// Router logits on the tensor cores (bf16 inputs).  A block takes 16 tokens;
+// its 4 warps split d into quarters (split-K) and each computes the partial
+// logits of all router rows (and the constant experts' mixing rows) as the N
+// side of m16n8k16 tiles, in groups of 64 rows.  For each 64-element slice of
+// d, lane (g, q) loads 32 contiguous bytes of its A rows (tokens g, g+8) and
+// B rows (router row g of each n8 tile), which feed four k16 steps in the
+// same k order for A and B.  bf16 x bf16 products are exact in fp32 and
+// accumulate in fp32, as in the FMA kernel (only the order of the sums
+// differs); the four partials are added in warp order.  Each warp then
+// routes 4 of the 16 tokens with route_token.
+constexpr int RM_WARPS = 4;
+constexpr int RM_NG = 8;                     // n8 tiles per group: 64 router rows
+
+__global__ void __launch_bounds__(RM_WARPS * 32) router_mma_kernel(const RouterArgs a)
+{
+    extern __shared__ __align__(16) float rm_z[];   // [RM_WARPS][16][zpitch] partial logits
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, wib = threadIdx.x >> 5;
+    const int R = a.E_r + 2 * a.n_const;
+    const int zpitch = (R + 7) & ~7;
+    float* zw = rm_z + (size_t)wib * 16 * zpitch;
+    const size_t rowb = (size_t)a.d * 2;
+    const unsigned char* xb = static_cast<const unsigned char*>(a.x);
+    const unsigned char* wr = static_cast<const unsigned char*>(a.w_router);
+    const unsigned char* wc = static_cast<const unsigned char*>(a.w_const_mix);
+    const int nsc = a.d / 64;
+    const int sc0 = wib * nsc / RM_WARPS, sc1 = (wib + 1) * nsc / RM_WARPS;   // this warp's slices
+    const int tiles = (a.T + 15) / 16;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int t0 = tile * 16;
+        const unsigned char* xr0 = xb + (size_t)min(t0 + g, a.T - 1) * rowb;
+        const unsigned char* xr1 = xb + (size_t)min(t0 + g + 8, a.T - 1) * rowb;
+        for (int n0 = 0; n0 < R; n0 += 8 * RM_NG) {
+            const unsigned char* wrow[RM_NG];
+#pragma unroll
+            for (int nt = 0; nt < RM_NG; ++nt) {
+                const int j = min(n0 + nt * 8 + g, R - 1);   // rows past R repeat the last; never read
+                wrow[nt] = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
+            }
+            const int ntiles = min(RM_NG, (R - n0 + 7) / 8);
+            float acc[RM_NG][4];
+#pragma unroll
+            for (int nt = 0; nt < RM_NG; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 1
+            for (int sc = sc0; sc < sc1; ++sc) {
+                const int off = sc * 128 + q * 32;
+                uint32_t xa[8], xb2[8];
+                ld256(xr0 + off, xa);
+                ld256(xr1 + off, xb2);
+#pragma unroll
+                for (int nt = 0; nt < RM_NG; ++nt) {
+                    if (nt < ntiles) {
+                        uint32_t w[8];
+                        ld256(wrow[nt] + off, w);
+#pragma unroll
+                        for (int st = 0; st < 4; ++st)
+                            mma_16816(acc[nt], xa[2 * st], xb2[2 * st], xa[2 * st + 1], xb2[2 * st + 1], w[2 * st],
+                                      w[2 * st + 1]);
+                    }
+                }
+            }
+            // D fragment: acc[0], acc[1] = token g, rows 2q, 2q+1; acc[2], acc[3] = token g+8
+#pragma unroll
+            for (int nt = 0; nt < RM_NG; ++nt) {
+                const int col = n0 + nt * 8 + 2 * q;
+                if (nt < ntiles && col < zpitch) {
+                    zw[g * zpitch + col] = acc[nt][0];
+                    zw[g * zpitch + col + 1] = acc[nt][1];
+                    zw[(g + 8) * zpitch + col] = acc[nt][2];
+                    zw[(g + 8) * zpitch + col + 1] = acc[nt][3];
+                }
+            }
+        }
+        __syncthreads();
+        // sum the partials in warp order into warp 0's buffer
+        for (int i = threadIdx.x; i < 16 * zpitch; i += RM_WARPS * 32) {
+            float v = rm_z[i];
+#pragma unroll
+            for (int w2 = 1; w2 < RM_WARPS; ++w2) v += rm_z[(size_t)w2 * 16 * zpitch + i];
+            rm_z[i] = v;
+        }
+        __syncthreads();
+        for (int tt = wib; tt < 16; tt += RM_WARPS) {
+            const int t = t0 + tt;
+            if (t < a.T) route_token(a, t, rm_z + tt * zpitch, lane);
+        }
+        __syncthreads();   // buffers free for the next tile
     }
 }
 
@@ -505,6 +603,20 @@ __global__ void pk_prep_keys_kernel(const __nv_bfloat16* kr, const __nv_bfloat16
 moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
+    if (dtype == MOE_BF16 && a.d % 64 == 0) {
+        const int R = a.E_r + 2 * a.n_const;
+        const int smem = RM_WARPS * 16 * ((R + 7) & ~7) * 4;
+        static bool mma_attr = false;
+        if (!mma_attr) {
+            cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RM_WARPS * 16 * 256 * 4);
+            mma_attr = true;
+        }
+        const int tiles = cdiv(a.T, 16);
+        const int grid = std::max(1, std::min(tiles, num_sms() * 8));
+        router_mma_kernel<<<grid, RM_WARPS * 32, smem, st>>>(a);
+        count_launch();
+        return cuda_status(cudaGetLastError());
+    }
     const int grid = std::max(1, std::min(cdiv(a.T, R_TILE), num_sms()));
     static bool attr_done = false;
     if (!attr_done) {
