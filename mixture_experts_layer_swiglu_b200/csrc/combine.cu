@@ -552,13 +552,15 @@ __global__ void __launch_bounds__(PB_WARPS * 32, 1) atomic_phase_b_kernel(const 
 template <template <int> class K, typename... Args>
 moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
 {
+    cudaError_t e;
     switch (nv) {
-        case 1: K<1>::launch(grid, st, a); break;
-        case 2: K<2>::launch(grid, st, a); break;
-        case 4: K<4>::launch(grid, st, a); break;
-        case 8: K<8>::launch(grid, st, a); break;
+        case 1: e = K<1>::launch(grid, st, a); break;
+        case 2: e = K<2>::launch(grid, st, a); break;
+        case 4: e = K<4>::launch(grid, st, a); break;
+        case 8: e = K<8>::launch(grid, st, a); break;
         default: return MOE_ERR_UNSUPPORTED;
     }
+    if (e != cudaSuccess) return cuda_status(e);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
@@ -566,14 +568,12 @@ moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
 constexpr int kPbSmem = PB_WARPS * PB_STAGES * (PB_STAGE + 8);
 
 template <int NV> struct PhaseB {
-    static void launch(int grid, cudaStream_t st, const AtomicArgs& a)
+    static cudaError_t launch(int grid, cudaStream_t st, const AtomicArgs& a)
     {
-        static bool attr_done = false;
-        if (!attr_done) {
-            cudaFuncSetAttribute(atomic_phase_b_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPbSmem);
-            attr_done = true;
-        }
+        const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(atomic_phase_b_kernel<NV>), kPbSmem);
+        if (e != cudaSuccess) return e;
         atomic_phase_b_kernel<NV><<<grid, PB_WARPS * 32, kPbSmem, st>>>(a);
+        return cudaSuccess;
     }
 };
 

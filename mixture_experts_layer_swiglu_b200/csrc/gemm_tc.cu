@@ -736,7 +736,6 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     if (EPI == EPI_PK_SPLIT) mo = mA;   // direct stores; the map is unused
     else if (!make_out_map(&mo, p.out, std::min<long long>(p.rows_cap, 1ll << 31), p.N, p.ldo, EPI == EPI_F32))
         return MOE_ERR_CUDA;
-    static bool attr_done = false, attr_pair_done = false;
     DevArgs a;
     a.offsets = p.offsets;
     a.n_groups = p.n_groups;
@@ -753,22 +752,14 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
     const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
     if (p.pair) {
-        if (!attr_pair_done) {
-            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-            if (e != cudaSuccess) return cuda_status(e);
-            attr_pair_done = true;
-        }
+        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_pair_kernel<EPI>), P_SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
         const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
         const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
         grouped_gemm_pair_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, mo, a);
     } else {
-        if (!attr_done) {
-            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-            if (e != cudaSuccess) return cuda_status(e);
-            attr_done = true;
-        }
+        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI>), SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
         const long long tiles_ub = (long long)(cdiv((int)rows, BM) + p.n_groups) * ntn;
         const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms()));
         grouped_gemm_kernel<EPI><<<grid, NTHREADS, SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, mo, a);

@@ -14,6 +14,9 @@ inline void count_launch(int n = 1) { t_launches += n; }
 
 moe_status cuda_status(cudaError_t e);
 int num_sms();
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device (the attribute belongs to each device's context), once per device.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
 moe_status validate_desc(const moe_layer_desc* d);   // the descriptor checks of every entry point
 
 // ------------------------------------------------------------ grouped GEMM

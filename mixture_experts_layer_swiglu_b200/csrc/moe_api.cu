@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <map>
 #include <mutex>
 
 #include "common.cuh"
@@ -19,6 +20,21 @@ __device__ int g_status = 0;
 thread_local int t_launches = 0;
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaError_t ensure_smem_attr(const void* func, int bytes)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int& have = done[{func, dev}];
+    if (have >= bytes) return cudaSuccess;
+    if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) == cudaSuccess)
+        have = bytes;
+    return e;
+}
 
 int num_sms()
 {

@@ -606,11 +606,8 @@ moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
     if (dtype == MOE_BF16 && a.d % 64 == 0) {
         const int R = a.E_r + 2 * a.n_const;
         const int smem = RM_WARPS * 16 * ((R + 7) & ~7) * 4;
-        static bool mma_attr = false;
-        if (!mma_attr) {
-            cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RM_WARPS * 16 * 256 * 4);
-            mma_attr = true;
-        }
+        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(router_mma_kernel), smem);
+        if (e != cudaSuccess) return cuda_status(e);
         const int tiles = cdiv(a.T, 16);
         const int grid = std::max(1, std::min(tiles, num_sms() * 8));
         router_mma_kernel<<<grid, RM_WARPS * 32, smem, st>>>(a);
@@ -618,12 +615,10 @@ moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
         return cuda_status(cudaGetLastError());
     }
     const int grid = std::max(1, std::min(cdiv(a.T, R_TILE), num_sms()));
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM);
-        cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM);
-        attr_done = true;
-    }
+    cudaError_t e = dtype == MOE_BF16
+                        ? ensure_smem_attr(reinterpret_cast<const void*>(router_kernel<__nv_bfloat16>), R_SMEM)
+                        : ensure_smem_attr(reinterpret_cast<const void*>(router_kernel<float>), R_SMEM);
+    if (e != cudaSuccess) return cuda_status(e);
     if (dtype == MOE_BF16) router_kernel<__nv_bfloat16><<<grid, R_WARPS * 32, R_SMEM, st>>>(a);
     else router_kernel<float><<<grid, R_WARPS * 32, R_SMEM, st>>>(a);
     count_launch();
@@ -634,14 +629,12 @@ moe_status launch_pk_select(const PkSelectArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
     constexpr int warps = 8;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaFuncSetAttribute(pk_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             warps * (int)sizeof(PkWarpSmem<16>));
-        cudaFuncSetAttribute(pk_select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             warps * (int)sizeof(PkWarpSmem<32>));
-        attr_done = true;
-    }
+    const int n_max = std::max(a.rows, a.cols);
+    cudaError_t e = n_max <= 512 ? ensure_smem_attr(reinterpret_cast<const void*>(pk_select_kernel<16>),
+                                                    warps * (int)sizeof(PkWarpSmem<16>))
+                                 : ensure_smem_attr(reinterpret_cast<const void*>(pk_select_kernel<32>),
+                                                    warps * (int)sizeof(PkWarpSmem<32>));
+    if (e != cudaSuccess) return cuda_status(e);
     const int grid = std::max(1, std::min(cdiv(a.T, warps), num_sms() * MOE_PK_MINB));
     const int n = std::max(a.rows, a.cols);
     if (n <= 512) pk_select_kernel<16><<<grid, warps * 32, warps * sizeof(PkWarpSmem<16>), st>>>(a);
