@@ -16,6 +16,10 @@
 //            MMAs of the next.
 //   warps 2-5 epilogue: tcgen05.ld of their 32-lane quarter, fused
 //            activation (SwiGLU: silu(gate) * up), bf16/fp32 store.
+// Two more forms run on clusters of two CTAs (tcgen05.mma.cta_group::2,
+// M = 256): 256-row tiles of a group's rows, and the token-column form
+// (weight rows as M, a group's rows as N in steps of 16), which the pair form
+// uses for the fp32 down projection and for SwiGLU from K = 2048.
 // Every mbarrier wait is bounded (2 s); a timeout sets MOE_ERR_TIMEOUT, all
 // roles leave their loops, in-flight TMA copies are drained and TMEM freed.
 
@@ -665,6 +669,371 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     }
 }
 
+// ------------------------------------------------ token-column pair kernel
+//
+// The pair kernel above makes a group's rows the MMA's M side, so a group
+// whose row count is not a multiple of 256 pays for a whole 256-row tile at
+// its end: Mixtral-shaped groups of about 1024 +- 30 rows cost 36 tiles of
+// MMA work for 32 tiles of rows, and the last wave of the static schedule
+// decides the time.  This form swaps the operands: the expert's weight rows
+// are M (256 per pair, always full) and the group's rows are N, which the
+// tensor cores take in steps of 16.  A group of c rows is cut into
+// ceil(c / 256) token tiles of one width w = ceil16(c / that count), so the
+// tiles of a group cost the same, the round-robin schedule stays balanced and
+// the padding is under 16 rows per tile.  Tile order: group, weight block,
+// token tile (the token tiles sharing a weight block run side by side).
+//   fp32 epilogue (down projection): TMEM lane = output feature, column =
+//     token; each warp stores one token's 32 features (128 B) per instruction.
+//   SwiGLU epilogue: each CTA stages 64 gate rows and the 64 up rows of the
+//     same hidden units as its 128 A rows, so TMEM lanes 0-63 hold gate and
+//     lanes 64-127 up of the same units; epilogue warps q and q + 2 swap
+//     half of each 32-column chunk through shared memory and each applies
+//     silu(gate) * up to its half.
+// Used for the pair form's SwiGLU (N % 128 == 0) and fp32 (N % 256 == 0)
+// epilogues; the other forms keep the row-tiled kernels.
+
+#ifndef MOE_GEMM_TN
+#define MOE_GEMM_TN 1
+#endif
+#ifndef MOE_TN_SWIGLU_MIN_K
+#define MOE_TN_SWIGLU_MIN_K 2048
+#endif
+
+struct TnTile {
+    int g;        // group
+    int m;        // weight block (256 output features, or 128 hidden units for SwiGLU)
+    int tok0;     // first row of the token tile
+    int valid;    // rows of the tile (1..256)
+    int nt;       // MMA N: valid rounded up to 16
+};
+
+__device__ __forceinline__ int tn_width(int cnt)
+{
+    const int t = cdiv(cnt, 256);
+    return (cdiv(cnt, t) + 15) & ~15;
+}
+
+__device__ __forceinline__ int tn_tiles(int cnt, int ntm)
+{
+    return cnt > 0 ? cdiv(cnt, tn_width(cnt)) * ntm : 0;
+}
+
+__device__ __forceinline__ TnTile decode_tn(int tile, const int* tile_start, const int* g_lo, const int* g_cnt,
+                                            int n_groups, int ntm)
+{
+    int lo = 0, hi = n_groups - 1;   // last g with tile_start[g] <= tile
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    TnTile ti;
+    ti.g = lo;
+    const int cnt = g_cnt[lo];
+    const int w = tn_width(cnt);
+    const int nj = cdiv(cnt, w);
+    const int local = tile - tile_start[lo];
+    ti.m = local / nj;
+    const int j = local - ti.m * nj;
+    ti.tok0 = g_lo[lo] + j * w;
+    ti.valid = min(w, cnt - j * w);
+    ti.nt = (ti.valid + 15) & ~15;
+    return ti;
+}
+
+__device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, int lane, int* tile_start,
+                                                     int* g_lo, int* g_cnt)
+{
+    const int n = a.n_groups;
+    const int chunk = cdiv(n, 32);
+    const int g0 = min(n, lane * chunk), g1 = min(n, g0 + chunk);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+        int lo, hi;
+        if (a.offsets) { lo = a.offsets[g]; hi = a.offsets[g + 1]; }
+        else { lo = g * a.group_rows; hi = lo + a.group_rows; }
+        int cnt = hi - lo;
+        if (cnt < 0 || lo < 0) { set_status(MOE_ERR_DEVICE_BOUNDS); cnt = 0; lo = 0; }
+        g_lo[g] = lo;
+        g_cnt[g] = cnt;
+        local += tn_tiles(cnt, ntm);
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+        tile_start[g] = run;
+        run += tn_tiles(g_cnt[g], ntm);
+    }
+    if (lane == 31) tile_start[n] = incl;
+}
+
+// Named barrier of the two warps (64 threads) of one SwiGLU epilogue team.
+__device__ __forceinline__ void team_sync(int id)
+{
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
+// Team barrier that also returns whether `v` holds in every thread of both warps.
+__device__ __forceinline__ bool team_all(bool v, int id)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, 64, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v), "r"(id) : "memory");
+    return r != 0;
+}
+
+// Runs body(v, ch) over the 32-column chunks 0..nch-1 of an accumulator,
+// loading chunk ch + 1 from TMEM while chunk ch is processed.
+template <typename F>
+__device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body)
+{
+    uint32_t va[32], vb[32];
+    tmem_ld32(tacc, va);
+    tc_wait_ld_regs(va);
+#pragma unroll 1
+    for (int ch = 0; ch < nch; ch += 2) {
+        const bool more = ch + 1 < nch;
+        if (more) tmem_ld32(tacc + (ch + 1) * 32, vb);
+        body(va, ch);
+        if (more) {
+            tc_wait_ld_regs(vb);
+            if (ch + 2 < nch) tmem_ld32(tacc + (ch + 2) * 32, va);
+            body(vb, ch + 1);
+            if (ch + 2 < nch) tc_wait_ld_regs(va);
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW0,
+                       const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
+                       const __grid_constant__ CUtensorMap tmW3, const DevArgs a)
+{
+    static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "token-column form: SwiGLU or fp32 epilogue");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + P_STAGES * P_TILE_A;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + P_STAGES * P_TILE_B);
+    uint64_t* empty = full + P_STAGES;
+    uint64_t* acc_full = empty + P_STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* mma_done = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* tile_start = reinterpret_cast<int*>(smem + P_STAGES * P_STAGE_BYTES + 256);
+    int* g_lo = tile_start + (kMaxGemmGroups + 1);
+    int* g_cnt = g_lo + kMaxGemmGroups;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int ntm = (EPI == EPI_SWIGLU) ? a.N / 128 : a.N / 256;   // weight blocks per expert
+
+    if (warp == 0) build_group_table_tn(a, ntm, lane, tile_start, g_lo, g_cnt);
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) { tmem_alloc_pair(tmem_slot, TMEM_COLS); tmem_relinquish_pair(); }
+    if (threadIdx.x == 64) {
+        tma_prefetch_desc(&tmX); tma_prefetch_desc(&tmW0); tma_prefetch_desc(&tmW1);
+        tma_prefetch_desc(&tmW2); tma_prefetch_desc(&tmW3);
+    }
+    tc_fence_before();
+    cluster_sync_all();          // both CTAs: barriers initialised, TMEM allocated
+    tc_fence_after();
+
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[a.n_groups];
+    const int pnk = cdiv(a.K, BK * P_KH);
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const uint32_t full_leader = mapa_shared(smem_u32(&full[0]), 0);
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // -------------------------------------------- TMA producer (both CTAs)
+            int s = 0;
+            uint32_t ph = 0;
+            bool bad = false;
+            for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
+                const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+                const bool first = ti.g < a.n_first;
+                const int gb = first ? ti.g : ti.g - a.n_first;
+                // A: weight rows of this CTA's half of M; B: this CTA's half of the tokens
+                const int wrow = (EPI == EPI_SWIGLU) ? gb * a.N + ti.m * 128 + (int)rank * 64
+                                                     : gb * a.N + ti.m * 256 + (int)rank * 128;
+                const CUtensorMap* mw = first ? &tmW0 : &tmW2;
+                const CUtensorMap* mu = first ? &tmW1 : &tmW3;
+                const int xrow = ti.tok0 + (int)rank * (ti.nt >> 1);
+                if (*abort_flag) { bad = true; break; }
+                for (int kb = 0; kb < pnk; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
+#pragma unroll
+                    for (int h = 0; h < P_KH; ++h) {
+                        const int k0 = (kb * P_KH + h) * BK;      // past K: zero fill
+                        uint8_t* da = sA + s * P_TILE_A + h * P_HALF;
+                        if (EPI == EPI_SWIGLU) {   // 64 gate rows, then the 64 up rows of the same units
+                            tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
+                            tma_load_2d_pair(da + P_HALF / 2, mu, full_leader + 8 * s, k0, wrow);
+                        } else {
+                            tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
+                        }
+                        tma_load_2d_pair(sB + s * P_TILE_B + h * P_HALF, &tmX, full_leader + 8 * s, k0, xrow);
+                    }
+                    if (++s == P_STAGES) { s = 0; ph ^= 1; }
+                }
+            }
+            if (bad) {   // copies already issued land within microseconds; let them
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) { }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // -------------------------------------------- MMA issuer (leader only)
+            int s = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            bool bad = false;
+            const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
+            const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
+            for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
+                const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+                const uint32_t idesc = idesc_bf16_f32(P_BM, ti.nt);
+                if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < pnk; ++kb) {
+                    if (!mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
+                    const uint64_t ad = ad0 + (uint64_t)((s * P_TILE_A) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)((s * P_TILE_B) >> 4);
+#pragma unroll
+                    for (int h = 0; h < P_KH; ++h)
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma_bf16_pair(d_tmem, ad + (h * P_HALF >> 4) + 2 * kk, bd + (h * P_HALF >> 4) + 2 * kk,
+                                             idesc, (kb | h | kk) != 0);
+                    tc_commit_pair(&empty[s], 0x3);
+                    if (++s == P_STAGES) { s = 0; ph ^= 1; }
+                }
+                if (bad) break;
+                tc_commit_pair(&acc_full[acc], 0x3);
+                if (++acc == 2) { acc = 0; aph ^= 1; }
+            }
+            tc_commit_pair(mma_done, 0x1);
+            mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;                   // TMEM lanes 32q .. 32q + 31
+        uint8_t* epi0 = smem + epi_stage_offset(P_STAGES * P_STAGE_BYTES);
+        float* mine = reinterpret_cast<float*>(epi0 + (warp - 2) * EPI_STAGE_BYTES);
+        const float* theirs = reinterpret_cast<const float*>(epi0 + ((warp - 2) ^ 2) * EPI_STAGE_BYTES);
+        const bool gate_warp = q < 2;
+        const int team = 1 + (q & 1);             // named barrier id of warps q and q ^ 2
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int tile = cluster; tile < total; tile += n_clusters) {
+            const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+            bool ok = !*abort_flag && mbar_wait(&acc_full[acc], aph);
+            if (EPI == EPI_SWIGLU) ok = team_all(ok, team);   // both warps of a team leave together
+            if (!ok) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+            const int nch = cdiv(ti.valid, 32);
+            // Each chunk is turned in shared memory from (lane = feature, column =
+            // token) into token rows, which the warp writes as 16-byte pieces.
+            if constexpr (EPI == EPI_F32) {
+                float* out = reinterpret_cast<float*>(a.out);
+                float* stg = mine;                        // [32 tokens][32 features]
+                const int f0 = ti.m * 256 + (int)rank * 128 + q * 32;
+                tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
+                    __syncwarp();                         // the previous chunk has been read
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = __uint_as_float(v[i]);
+                    __syncwarp();
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int idx = r * 32 + lane, row = idx >> 3, piece = idx & 7;
+                        const int c = ch * 32 + row;
+                        const long long grow = (long long)ti.tok0 + c;
+                        if (c < ti.valid && grow < a.rows_cap)
+                            *reinterpret_cast<float4*>(out + grow * a.ldo + f0 + piece * 4) =
+                                *reinterpret_cast<const float4*>(stg + row * 32 + piece * 4);
+                    }
+                });
+            } else {
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+                __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(mine) + 2048);
+                const int unit0 = ti.m * 128 + (int)rank * 64 + (q & 1) * 32;
+                // the gate warp finishes columns 0-15 of each chunk, the up warp 16-31
+                auto finish = [&](const float (&g)[16], const float (&u)[16], int c0) {
+                    __syncwarp();                         // the previous chunk has been read
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)          // [16 tokens][32 units]
+                        stg[i * 32 + lane] = __float2bfloat16_rn(__fdividef(g[i], 1.0f + __expf(-g[i])) * u[i]);
+                    __syncwarp();
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int idx = r * 32 + lane, row = idx >> 2, piece = idx & 3;
+                        const int c = c0 + row;
+                        const long long grow = (long long)ti.tok0 + c;
+                        if (c < ti.valid && grow < a.rows_cap)
+                            *reinterpret_cast<uint4*>(out + grow * a.ldo + unit0 + piece * 8) =
+                                *reinterpret_cast<const uint4*>(stg + row * 32 + piece * 8);
+                    }
+                };
+                tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
+                    team_sync(team);                      // the partner has read the previous chunk
+                    float g[16], u[16];
+                    if (gate_warp) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = __uint_as_float(v[16 + i]);
+                        team_sync(team);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) { g[i] = __uint_as_float(v[i]); u[i] = theirs[i * 32 + lane]; }
+                        finish(g, u, ch * 32);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = __uint_as_float(v[i]);
+                        team_sync(team);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) { g[i] = theirs[i * 32 + lane]; u[i] = __uint_as_float(v[16 + i]); }
+                        finish(g, u, ch * 32 + 16);
+                    }
+                });
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8 * acc);
+            if (++acc == 2) { acc = 0; aph ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();          // all MMAs done and all TMEM reads issued in both CTAs
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -686,8 +1055,8 @@ EncodeTiledFn get_encode()
     return fn;
 }
 
-// bf16 [rows, K] row-major, box {64 (K), 128 rows}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int K)
+// bf16 [rows, K] row-major, box {64 (K), box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows = 128)
 {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
@@ -696,7 +1065,7 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int K)
     }
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, 128};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -730,8 +1099,18 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     const void* b3 = p.B3 ? p.B3 : (p.B2 ? p.B2 : b1);
     const long long r23 = p.B2 ? p.b23_rows : p.b01_rows;
     const int kb = p.b_kmod > 0 ? p.b_kmod : p.K;   // B's own K extent
-    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, kb) ||
-        !make_map(&m1, b1, p.b01_rows, kb) || !make_map(&m2, b2, r23, kb) || !make_map(&m3, b3, r23, kb))
+    // token-column form: weight rows are the MMA's M side (SwiGLU stages 64
+    // gate + 64 up rows per CTA, so its weight boxes are 64 rows high)
+    // (SwiGLU from K = MOE_TN_SWIGLU_MIN_K: its epilogue swaps halves between
+    // warps, which a short mainloop does not hide; measured on B200, K = 1024
+    // shared-branch gate/up 72 us row-tiled vs 84 us in this form)
+    const bool tn = MOE_GEMM_TN && p.pair && p.b_kmod == 0 &&
+                    ((EPI == EPI_SWIGLU && p.N % 128 == 0 && p.K >= MOE_TN_SWIGLU_MIN_K) ||
+                     (EPI == EPI_F32 && p.N % 256 == 0));
+    const int wbox = (tn && EPI == EPI_SWIGLU) ? 64 : 128;
+    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, kb, wbox) ||
+        !make_map(&m1, b1, p.b01_rows, kb, wbox) || !make_map(&m2, b2, r23, kb, wbox) ||
+        !make_map(&m3, b3, r23, kb, wbox))
         return MOE_ERR_CUDA;
     if (EPI == EPI_PK_SPLIT) mo = mA;   // direct stores; the map is unused
     else if (!make_out_map(&mo, p.out, std::min<long long>(p.rows_cap, 1ll << 31), p.N, p.ldo, EPI == EPI_F32))
@@ -751,6 +1130,18 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     a.pk_dq = p.pk_dq;
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
     const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
+    if constexpr (EPI == EPI_SWIGLU || EPI == EPI_F32) {
+        if (tn) {
+            cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI>), P_SMEM_BYTES);
+            if (e != cudaSuccess) return cuda_status(e);
+            // a group of c rows has at most ceil(c / 256) token tiles
+            const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
+            const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
+            grouped_gemm_tn_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+            count_launch();
+            return cuda_status(cudaGetLastError());
+        }
+    }
     if (p.pair) {
         cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_pair_kernel<EPI>), P_SMEM_BYTES);
         if (e != cudaSuccess) return cuda_status(e);

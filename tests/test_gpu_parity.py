@@ -80,12 +80,23 @@ def test_full_omnimoe_layer_small(T):
     check_atomic_layer(cfg, make_inputs(cfg))
 
 
-@pytest.mark.parametrize("E,T", [(2, 600), (4, 1100), (2, 513)])
-def test_cta_pair_gemm_ragged_groups(E, T):
-    """>= 512 rows per expert on average: the grouped GEMMs run on CTA pairs
-    (256-row tiles); group sizes are not multiples of 256."""
-    cfg = scaled(get_config("mixtral"), T=T, d=512, hidden=1024, n_ffn=E)
+@pytest.mark.parametrize("E,T,d", [(2, 600, 512), (4, 1100, 2048), (2, 513, 512)])
+def test_cta_pair_gemm_ragged_groups(E, T, d):
+    """>= 512 rows per expert on average: the grouped GEMMs run on CTA pairs;
+    group sizes are not multiples of 256.  d = 2048 takes the token-column
+    form for the SwiGLU GEMM too (d = 512: row tiles for it)."""
+    cfg = scaled(get_config("mixtral"), T=T, d=d, hidden=1024, n_ffn=E)
     check_swiglu_layer(cfg, make_inputs(cfg))
+
+
+def test_cta_pair_gemm_nearly_empty_group():
+    """CTA-pair GEMMs with one group of ~1090 rows and one of a few rows:
+    the small group's token tile is narrower than 32 rows (MMA N = 16)."""
+    cfg = scaled(get_config("mixtral"), T=1100, d=2048, hidden=1024, n_ffn=2, top_k=1)
+    inp = make_inputs(cfg)
+    inp["router_bias"] = torch.tensor([3.5, 0.0])
+    rep = check_swiglu_layer(cfg, inp)
+    assert rep["R"] == 1100
 
 
 def test_atomic_cta_pair_router():
