@@ -1104,7 +1104,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     // (SwiGLU from K = MOE_TN_SWIGLU_MIN_K: its epilogue swaps halves between
     // warps, which a short mainloop does not hide; measured on B200, K = 1024
     // shared-branch gate/up 72 us row-tiled vs 84 us in this form)
-    const bool tn = MOE_GEMM_TN && p.pair && p.b_kmod == 0 &&
+    // (its epilogue writes 16-byte pieces of output rows: row stride and base aligned)
+    const bool tn = MOE_GEMM_TN && p.pair && p.b_kmod == 0 && p.ldo % 8 == 0 &&
+                    reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
                     ((EPI == EPI_SWIGLU && p.N % 128 == 0 && p.K >= MOE_TN_SWIGLU_MIN_K) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));
     const int wbox = (tn && EPI == EPI_SWIGLU) ? 64 : 128;
