@@ -260,7 +260,9 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
  * Asynchronous on `stream`: y_host is complete when `stream` reaches this
  * point (the internal streams are joined back into `stream`, so the call can
  * be captured in a CUDA graph).  Calls from several host threads on one
- * device share the internal streams (correct, but not concurrent).
+ * device share the internal streams and events: a per-device lock orders
+ * their enqueueing, so they are correct but their copies do not overlap
+ * each other.
  */
 MOE_API int64_t moe_layer_host_workspace_size(const moe_layer_desc* desc, int chunks);
 MOE_API moe_status moe_layer_forward_host(const moe_layer_desc* desc, const moe_layer_weights* w,

@@ -536,6 +536,10 @@ namespace {
 constexpr int kMaxHostChunks = 8;
 
 struct HostPipe {                       // per device: two copy streams and their events
+    // Held while one call enqueues its copies, records and waits: the events
+    // are shared, and a wait binds to an event's latest record, so another
+    // call's records in between would make this call wait on the wrong work.
+    std::mutex call_mu;
     bool ok = false;
     cudaStream_t in = nullptr, out = nullptr;
     cudaEvent_t fork = nullptr;
@@ -738,6 +742,7 @@ moe_status moe_layer_forward_host(const moe_layer_desc* d, const moe_layer_weigh
     if (d->T == 0) return MOE_OK;
     HostPipe* pp = host_pipe();
     if (!pp) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> call_lock(pp->call_mu);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char* base = static_cast<char*>(workspace);
     void* layer_ws = base;
