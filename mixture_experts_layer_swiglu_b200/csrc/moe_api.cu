@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <map>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -38,16 +39,16 @@ cudaError_t ensure_smem_attr(const void* func, int bytes)
 
 int num_sms()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];         // per device; 0 = not looked up yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
     if (dev < 0 || dev >= 64) dev = 0;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 namespace {
