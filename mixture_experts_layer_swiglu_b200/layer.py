@@ -94,6 +94,13 @@ def run_stages(desc, weights, x, bufs: StageBuffers, prev_logits=None, stream=No
     return b.y
 
 
+def _check_2d(name: str, t, rows: int, cols: int, dtype) -> None:
+    if t is None:
+        return
+    if t.dim() != 2 or tuple(t.shape) != (rows, cols) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected a [{rows}, {cols}] {dtype} tensor, got {list(t.shape)} {t.dtype}")
+
+
 class MoELayer:
     """One MoE FFN layer with device-resident weights; forward() = moe_layer_forward."""
 
@@ -111,7 +118,19 @@ class MoELayer:
             self._workspace = torch.empty((need,), dtype=torch.uint8, device=device)
         return self._workspace
 
+    def _check_io(self, x, prev_logits=None, logits_out=None, y=None) -> None:
+        """The library reads and writes these through raw pointers sized by the
+        descriptor, so their shapes and dtypes must be the descriptor's."""
+        d = self.desc
+        _check_2d("x", x, d.T, d.d_model, torch_dtype(d))
+        _check_2d("y", y, d.T, d.d_model, out_dtype(d))
+        if prev_logits is not None and d.kind != abi.MOE_EXPERT_SWIGLU:
+            raise ValueError("prev_logits: the gating residual belongs to the SwiGLU kind")
+        _check_2d("prev_logits", prev_logits, d.T, router_width(d), torch.float32)
+        _check_2d("logits_out", logits_out, d.T, router_width(d), torch.float32)
+
     def forward(self, x: torch.Tensor, prev_logits=None, logits_out=None, y=None, stream=None):
+        self._check_io(x, prev_logits, logits_out, y)
         if y is None:
             y = torch.empty(x.shape, dtype=out_dtype(self.desc), device=x.device)
         abi.moe_layer_forward(self.desc, self._ws_struct, x, prev_logits, y, logits_out,
@@ -123,6 +142,7 @@ class MoELayer:
         """moe_layer_forward_host: x from host memory, y to host memory, the
         copies pipelined against the layer in token ranges.  Returns y_host
         (complete once `stream` reaches this point)."""
+        self._check_io(x_host, prev_logits, None, y_host)
         device = torch.device(device or "cuda")
         if y_host is None:
             y_host = torch.empty(x_host.shape, dtype=out_dtype(self.desc), pin_memory=True)

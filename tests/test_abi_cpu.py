@@ -110,3 +110,35 @@ def test_argument_errors_without_a_device(abi):
     assert lib.moe_layer_forward_host(ctypes.byref(a), ctypes.byref(w), 16, 16, 16, 0, 16, 1 << 30, None) == 1
     assert lib.moe_last_launch_count() == 0
     assert abi.status_string(3) == "workspace too small"
+
+
+def test_layer_object_rejects_buffers_that_disagree_with_the_descriptor():
+    """MoELayer hands raw pointers to the library, sized by the descriptor: a
+    tensor of another shape or dtype is refused before any device work."""
+    import torch
+
+    from mixture_experts_layer_swiglu_b200 import layer as L
+
+    desc = L.make_desc(T=8, d_model=256, top_k=2, dtype="bf16", n_ffn=4, hidden=256, n_zero=1)
+    lay = L.MoELayer(desc, {})
+    bf, f32 = torch.bfloat16, torch.float32
+    bad_calls = [
+        lambda: lay.forward(torch.zeros(9, 256, dtype=bf)),                           # rows
+        lambda: lay.forward(torch.zeros(8, 128, dtype=bf)),                           # width
+        lambda: lay.forward(torch.zeros(8, 256, dtype=f32)),                          # dtype
+        lambda: lay.forward(torch.zeros(8 * 256, dtype=bf)),                          # rank
+        lambda: lay.forward(torch.zeros(8, 256, dtype=bf), y=torch.zeros(8, 256, dtype=f32)),
+        lambda: lay.forward(torch.zeros(8, 256, dtype=bf), prev_logits=torch.zeros(8, 4, dtype=f32)),
+        lambda: lay.forward(torch.zeros(8, 256, dtype=bf), logits_out=torch.zeros(8, 5, dtype=bf)),
+        lambda: lay.forward_host(torch.zeros(8, 256, dtype=bf), y_host=torch.zeros(7, 256, dtype=bf)),
+    ]
+    for call in bad_calls:
+        with pytest.raises(ValueError, match="expected a"):
+            call()
+    # the right shapes pass the check and reach the device-pointer step (host tensors here)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        lay.forward(torch.zeros(8, 256, dtype=bf), prev_logits=torch.zeros(8, 5, dtype=f32))
+    atomic = L.make_desc(T=8, d_model=256, top_k=4, dtype="bf16", kind="atomic", pk_rows=32, pk_cols=32,
+                         pk_topk_half=4, d_query=64)
+    with pytest.raises(ValueError, match="gating residual"):
+        L.MoELayer(atomic, {}).forward(torch.zeros(8, 256, dtype=bf), prev_logits=torch.zeros(8, 64, dtype=f32))
