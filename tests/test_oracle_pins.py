@@ -366,6 +366,31 @@ def test_atomic_layer_dense_masked_bruteforce():
     np.testing.assert_allclose(gate.sum(1), 1.0, atol=1e-14)
 
 
+def test_atomic_layer_top1_is_one_expert_with_gate_one():
+    """K = 1: the best pair of the product grid is (best row, best column), so
+    the product-key choice equals brute force over all N experts for any kept
+    half size, the gate is exactly 1, and y_t = GELU(u_e . x_t) v_e (worked
+    here with math.erf, element by element)."""
+    rows = cols = 8
+    x, wq, kr, kc = _pk_inputs(9, T=6, d=16, dq=8, rows=rows, cols=cols)
+    g = torch.Generator().manual_seed(13)
+    u = torch.randn(rows * cols, 16, generator=g) * 0.25
+    v = torch.randn(rows * cols, 16, generator=g) * 0.25
+    sr, sc = oracle.pk_scores(x, wq, kr, kc)
+    for kh in (1, 3, 8):
+        idx, gate, _ = oracle.pk_select(sr, sc, kh=kh, K=1)
+        full = sr[:, :, None] + sc[:, None, :]                    # [T, rows, cols]
+        assert idx[:, 0].tolist() == [int(np.argmax(f.reshape(-1))) for f in full]
+        assert (gate == 1.0).all()
+    y = oracle.atomic_tokens(x, u, v, np.arange(6), idx, gate)
+    xd, ud, vd = x.double().numpy(), u.double().numpy(), v.double().numpy()
+    for t in range(6):
+        e = int(idx[t, 0])
+        a = float(sum(ud[e, i] * xd[t, i] for i in range(16)))
+        act = 0.5 * a * (1.0 + math.erf(a / math.sqrt(2.0)))
+        np.testing.assert_allclose(y[t], act * vd[e], rtol=0, atol=1e-13)
+
+
 def test_full_omnimoe_layer_is_atomic_plus_shared_swiglu():
     """The full OmniMoE layer (shared dense branch beside the atomic experts)
     minus the atomic-only layer equals the shared SwiGLU branch, computed two
