@@ -417,3 +417,132 @@ def test_full_omnimoe_layer_is_atomic_plus_shared_swiglu():
     dense = ((a * torch.sigmoid(a)) * (xd @ sh["ws_up"][0].double().T)) @ sh["ws_down"][0].double().T
     np.testing.assert_allclose(y_full - y_atom, dense.numpy(), rtol=0, atol=1e-13)
     assert np.abs(dense.numpy()).max() > 0.05          # the branch is not negligible here
+
+
+# ----------------------------------------------------------- constant-expert mix
+#
+# "MoE++" summary, Approach: a constant expert mixes the token with a
+# trainable vector, y = a1 x + a2 v, with (a1, a2) a 2-way softmax of W_c x.
+# The GPU's const_mix output is checked against orc_const_mix, so that routine
+# is pinned here by itself (the layer's own constant-expert arithmetic is a
+# separate code path, pinned by test_moepp_zero_copy_const_special_cases).
+
+def _logistic(u: float) -> float:
+    """a1 of a 2-way softmax (l0, l1) = 1 / (1 + e^(l1 - l0)) for u = l0 - l1."""
+    return 1.0 / (1.0 + math.exp(-u))
+
+
+def test_const_mix_zero_weights_give_halves():
+    x = torch.randn(5, 8, generator=torch.Generator().manual_seed(0))
+    a = oracle.const_mix(x, torch.zeros(3, 2, 8))
+    assert a.shape == (5, 3, 2)
+    assert (a == 0.5).all()
+
+
+def test_const_mix_one_dim_hand_computed():
+    # d = 1: l0 = w0 x, l1 = w1 x, so a1 = logistic((w0 - w1) x) and a2 = 1 - a1
+    x = torch.tensor([[1.0], [2.0], [-4.0]])
+    wc = torch.tensor([[[0.5], [-0.25]]])            # one constant expert
+    a = oracle.const_mix(x, wc)
+    for t, xv in enumerate((1.0, 2.0, -4.0)):
+        a1 = _logistic(0.75 * xv)
+        assert abs(a[t, 0, 0] - a1) < 1e-15
+        assert abs(a[t, 0, 1] - (1.0 - a1)) < 1e-15
+    # x = 1: 1 / (1 + e^-0.75), to the digits printed by any table of e^x
+    assert abs(a[0, 0, 0] - 0.679178699175393) < 1e-14
+
+
+def test_const_mix_dominant_row_and_slot_swap():
+    x = torch.ones(2, 4)
+    wc = torch.zeros(1, 2, 4)
+    wc[0, 1, :] = 25.0                                # l1 = 100, l0 = 0
+    a = oracle.const_mix(x, wc)
+    assert a[0, 0, 0] < 1e-40 and a[0, 0, 1] == 1.0
+    a_sw = oracle.const_mix(x, wc.flip(1).contiguous())   # rows swapped -> slots swapped
+    assert a_sw[0, 0, 0] == 1.0 and a_sw[0, 0, 1] < 1e-40
+    # a mild case: the swap maps (a1, a2) to (a2, a1) exactly
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(6, 4, generator=g)
+    wc = torch.randn(1, 2, 4, generator=g)
+    a, a_sw = oracle.const_mix(x, wc), oracle.const_mix(x, wc.flip(1).contiguous())
+    np.testing.assert_allclose(a_sw[:, :, ::-1], a, atol=1e-15)
+
+
+def test_const_mix_experts_use_their_own_row_pairs():
+    # expert c reads rows (2c, 2c + 1) of the flattened [n_const * 2, d] weights:
+    # distinct pairs per expert, each checked by hand (d = 1, x = 1)
+    x = torch.ones(1, 1)
+    wc = torch.tensor([[[1.0], [0.0]],               # expert 0: l = (1, 0)
+                       [[0.0], [2.0]],               # expert 1: l = (0, 2)
+                       [[3.0], [3.0]]])              # expert 2: l = (3, 3)
+    a = oracle.const_mix(x, wc)
+    assert abs(a[0, 0, 0] - _logistic(1.0)) < 1e-15
+    assert abs(a[0, 1, 0] - _logistic(-2.0)) < 1e-15
+    assert a[0, 2, 0] == 0.5 and a[0, 2, 1] == 0.5
+
+
+def test_const_mix_matches_layer_forced_to_constant_expert():
+    # with v = 0 the layer forced onto constant expert c outputs a1 * x, so
+    # y / x recovers a1: the layer's constant-expert code and orc_const_mix
+    # agree (two separate code paths of the oracle)
+    cfg = _cfg(n_zero=1, n_copy=1, n_const=2, top_k=1)
+    inp = _rand_inputs(cfg, seed=12)
+    inp["const_vec"] = torch.zeros_like(inp["const_vec"])
+    a = oracle.const_mix(inp["x"], inp["w_const_mix"])
+    xd = inp["x"].double().numpy()
+    for c in range(2):
+        y, idx, gate, _ = _forced(cfg, inp, cfg.n_ffn + cfg.n_zero + cfg.n_copy + c)
+        assert (gate == 1.0).all()
+        np.testing.assert_allclose(y, a[:, c, 0:1] * xd, rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------------------ product-key margins
+#
+# "OmniMoE" technical summary, 2.2 Cartesian Product Router.  pk_select's
+# margins set which mis-routed tokens the GPU parity check forgives: [0] the
+# kh-th minus the (kh+1)-th row sub-score, [1] the same for the columns, [2]
+# the K-th minus the (K+1)-th candidate sum; +inf where nothing is left out.
+
+def test_pk_margins_hand_built():
+    sr = np.array([[5.0, 1.0, 3.0, 2.0]])      # rows by score: 0 (5), 2 (3) | 3 (2), 1 (1)
+    sc = np.array([[0.5, 4.0, 0.25, 3.5]])     # cols by score: 1 (4), 3 (3.5) | 0 (0.5), 2
+    idx, gate, mg = oracle.pk_select(sr, sc, kh=2, K=3)
+    # candidates (0,1) 9, (0,3) 8.5, (2,1) 7, (2,3) 6.5 -> the best 3
+    assert idx[0].tolist() == [0 * 4 + 1, 0 * 4 + 3, 2 * 4 + 1]
+    assert mg[0, 0] == 3.0 - 2.0                # kh-th row minus (kh+1)-th
+    assert mg[0, 1] == 3.5 - 0.5                # kh-th column minus (kh+1)-th
+    assert mg[0, 2] == 7.0 - 6.5                # K-th candidate minus (K+1)-th, not 8.5 - 7
+    p = np.exp(np.array([9.0, 8.5, 7.0]) - 9.0)
+    np.testing.assert_allclose(gate[0], p / p.sum(), atol=1e-15)
+
+
+def test_pk_margins_infinite_when_nothing_left_out():
+    sr = np.array([[2.0, -1.0, 0.5, 4.0]])
+    sc = np.array([[1.0, 3.0, -2.0, 0.0]])
+    _, _, mg = oracle.pk_select(sr, sc, kh=4, K=16)   # every row, column and candidate kept
+    assert np.isinf(mg[0]).all() and (mg[0] > 0).all()
+    _, _, mg = oracle.pk_select(sr, sc, kh=4, K=15)   # halves complete, one candidate out
+    assert np.isinf(mg[0, :2]).all()
+    assert mg[0, 2] == (0.5 - 2.0) - (-1.0 - 2.0)     # 15th best sum minus the 16th (the worst)
+
+
+def test_pk_margins_zero_on_ties():
+    sr = np.array([[1.0, 1.0, 0.0]])               # rows 0 and 1 tie at the kh = 1 boundary
+    sc = np.array([[2.0, 0.0, 2.0]])               # columns 0 and 2 tie likewise
+    idx, _, mg = oracle.pk_select(sr, sc, kh=1, K=1)
+    assert idx[0].tolist() == [0]                  # ties go to the lower sub-index
+    assert mg[0, 0] == 0.0 and mg[0, 1] == 0.0
+
+
+def test_pk_margins_match_sorted_scores_random():
+    rng = np.random.default_rng(11)
+    sr, sc = rng.standard_normal((7, 12)), rng.standard_normal((7, 10))
+    kh, K = 3, 5
+    idx, _, mg = oracle.pk_select(sr, sc, kh=kh, K=K)
+    for t in range(7):
+        r_sorted, c_sorted = np.sort(sr[t])[::-1], np.sort(sc[t])[::-1]
+        assert mg[t, 0] == r_sorted[kh - 1] - r_sorted[kh]
+        assert mg[t, 1] == c_sorted[kh - 1] - c_sorted[kh]
+        cand = np.sort((r_sorted[:kh][:, None] + c_sorted[:kh][None, :]).reshape(-1))[::-1]
+        assert mg[t, 2] == cand[K - 1] - cand[K]
+        assert mg[t].min() > 0
