@@ -12,9 +12,12 @@
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds it (kStaticPermuteInts * 4 bytes = 256 KiB) until the process
-// exits.  Its device address is looked up once per device with
-// cudaGetSymbolAddress, on the first call made with that device current.
+// exits.  In host code its name is only a host-side stand-in, so its device
+// address is looked up with cudaGetSymbolAddress, with the device current, on
+// the first call made in each CUDA context (a device's primary context, and
+// again after cudaDeviceReset replaces it), and passed to the kernels.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -31,21 +34,51 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_permute_scratch[kStaticPermuteInts];
 
-std::mutex g_scratch_mu;
-int32_t* g_scratch_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
-// Device address of g_permute_scratch on the current device (looked up once).
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+struct ScratchAddr {
+    CUcontext ctx;     // the context the address belongs to
+    int32_t* ptr;
+};
+
+std::mutex g_scratch_mu;
+ScratchAddr g_scratch[kMaxDevices] = {};
+
+// Device address of g_permute_scratch in the current device's current context.
+// A cached address is reused only while that context is still the current
+// one: after a device reset the array lives at a new address in a new context.
 moe_status static_scratch(int32_t** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    CtxGetCurrentFn get_ctx = ctx_get_current();
+    if (!get_ctx) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    ScratchAddr& c = g_scratch[dev];
+    if (!c.ptr || !ctx || ctx != c.ctx) {
+        void* p = nullptr;    // also makes the device's primary context current if none was
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return MOE_ERR_CUDA;
+        c.ctx = ctx;
+        c.ptr = static_cast<int32_t*>(p);
     }
-    *out = g_scratch_ptr[dev];
+    *out = c.ptr;
     return MOE_OK;
 }
 

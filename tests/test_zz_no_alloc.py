@@ -88,3 +88,21 @@ def test_static_scratch_permute_rejects_sizes_beyond_its_array():
     with pytest.raises(moe.MoEError) as e:
         moe.moe_permute_static(atomic, idx, buf, i32, i32, i32, None)
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_static_scratch_permute_at_its_size_limit():
+    # ceil(T / 256) * n_ffn = 65536 exactly: every entry of the array is used
+    # once, so an off-by-one in the size check or the kernels' indexing shows
+    dev = torch.device("cuda")
+    T, k, E, d = 256 * 256, 2, 256, 256
+    desc = moe.make_desc(T=T, d_model=d, top_k=k, n_ffn=E, hidden=256)
+    g = torch.Generator(device=dev).manual_seed(5)
+    first = torch.randint(0, E, (T,), device=dev, generator=g, dtype=torch.int32)
+    second = (first + torch.randint(1, E, (T,), device=dev, generator=g, dtype=torch.int32)) % E
+    x = torch.randn((T, d), device=dev, generator=g).to(torch.bfloat16)
+    b = moe.StageBuffers(desc, device=dev)
+    b.idx.copy_(torch.stack([first, second], dim=1))        # two distinct experts per token
+    ref = _with_workspace({"x": x}, desc, b)
+    got = _static({"x": x}, desc, b)
+    _assert_same(ref, got)
+    assert int(ref[0][-1].item()) == T * k
