@@ -9,7 +9,8 @@
 //
 // Structure (one CTA per SM, 6 warps):
 //   warp 0   TMA producer: A tile [128 x 64] + B tile [256 x 64] per stage,
-//            128-byte swizzle, 4-stage mbarrier ring (no multicast).
+//            128-byte swizzle, 4-stage mbarrier ring (no multicast); the
+//            CTA-pair forms below use 3 stages of 128-wide K instead.
 //   warp 1   TMEM allocator and MMA issuer: tcgen05.mma kind::f16,
 //            M=128 N=256 K=16, fp32 accumulators in TMEM, two accumulator
 //            buffers (512 columns) so the epilogue of one tile overlaps the
@@ -1105,7 +1106,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     // warps, which a short mainloop does not hide; measured on B200, K = 1024
     // shared-branch gate/up 72 us row-tiled vs 84 us in this form)
     // (its epilogue writes 16-byte pieces of output rows: row stride and base aligned)
-    const bool tn = MOE_GEMM_TN && p.pair && p.b_kmod == 0 && p.ldo % 8 == 0 &&
+    const bool tn = MOE_GEMM_TN && (p.pair || p.tn_any) && p.b_kmod == 0 && p.ldo % 8 == 0 &&
                     reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
                     ((EPI == EPI_SWIGLU && p.N % 128 == 0 && p.K >= MOE_TN_SWIGLU_MIN_K) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));

@@ -52,6 +52,7 @@ struct GemmProblem {
     int pk_T;             // EPI_PK_SPLIT: tokens
     int pk_dq;            // EPI_PK_SPLIT: query width
     int pair;             // 1: 256-row tiles on CTA pairs (cta_group::2); 0: 128-row tiles per CTA
+    int tn_any;           // 1: the token-column pair form may run whatever `pair` says (groups of any size)
     int b_kmod;           // > 0: B has b_kmod columns and is repeated along K (B k = k mod b_kmod)
 };
 

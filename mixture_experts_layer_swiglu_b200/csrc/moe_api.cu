@@ -409,8 +409,12 @@ moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, i
     g.rows_cap = cap;
     // 256-row tiles on CTA pairs halve the B traffic per SM; with small groups
     // their padding costs more than that saves, so they need >= 512 rows per
-    // group on average (the group sizes are only known on the device).
+    // group on average (the group sizes are only known on the device).  The
+    // token-column pair form pads a group only to a multiple of 16 rows and
+    // reads each weight block once per 256 rows of a group (a 128-row tile
+    // reads it once per 128), so it runs whatever the group sizes.
     g.pair = (long long)d->T * d->top_k >= 512ll * std::max(d->n_ffn, 1) ? 1 : 0;
+    g.tn_any = 1;
     if (phase == 1) {
         g.epi = EPI_SWIGLU;
         g.A = xs;
@@ -544,6 +548,7 @@ struct HostPipe {                       // per device: two copy streams and thei
     bool ok = false;
     cudaStream_t in = nullptr, out = nullptr;
     cudaEvent_t fork = nullptr;
+    cudaEvent_t join_in = nullptr, join_out = nullptr;   // error exits: the copy streams' last work
     cudaEvent_t in_done[kMaxHostChunks], comp_done[kMaxHostChunks], out_done[kMaxHostChunks];
 };
 
@@ -558,7 +563,9 @@ HostPipe* host_pipe()
     if (!p.ok) {
         bool good = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
                     cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) == cudaSuccess &&
-                    cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess;
+                    cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&p.join_in, cudaEventDisableTiming) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&p.join_out, cudaEventDisableTiming) == cudaSuccess;
         for (int c = 0; good && c < kMaxHostChunks; ++c)
             good = cudaEventCreateWithFlags(&p.in_done[c], cudaEventDisableTiming) == cudaSuccess &&
                    cudaEventCreateWithFlags(&p.comp_done[c], cudaEventDisableTiming) == cudaSuccess &&
@@ -753,46 +760,61 @@ moe_status moe_layer_forward_host(const moe_layer_desc* d, const moe_layer_weigh
     const size_t xrow = (size_t)d->d_model * elt(d);
     const size_t yrow = (size_t)d->d_model * (d->out_f32 ? 4 : elt(d));
     const size_t zrow = (size_t)n_router_rows(d) * 4;
-    cudaError_t e;
-#define MOE_CU(call)                                    \
-    do {                                                \
-        if ((e = (call)) != cudaSuccess) return MOE_ERR_CUDA; \
-    } while (0)
-    MOE_CU(cudaEventRecord(pp->fork, st));              // the copy streams join `stream`'s work
-    MOE_CU(cudaStreamWaitEvent(pp->in, pp->fork, 0));
-    MOE_CU(cudaStreamWaitEvent(pp->out, pp->fork, 0));
+    // Everything after the fork runs in `run`; whatever it returns, the copy
+    // streams are joined back into `stream` first, so a caller that
+    // synchronises `stream` after an error has no copy still in flight into
+    // the workspace or the host buffers.
     int launches = 0;
-    for (int c = 0; c < nch; ++c) {
-        const int t0 = c * h.dc.T;
-        const int tc = std::min(h.dc.T, d->T - t0);
-        if (tc <= 0) break;
-        const int b = c & 1;
-        if (c >= 2) MOE_CU(cudaStreamWaitEvent(pp->in, pp->comp_done[c - 2], 0));   // staging b read
-        MOE_CU(cudaMemcpyAsync(xb[b], static_cast<const char*>(x_host) + (size_t)t0 * xrow, (size_t)tc * xrow,
-                               cudaMemcpyHostToDevice, pp->in));
-        if (prev_logits_host)
-            MOE_CU(cudaMemcpyAsync(zb[b], reinterpret_cast<const char*>(prev_logits_host) + (size_t)t0 * zrow,
-                                   (size_t)tc * zrow, cudaMemcpyHostToDevice, pp->in));
-        MOE_CU(cudaEventRecord(pp->in_done[c], pp->in));
-        MOE_CU(cudaStreamWaitEvent(st, pp->in_done[c], 0));
-        if (c >= 2) MOE_CU(cudaStreamWaitEvent(st, pp->out_done[c - 2], 0));     // output b copied out
-        moe_layer_desc dcc = h.dc;
-        dcc.T = tc;
-        s = moe_layer_forward(&dcc, w, xb[b], prev_logits_host ? reinterpret_cast<const float*>(zb[b]) : nullptr,
-                              yb[b], nullptr, layer_ws, h.layer_bytes, stream);
-        launches += t_launches;
-        if (s != MOE_OK) return s;
-        MOE_CU(cudaEventRecord(pp->comp_done[c], st));
-        MOE_CU(cudaStreamWaitEvent(pp->out, pp->comp_done[c], 0));
-        MOE_CU(cudaMemcpyAsync(static_cast<char*>(y_host) + (size_t)t0 * yrow, yb[b], (size_t)tc * yrow,
-                               cudaMemcpyDeviceToHost, pp->out));
-        MOE_CU(cudaEventRecord(pp->out_done[c], pp->out));
-        if (c == nch - 1 || (c + 1) * h.dc.T >= d->T) {   // join both copy streams back into `stream`
-            MOE_CU(cudaStreamWaitEvent(st, pp->out_done[c], 0));
+    auto run = [&]() -> moe_status {
+#define MOE_CU(call)                                              \
+    do {                                                          \
+        if ((call) != cudaSuccess) return MOE_ERR_CUDA;           \
+    } while (0)
+        for (int c = 0; c < nch; ++c) {
+            const int t0 = c * h.dc.T;
+            const int tc = std::min(h.dc.T, d->T - t0);
+            if (tc <= 0) break;
+            const int b = c & 1;
+            if (c >= 2) MOE_CU(cudaStreamWaitEvent(pp->in, pp->comp_done[c - 2], 0));   // staging b read
+            MOE_CU(cudaMemcpyAsync(xb[b], static_cast<const char*>(x_host) + (size_t)t0 * xrow, (size_t)tc * xrow,
+                                   cudaMemcpyHostToDevice, pp->in));
+            if (prev_logits_host)
+                MOE_CU(cudaMemcpyAsync(zb[b], reinterpret_cast<const char*>(prev_logits_host) + (size_t)t0 * zrow,
+                                       (size_t)tc * zrow, cudaMemcpyHostToDevice, pp->in));
+            MOE_CU(cudaEventRecord(pp->in_done[c], pp->in));
             MOE_CU(cudaStreamWaitEvent(st, pp->in_done[c], 0));
+            if (c >= 2) MOE_CU(cudaStreamWaitEvent(st, pp->out_done[c - 2], 0));     // output b copied out
+            moe_layer_desc dcc = h.dc;
+            dcc.T = tc;
+            const moe_status sl = moe_layer_forward(&dcc, w, xb[b],
+                                                    prev_logits_host ? reinterpret_cast<const float*>(zb[b]) : nullptr,
+                                                    yb[b], nullptr, layer_ws, h.layer_bytes, stream);
+            launches += t_launches;
+            if (sl != MOE_OK) return sl;
+            MOE_CU(cudaEventRecord(pp->comp_done[c], st));
+            MOE_CU(cudaStreamWaitEvent(pp->out, pp->comp_done[c], 0));
+            MOE_CU(cudaMemcpyAsync(static_cast<char*>(y_host) + (size_t)t0 * yrow, yb[b], (size_t)tc * yrow,
+                                   cudaMemcpyDeviceToHost, pp->out));
+            MOE_CU(cudaEventRecord(pp->out_done[c], pp->out));
         }
-    }
+        return MOE_OK;
 #undef MOE_CU
+    };
+    if (cudaEventRecord(pp->fork, st) != cudaSuccess) return MOE_ERR_CUDA;   // the copy streams join `stream`'s work
+    if (cudaStreamWaitEvent(pp->in, pp->fork, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(pp->out, pp->fork, 0) != cudaSuccess) {
+        // `in` already waits on the fork: join it back before leaving
+        if (cudaEventRecord(pp->join_in, pp->in) == cudaSuccess) cudaStreamWaitEvent(st, pp->join_in, 0);
+        return MOE_ERR_CUDA;
+    }
+    s = run();
+    // join both copy streams back into `stream` (on success as on error)
+    const bool joined = cudaEventRecord(pp->join_in, pp->in) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, pp->join_in, 0) == cudaSuccess &&
+                        cudaEventRecord(pp->join_out, pp->out) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, pp->join_out, 0) == cudaSuccess;
+    if (s != MOE_OK) return s;
+    if (!joined) return MOE_ERR_CUDA;
     t_launches = launches;
     return MOE_OK;
 }
