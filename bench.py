@@ -55,6 +55,8 @@ def parse():
     p.add_argument("--workload", default=WORKLOAD,
                    help="tiny_f32 | mixtral | longtail | moepp | atomic | omnimoe (default: the Mixtral-shaped layer)")
     p.add_argument("--no-library-ref", action="store_true", help="skip the cuBLAS same-shape reference")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="time only --workload (skip the per-workload lines of the other layers)")
     return p.parse_args()
 
 
@@ -162,29 +164,39 @@ def oracle_sample(cfg, inp, toks) -> None:
         oracle.moe_tokens(cfg, inp, toks)
 
 
-def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0) -> dict:
+def cpu_oracle_leg(cfg, inp, n_tokens: int, seconds: float = 15.0, single_seconds: float = 5.0) -> dict:
     """The fp64 oracle as it stands on a bounded sample of the workload's
-    tokens (routing + experts of each token), on all host cores."""
+    tokens (routing + experts of each token): on all host cores (OpenMP over
+    tokens), then on one thread."""
     import numpy as np
 
     import oracle
     threads = oracle.num_threads()
 
-    def run(toks):
-        oracle_sample(cfg, inp, toks)
+    def timed(n: int, nthreads: int, budget: float):
+        """tokens/s of the oracle on n evenly spaced tokens (n <= 0: sized to
+        about `budget` seconds from a small probe)."""
+        oracle.set_num_threads(nthreads)
+        try:
+            if n <= 0:
+                t0 = time.perf_counter()
+                oracle_sample(cfg, inp, np.arange(nthreads, dtype=np.int32))
+                per_tok = (time.perf_counter() - t0) / nthreads
+                n = int(max(nthreads, min(cfg.T, budget / max(per_tok, 1e-6))))
+            toks = np.linspace(0, cfg.T - 1, n).astype(np.int32)
+            t0 = time.perf_counter()
+            oracle_sample(cfg, inp, toks)
+            return n, time.perf_counter() - t0
+        finally:
+            oracle.set_num_threads(threads)
 
-    if n_tokens <= 0:   # size the sample: time a small probe first
-        t0 = time.perf_counter()
-        run(np.arange(threads, dtype=np.int32))
-        per_tok = (time.perf_counter() - t0) / threads
-        n_tokens = int(max(threads, min(cfg.T, seconds / max(per_tok, 1e-6))))
-    toks = np.linspace(0, cfg.T - 1, n_tokens).astype(np.int32)
-    t0 = time.perf_counter()
-    run(toks)
-    el = time.perf_counter() - t0
-    return {"value": n_tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n_tokens} of the {cfg.T} tokens (evenly spaced), full routing + experts per token, "
-                      f"{el:.1f} s"}
+    n_all, el_all = timed(n_tokens, threads, seconds)
+    n_one, el_one = timed(0, 1, single_seconds)
+    return {"value": n_all / el_all, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_all} of the {cfg.T} tokens (evenly spaced), full routing + experts per token, "
+                      f"{el_all:.1f} s on {threads} threads (OpenMP over tokens)",
+            "single_thread": {"value": n_one / el_one, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n_one} of the {cfg.T} tokens (evenly spaced), {el_one:.1f} s"}}
 
 
 # ------------------------------------------------------------------- ranks
@@ -220,7 +232,10 @@ def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
     if cfg.kind == "atomic":
         dq, N = cfg.d_query, cfg.n_atomic
         return {
-            "router": ("tensor", 2.0 * T * d * dq + 2.0 * (2 * T) * (1.5 * dq) * cfg.pk_rows),
+            # q = W_q x, then each half of q (dq / 2 wide) against its sub-keys: the
+            # method's own work (the kernels' three-part bf16 split of q, which
+            # triples the score GEMM's K, is reported as router_split_flops)
+            "router": ("tensor", 2.0 * T * d * dq + 2.0 * T * (dq // 2) * (cfg.pk_rows + cfg.pk_cols)),
             "permute": ("hbm", T * k * 4 * 6 + N * 4 * 5),
             # each touched expert's u (phase A) and v (phase B) row once, x read
             # once, y written once (the token-centric phase B moves more: it
@@ -245,33 +260,50 @@ def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
     }
 
 
-def run_ours(args, rank: int, world: int, dist) -> dict | None:
-    import mixture_experts_layer_swiglu_b200 as moe
+class Peaks:
+    """Roofline denominators: MEASURED_PEAKS.json when present, else the fallback."""
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    cfg = bench_config(args)
-    w_cpu = make_weights(cfg, seed=0)
-    a_cpu = make_activations(cfg, seed=rank)           # each rank its own tokens
-    w = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in w_cpu.items()}
-    x = a_cpu["x"].to(dev)
-    zp = a_cpu["z_prev"].to(dev) if "z_prev" in a_cpu else None
-    desc = moe.desc_from(cfg)
-    desc_atomic = moe.desc_from(cfg)          # the same layer without its shared branch
-    desc_atomic.n_shared, desc_atomic.hidden_shared = 0, 0
-    ws = moe.weights_struct(w)
-    b = moe.StageBuffers(desc, device=dev)
-    cm = b.const_mix if cfg.n_const else None
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    atomic = cfg.kind == "atomic"
+    def __init__(self):
+        peaks = {}
+        pk = ROOT / "MEASURED_PEAKS.json"
+        if pk.exists():
+            peaks = json.loads(pk.read_text())
+        self.tf = peaks.get("bf16_tflops")
+        self.tf_sus = peaks.get("bf16_tflops_sustained")
+        self.tf_src = "of measured (MEASURED_PEAKS.json, burst)" if self.tf else "of fallback"
+        self.tf = self.tf or 1590.0
+        self.hbm = peaks.get("hbm_gbs")
+        self.hbm_src = "of measured (MEASURED_PEAKS.json)" if self.hbm else "of fallback"
+        self.hbm = self.hbm or 6650.0
 
-    def calls(st=stream):
-        c = [lambda: moe.moe_route(desc, ws, x, zp, None, b.idx, b.gate, cm, b.workspace, st),
+
+class Workload:
+    """One layer's weights, inputs and stage buffers on the device, and its
+    hot path as a list of C-ABI calls (route, permute, expert GEMMs, combine)."""
+
+    def __init__(self, cfg, dev, rank: int):
+        import mixture_experts_layer_swiglu_b200 as moe
+        self.moe, self.cfg, self.dev = moe, cfg, dev
+        self.w_cpu = make_weights(cfg, seed=0)
+        self.a_cpu = make_activations(cfg, seed=rank)          # each rank its own tokens
+        self.w = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.w_cpu.items()}
+        self.x = self.a_cpu["x"].to(dev)
+        self.zp = self.a_cpu["z_prev"].to(dev) if "z_prev" in self.a_cpu else None
+        self.desc = moe.desc_from(cfg)
+        self.desc_atomic = moe.desc_from(cfg)      # the same layer without its shared branch
+        self.desc_atomic.n_shared, self.desc_atomic.hidden_shared = 0, 0
+        self.ws = moe.weights_struct(self.w)
+        self.b = moe.StageBuffers(self.desc, device=dev)
+        self.atomic = cfg.kind == "atomic"
+
+    def calls(self, st):
+        moe, cfg, b, x, ws, desc = self.moe, self.cfg, self.b, self.x, self.ws, self.desc
+        cm = b.const_mix if cfg.n_const else None
+        c = [lambda: moe.moe_route(desc, ws, x, self.zp, None, b.idx, b.gate, cm, b.workspace, st),
              lambda: moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace,
                                      st)]
-        if atomic:   # the atomic step alone, then the shared dense branch's two GEMMs (if any)
-            c.append(lambda: moe.moe_grouped_ffn(desc_atomic, ws, None, b.offsets, b.token_of, x, b.gate,
+        if self.atomic:   # the atomic step alone, then the shared dense branch's two GEMMs (if any)
+            c.append(lambda: moe.moe_grouped_ffn(self.desc_atomic, ws, None, b.offsets, b.token_of, x, b.gate,
                                                  b.y_sorted, b.workspace, st))
             if cfg.n_shared:
                 c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 1, x, b.offsets, b.y_sorted, b.workspace, st))
@@ -281,12 +313,20 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
                                                        b.workspace, st))
             c.append(lambda: moe.moe_grouped_ffn_phase(desc, ws, 2, b.x_sorted, b.offsets, b.y_sorted,
                                                        b.workspace, st))
-        c.append(lambda: moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, cm, x, b.y,
-                                         st))
+        c.append(lambda: moe.moe_combine(desc, ws, b.y_sorted, b.offsets, b.row_of, b.idx, b.gate, cm, x, b.y, st))
         return c
 
-    stage_calls = calls()
-    names = stage_names(cfg)
+
+def time_workload(wl: Workload, K: int, warmup: int, dist, flush, want_graph: bool) -> dict:
+    """Warm-up, then K timed steps (L2 flushed and a GPU sleep before each,
+    outside the events; CUDA events between the stages on the launching
+    stream; SM clocks sampled meanwhile); times reduced to their maximum over
+    ranks.  Every rank takes the same collective steps."""
+    moe, dev = wl.moe, wl.dev
+    stream = torch.cuda.current_stream(dev)
+    stage_calls = wl.calls(stream)
+    names = stage_names(wl.cfg)
+    nst = len(stage_calls)
 
     def step(ev=None):
         """One pass of the hot path; events between the stages if given."""
@@ -297,17 +337,15 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
             f()
             launches += moe.moe_last_launch_count()
         if ev:
-            ev[len(stage_calls)].record(stream)
+            ev[nst].record(stream)
         return launches
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
 
-    K = args.steps
-    nst = len(stage_calls)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(K)]
     # ~0.5 ms of GPU sleep after each flush, outside the events: the host has
     # queued the whole step before the device reaches the first event, so the
@@ -329,21 +367,71 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     assert status == moe.MOE_OK, moe.status_string(status)
     per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)] for j, n in enumerate(names)}
     total_ms = sum(evs[i][0].elapsed_time(evs[i][nst]) for i in range(K))
-    off = b.offsets.cpu()
+    off = wl.b.offsets.cpu()
     R_total = int(off[-1].item())
-    R_ffn = int(off[cfg.n_ffn].item()) if not atomic else R_total
-    touched = int((off[1:] > off[:-1]).sum().item()) if atomic else 0
-
-    graph_ms = graph_step_ms(calls, stream, flush, sleep_cycles, K)
+    R_ffn = int(off[wl.cfg.n_ffn].item()) if not wl.atomic else R_total
+    touched = int((off[1:] > off[:-1]).sum().item()) if wl.atomic else 0
+    graph_ms = graph_step_ms(wl.calls, stream, flush, sleep_cycles, K) if want_graph else 0.0
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+    mean = {n: sum(v) / K for n, v in per.items()}
+    red = reduce_max_over_ranks(dist, [total_ms, graph_ms] + [mean[n] for n in names], dev)
+    return {"names": names, "ms_step": red[0] / K, "graph_ms": red[1],
+            "mean": {n: red[2 + j] for j, n in enumerate(names)}, "launches": launches,
+            "clocks": clk.summary(), "R_total": R_total, "R_ffn": R_ffn, "touched": touched}
+
+
+def kernel_table(cfg, t: dict, peaks: Peaks) -> dict:
+    """Per-stage time, share of the step and fraction of its roofline."""
+    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"])
+    kern = {}
+    for n in t["names"]:
+        ms = t["mean"][n]
+        unit, amount = work[n]
+        kern[n] = {"ms": round(ms, 4), "share": round(ms / t["ms_step"], 4)}
+        if unit == "tensor":
+            kern[n]["tflops"] = round(amount / (ms / 1e3) / 1e12, 1)
+            kern[n]["tensor_frac"] = round(kern[n]["tflops"] / peaks.tf, 4)
+        else:
+            kern[n]["gbs"] = round(amount / (ms / 1e3) / 1e9, 1)
+            kern[n]["hbm_frac"] = round(kern[n]["gbs"] / peaks.hbm, 4)
+    if cfg.kind == "atomic":   # what the three-part split of q costs on top of the method's work
+        kern["router"]["router_split_flops"] = 2.0 * cfg.T * cfg.d * cfg.d_query + \
+            2.0 * cfg.T * (3 * cfg.d_query // 2) * (cfg.pk_rows + cfg.pk_cols)
+    return kern
+
+
+def workload_line(cfg, t: dict, world: int, peaks: Peaks) -> dict:
+    """The compact per-workload entry of the JSON line's `workloads` map."""
+    return {"config": workload_config(cfg)["workload"], "dtype": cfg.dtype, "ms_per_step": round(t["ms_step"], 4),
+            "value": round(job_value(world, cfg.T, t["ms_step"]), 1), "unit": "tokens/s",
+            "graph": {"ms_per_step": round(t["graph_ms"], 4),
+                      "value": round(job_value(world, cfg.T, t["graph_ms"]), 1)},
+            "kernels": kernel_table(cfg, t, peaks), "gpu_launches": t["launches"], "clocks": t["clocks"],
+            "rows": {"grouped": t["R_total"], "ffn": t["R_ffn"], "touched_experts": t["touched"]}}
+
+
+def run_ours(args, rank: int, world: int, dist) -> dict | None:
+    import mixture_experts_layer_swiglu_b200 as moe
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    cfg = bench_config(args)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = Peaks()
+    K = args.steps
+
+    wl = Workload(cfg, dev, rank)
+    t = time_workload(wl, K, args.warmup, dist, flush, want_graph=True)
+    sleep_cycles = int(0.5e-3 * torch.cuda.get_device_properties(dev).clock_rate * 1e3)
 
     # end to end through the public call with host buffers: moe_layer_forward_host
     # copies x (and the previous layer's router logits) in and y out inside the
     # timed region, pipelined against the layer over token ranges
-    x_host = a_cpu["x"].pin_memory()
-    zp_host = a_cpu["z_prev"].contiguous().pin_memory() if "z_prev" in a_cpu else None
-    y_host = torch.empty(x_host.shape, dtype=moe.out_dtype(desc)).pin_memory()
-    layer = moe.MoELayer(desc, w)
+    x_host = wl.a_cpu["x"].pin_memory()
+    zp_host = wl.a_cpu["z_prev"].contiguous().pin_memory() if "z_prev" in wl.a_cpu else None
+    y_host = torch.empty(x_host.shape, dtype=moe.out_dtype(wl.desc)).pin_memory()
+    layer = moe.MoELayer(wl.desc, wl.w)
     for _ in range(2):
         layer.forward_host(x_host, prev_logits=zp_host, y_host=y_host, stream=stream, device=dev)
     torch.cuda.synchronize()
@@ -360,55 +448,46 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         e2e_ms += e0.elapsed_time(e1)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
+    e2e_ms = reduce_max_over_ranks(dist, [e2e_ms / KE], dev)[0]
+    del layer
 
     cublas = None
-    if not atomic and cfg.dtype == "bf16" and rank == 0 and not args.no_library_ref:
-        cublas = library_reference(cfg, R_total, dev)
+    if wl.atomic is False and cfg.dtype == "bf16" and rank == 0 and not args.no_library_ref:
+        cublas = library_reference(cfg, t["R_total"], dev)
 
-    mean = {n: sum(v) / K for n, v in per.items()}
-    red = reduce_max_over_ranks(dist, [total_ms, e2e_ms / KE, graph_ms] + [mean[n] for n in names], dev)
-    res = {"total_ms": red[0], "e2e_ms": red[1], "graph_ms": red[2],
-           "mean": {n: red[3 + j] for j, n in enumerate(names)}}
+    # every other workload, timed the same way (each rank runs them all, so the
+    # collective steps stay in step)
+    others = {}
+    if not args.no_workloads and not args.tokens and not args.experts:
+        from moe_workloads.configs import ORDER
+        for name in ORDER:
+            if name == cfg.name:
+                continue
+            c2 = get_config(name)
+            w2 = Workload(c2, dev, rank)
+            t2 = time_workload(w2, K, args.warmup, dist, flush, want_graph=True)
+            others[name] = workload_line(c2, t2, world, peaks)
+            del w2
+            torch.cuda.empty_cache()
     if rank != 0:
         return None
 
-    peaks = {}
-    pk = ROOT / "MEASURED_PEAKS.json"
-    if pk.exists():
-        peaks = json.loads(pk.read_text())
-    peak_tf = peaks.get("bf16_tflops")
-    peak_tf_sus = peaks.get("bf16_tflops_sustained")
-    peak_src = "of measured (MEASURED_PEAKS.json, burst)" if peak_tf else "of fallback"
-    if not peak_tf:
-        peak_tf = 1590.0
-    hbm = peaks.get("hbm_gbs")
-    hbm_src = "of measured (MEASURED_PEAKS.json)" if hbm else "of fallback"
-    hbm = hbm or 6650.0
-    work = work_model(cfg, R_total, R_ffn, touched)
-    ms_step = res["total_ms"] / K
+    kern = kernel_table(cfg, t, peaks)
+    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"])
+    ms_step = t["ms_step"]
     value = job_value(world, cfg.T, ms_step)
-    kern = {}
-    for n in names:
-        ms = res["mean"][n]
-        unit, amount = work[n]
-        kern[n] = {"ms": round(ms, 4), "share": round(ms / ms_step, 4)}
-        if unit == "tensor":
-            kern[n]["tflops"] = round(amount / (ms / 1e3) / 1e12, 1)
-            kern[n]["tensor_frac"] = round(kern[n]["tflops"] / peak_tf, 4)
-        else:
-            kern[n]["gbs"] = round(amount / (ms / 1e3) / 1e9, 1)
-            kern[n]["hbm_frac"] = round(kern[n]["gbs"] / hbm, 4)
-    dom = max(names, key=lambda n: res["mean"][n])
+    names = t["names"]
+    dom = max(names, key=lambda n: t["mean"][n])
     unit, amount = work[dom]
-    dom_s = res["mean"][dom] / 1e3
+    dom_s = t["mean"][dom] / 1e3
     if unit == "tensor":
-        roof = {"bound": "tensor", "kernel": dom, "achieved": round(amount / dom_s / 1e12, 1), "peak": peak_tf,
-                "unit": "TFLOP/s", "peak_source": peak_src, "flops_per_launch": amount}
-        if peak_tf_sus:
-            roof["frac_of_sustained"] = round(roof["achieved"] / peak_tf_sus, 4)
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(amount / dom_s / 1e12, 1), "peak": peaks.tf,
+                "unit": "TFLOP/s", "peak_source": peaks.tf_src, "flops_per_launch": amount}
+        if peaks.tf_sus:
+            roof["frac_of_sustained"] = round(roof["achieved"] / peaks.tf_sus, 4)
     else:
-        roof = {"bound": "hbm", "kernel": dom, "achieved": round(amount / dom_s / 1e9, 1), "peak": hbm,
-                "unit": "GB/s", "peak_source": hbm_src, "bytes_per_launch": amount}
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(amount / dom_s / 1e9, 1), "peak": peaks.hbm,
+                "unit": "GB/s", "peak_source": peaks.hbm_src, "bytes_per_launch": amount}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["traffic"] = _ncu_traffic(dom, cfg.name)
     h2d = x_host.numel() * x_host.element_size() + (zp_host.numel() * 4 if zp_host is not None else 0)
@@ -422,21 +501,24 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         "roofline": roof,
         "kernels": kern,
         "step_tflops": round(flops / (ms_step / 1e3) / 1e12, 1),
-        "rows": {"grouped": R_total, "ffn": R_ffn, "touched_experts": touched},
-        "e2e": {"value": round(job_value(world, cfg.T, res["e2e_ms"]), 1), "unit": "tokens/s",
+        "rows": {"grouped": t["R_total"], "ffn": t["R_ffn"], "touched_experts": t["touched"]},
+        "e2e": {"value": round(job_value(world, cfg.T, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "moe_layer_forward_host: x (and previous router logits) from pinned host, y to pinned "
                         "host, copies pipelined against the layer over token ranges"},
-        "graph": {"ms_per_step": round(res["graph_ms"], 4),
-                  "value": round(job_value(world, cfg.T, res["graph_ms"]), 1), "unit": "tokens/s",
+        "graph": {"ms_per_step": round(t["graph_ms"], 4),
+                  "value": round(job_value(world, cfg.T, t["graph_ms"]), 1), "unit": "tokens/s",
                   "how": "the same step captured once in a CUDA graph and replayed; L2 flushed before each replay"},
-        "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "gpu_launches": t["launches"],
+        "clocks": t["clocks"],
     }
     if cublas:
         out["library_reference"] = cublas
+    if others:
+        out["workloads"] = others
     if world == 1 and not args.no_cpu_baseline:
-        w_cpu.update(a_cpu)
+        w_cpu = dict(wl.w_cpu)
+        w_cpu.update(wl.a_cpu)
         out["cpu_baseline"] = cpu_oracle_leg(cfg, w_cpu, args.oracle_tokens)
     return out
 
