@@ -284,8 +284,9 @@ MOE_API moe_status moe_layer_forward_host(const moe_layer_desc* desc, const moe_
  * Limit: ceil(T / 256) * n_ffn <= 65536 (e.g. T <= 65536 with 256 experts,
  *   T <= 2,097,152 with 8 experts); beyond it, or for the atomic kind, the
  *   call returns MOE_ERR_UNSUPPORTED and enqueues nothing.
- * The first call on a device looks up the array's device address (with that
- *   device current) and may fail with MOE_ERR_CUDA; make that first call
+ * The first call on a device (and the first after a cudaDeviceReset, which
+ *   gives the device a new context) looks up the array's device address with
+ *   that device current and may fail with MOE_ERR_CUDA; make that first call
  *   before any stream capture.
  * Every call on a device shares the one array and it keeps the last call's
  *   contents (nothing needs clearing: each call overwrites every entry it
@@ -295,6 +296,40 @@ MOE_API moe_status moe_layer_forward_host(const moe_layer_desc* desc, const moe_
 MOE_API moe_status moe_permute_static(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x,
                                       int32_t* expert_offsets, int32_t* row_of, int32_t* token_of,
                                       void* x_sorted, moe_stream_t stream);
+
+/*
+ * Expert parallelism (host functions; no device work).  With the routed
+ * experts split over G ranks, each rank routes, permutes and combines its own
+ * tokens, and the rows of expert e are computed by the rank that owns e.
+ * Ownership follows the grouping of tasks by contiguous ranges of expert ids
+ * ("OmniMoE" technical summary, 2.2 Expert-Centric Scheduling): rank r owns
+ * experts [r*E/G, (r+1)*E/G) (integer division; a rank may own none when
+ * E < G).  A rank's rows of expert e are rows [off[e], off[e+1]) of its
+ * x_sorted (moe_permute's expert_offsets); it sends that block to the owner,
+ * which lays the blocks it receives out expert-major with the source rank
+ * inside, so its owned experts are ordinary groups of the grouped GEMM; the
+ * results go back block by block to the rows they came from, and the combine
+ * is the single-rank one.  The exchange itself (NCCL send/receive of the
+ * blocks, in increasing expert order between every pair of ranks) is the
+ * caller's.  The pages describe expert parallelism only as prior art for
+ * other hardware; the split and layout here are this library's.
+ *
+ * moe_ep_expert_range: the experts [*lo, *hi) that `rank` owns.
+ * moe_ep_owner: the rank that owns `expert` (-1 for invalid arguments).
+ * moe_ep_plan: counts [G, E] host int32, counts[q*E + e] = rows of rank q
+ *   routed to expert e (the differences of every rank's expert_offsets).
+ *   For this rank's owned experts i = e - lo (n_own = hi - lo):
+ *   recv_offsets[i*G + q], recv_counts[i*G + q] (host int32, n_own*G each):
+ *   where the block of (expert e, source rank q) lands in the receive buffer
+ *   and its rows; local_offsets [n_own + 1] (host int32): the group offsets
+ *   of the owned experts in the receive buffer.  Returns the number of rows
+ *   received (>= 0), or -1 for invalid arguments, a negative count or a total
+ *   of 2^31 rows or more.  All buffers are the caller's.
+ */
+MOE_API moe_status moe_ep_expert_range(int G, int E, int rank, int32_t* lo, int32_t* hi);
+MOE_API int32_t moe_ep_owner(int G, int E, int expert);
+MOE_API int64_t moe_ep_plan(const int32_t* counts, int G, int E, int rank, int32_t* recv_offsets,
+                            int32_t* recv_counts, int32_t* local_offsets);
 
 /*
  * Self-test of the kernels' bounded waits (no counterpart on the pages): a

@@ -24,7 +24,8 @@ EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_lay
             "moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
             "moe_layer_forward", "moe_get_device_status", "moe_status_string",
             "moe_last_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
-            "moe_layer_host_workspace_size", "moe_layer_forward_host")
+            "moe_layer_host_workspace_size", "moe_layer_forward_host", "moe_ep_expert_range", "moe_ep_owner",
+            "moe_ep_plan")
 
 
 class MoEError(RuntimeError):
@@ -78,6 +79,12 @@ def load(path: Path | str | None = None):
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_launch_count.restype = I32
+    L.moe_ep_expert_range.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P(I32), P(I32)]
+    L.moe_ep_expert_range.restype = ctypes.c_int
+    L.moe_ep_owner.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.moe_ep_owner.restype = I32
+    L.moe_ep_plan.argtypes = [VP, ctypes.c_int, ctypes.c_int, ctypes.c_int, VP, VP, VP]
+    L.moe_ep_plan.restype = I64
     for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
                  "moe_layer_forward", "moe_get_device_status", "moe_permute_static",
                  "moe_selftest_wait_timeout", "moe_layer_forward_host"):
@@ -239,3 +246,38 @@ def moe_selftest_wait_timeout(limit_ns: int, waited_ok, stream=None) -> None:
 
 def moe_last_launch_count() -> int:
     return int(load().moe_last_launch_count())
+
+
+# ------------------------------------------------------ expert parallelism (host)
+
+def moe_ep_expert_range(G: int, E: int, rank: int) -> tuple[int, int]:
+    lo, hi = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("moe_ep_expert_range", load().moe_ep_expert_range(int(G), int(E), int(rank), ctypes.byref(lo),
+                                                              ctypes.byref(hi)))
+    return int(lo.value), int(hi.value)
+
+
+def moe_ep_owner(G: int, E: int, expert: int) -> int:
+    r = int(load().moe_ep_owner(int(G), int(E), int(expert)))
+    if r < 0:
+        raise MoEError("moe_ep_owner", MOE_ERR_INVALID_ARG)
+    return r
+
+
+def moe_ep_plan(counts, rank: int):
+    """counts: host int32 tensor [G, E].  Returns (recv_offsets [n_own, G],
+    recv_counts [n_own, G], local_offsets [n_own + 1], rows received)."""
+    if counts.is_cuda or counts.dtype != torch.int32 or counts.dim() != 2:
+        raise ValueError("moe_ep_plan takes a host int32 [G, E] tensor")
+    counts = counts.contiguous()
+    G, E = counts.shape
+    lo, hi = moe_ep_expert_range(G, E, rank)
+    n_own = hi - lo
+    ro = torch.zeros((max(n_own, 1), G), dtype=torch.int32)
+    rc = torch.zeros((max(n_own, 1), G), dtype=torch.int32)
+    lo_off = torch.zeros((n_own + 1,), dtype=torch.int32)
+    total = int(load().moe_ep_plan(counts.data_ptr(), G, E, int(rank), ro.data_ptr(), rc.data_ptr(),
+                                   lo_off.data_ptr()))
+    if total < 0:
+        raise MoEError("moe_ep_plan", MOE_ERR_INVALID_ARG)
+    return ro[:n_own], rc[:n_own], lo_off, total
