@@ -168,7 +168,9 @@ MOE_API moe_status moe_route(const moe_layer_desc* desc, const moe_layer_weights
  * token_of [row capacity]: SwiGLU: token of each row; atomic: flat slot id
  *   t*top_k + j of each task.
  * x_sorted [row capacity, d_model]: SwiGLU only, x_sorted[r] = x[token_of[r]];
- *   NULL for the atomic kind.  Rows past expert_offsets[groups] are untouched.
+ *   NULL for the atomic kind, and may be NULL for the SwiGLU kind when the
+ *   fused expert step (moe_fused_ffn_combine) gathers the rows itself.  Rows
+ *   past expert_offsets[groups] are untouched.
  * An id outside [0, n_ffn + n_zero + n_copy + n_const) (or the atomic grid)
  * sets MOE_ERR_DEVICE_BOUNDS in the device status and is skipped.
  */
@@ -232,6 +234,44 @@ MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weigh
                        const void* y_sorted, const int32_t* expert_offsets,
                        const int32_t* row_of, const int32_t* topk_idx, const float* topk_gate,
                        const float* const_mix, const void* x, void* y, moe_stream_t stream);
+
+/*
+ * The expert step with the permutation and the combine fused into the two
+ * grouped GEMMs ("OmniMoE" technical summary, 2.2 Expert-Centric
+ * Scheduling: the expert weights of a block are loaded once for the tokens of
+ * the expert's group; 2.1 Dynamic Expert Assembly: the routed outputs are
+ * assembled per token).  Same result as moe_grouped_ffn + moe_combine, with no
+ * x_sorted and no y_sorted in memory:
+ *   phase 1: h[r] = silu(W_gate[e] x[token_of[r]]) * (W_up[e] x[token_of[r]])
+ *            for the rows r of expert e's group; the token rows are gathered
+ *            by the GEMM's own loads (tile::gather4, no x_sorted); the same
+ *            kernel zeroes the fp32 accumulator rows of the groups' tokens;
+ *   phase 2: acc[t] += g(t, e) * (W_down[e] h[r]) for t = token_of[r], by
+ *            the GEMM's epilogue with vector atomics.  A token has at most
+ *            two FFN slots, and two fp32 additions into zero give the same sum
+ *            in either order, so the result does not depend on timing;
+ *   phase 3: y_t = acc[t] (if the token has an FFN slot) + the zero-
+ *            computation slots' terms in slot order (as in moe_combine),
+ *            rounded once to the output type.
+ *   phase 0: the three in order.
+ * Layers it applies to (else MOE_ERR_UNSUPPORTED, nothing enqueued): SwiGLU
+ * kind, bf16, n_ffn > 0, no shared experts, top_k <= 2, d_model a multiple
+ * of 256, hidden a multiple of 128.  moe_layer_forward uses this step for
+ * every such layer.
+ * Arguments as moe_route / moe_permute produce them (expert_offsets [n_ffn +
+ * 1], row_of [T, top_k], token_of [T * top_k]); x [T, d_model]; y [T,
+ * d_model] (bf16, or fp32 if desc->out_f32).  workspace: at least
+ * moe_fused_workspace_size(desc) bytes (h, then the accumulator at byte
+ * align256(cap * hidden * 2)); phases 1-3 called one by one must share it.
+ * moe_fused_workspace_size returns -1 for a descriptor the step does not
+ * apply to.
+ */
+MOE_API int64_t moe_fused_workspace_size(const moe_layer_desc* desc);
+MOE_API moe_status moe_fused_ffn_combine(const moe_layer_desc* desc, const moe_layer_weights* w, int phase,
+                                         const void* x, const int32_t* topk_idx, const float* topk_gate,
+                                         const float* const_mix, const int32_t* expert_offsets,
+                                         const int32_t* row_of, const int32_t* token_of, void* y,
+                                         void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * The whole layer: moe_route, moe_permute, moe_grouped_ffn and moe_combine

@@ -12,7 +12,7 @@ from ._abi import (  # noqa: F401
     MoEError, MoELayerDesc, MoELayerWeights, moe_combine, moe_get_device_status, moe_grouped_ffn,
     moe_grouped_ffn_phase, moe_last_launch_count, moe_layer_forward, moe_layer_forward_host,
     moe_layer_host_workspace_size, moe_layer_workspace_size, moe_num_groups, moe_permute, moe_permute_static,
-    moe_ep_expert_range, moe_ep_owner, moe_ep_plan, moe_route, moe_row_capacity, moe_selftest_wait_timeout,
+    moe_ep_expert_range, moe_ep_owner, moe_ep_plan, moe_fused_ffn_combine, moe_fused_workspace_size, moe_route, moe_row_capacity, moe_selftest_wait_timeout,
     moe_workspace_size, status_string, weights_struct)
 from .layer import (MoELayer, StageBuffers, desc_from, make_desc, out_dtype, run_stages,  # noqa: F401
                     torch_dtype)

@@ -25,7 +25,7 @@ EXPORTED = ("moe_num_groups", "moe_row_capacity", "moe_workspace_size", "moe_lay
             "moe_layer_forward", "moe_get_device_status", "moe_status_string",
             "moe_last_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
             "moe_layer_host_workspace_size", "moe_layer_forward_host", "moe_ep_expert_range", "moe_ep_owner",
-            "moe_ep_plan")
+            "moe_ep_plan", "moe_fused_workspace_size", "moe_fused_ffn_combine")
 
 
 class MoEError(RuntimeError):
@@ -72,6 +72,9 @@ def load(path: Path | str | None = None):
     L.moe_grouped_ffn_phase.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, SZ, VP]
     L.moe_combine.argtypes = [D, W, VP, VP, VP, VP, VP, VP, VP, VP, VP]
     L.moe_layer_forward.argtypes = [D, W, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_fused_workspace_size.argtypes = [D]
+    L.moe_fused_workspace_size.restype = I64
+    L.moe_fused_ffn_combine.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_layer_host_workspace_size.argtypes = [D, ctypes.c_int]
     L.moe_layer_host_workspace_size.restype = I64
     L.moe_layer_forward_host.argtypes = [D, W, VP, VP, VP, ctypes.c_int, VP, SZ, VP]
@@ -86,7 +89,7 @@ def load(path: Path | str | None = None):
     L.moe_ep_plan.argtypes = [VP, ctypes.c_int, ctypes.c_int, ctypes.c_int, VP, VP, VP]
     L.moe_ep_plan.restype = I64
     for name in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_phase", "moe_combine",
-                 "moe_layer_forward", "moe_get_device_status", "moe_permute_static",
+                 "moe_layer_forward", "moe_get_device_status", "moe_permute_static", "moe_fused_ffn_combine",
                  "moe_selftest_wait_timeout", "moe_layer_forward_host"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -217,6 +220,20 @@ def moe_layer_forward(desc, weights, x, prev_logits, y, logits_out, workspace, s
     _check("moe_layer_forward", load().moe_layer_forward(ctypes.byref(desc), ctypes.byref(ws), _p(x),
                                                          _p(prev_logits), _p(y), _p(logits_out),
                                                          _p(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def moe_fused_workspace_size(desc: MoELayerDesc) -> int:
+    """Workspace bytes of moe_fused_ffn_combine; -1 if the layer does not qualify."""
+    return int(load().moe_fused_workspace_size(ctypes.byref(desc)))
+
+
+def moe_fused_ffn_combine(desc, weights, phase, x, topk_idx, topk_gate, const_mix, expert_offsets, row_of,
+                          token_of, y, workspace, stream=None) -> None:
+    ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
+    _check("moe_fused_ffn_combine",
+           load().moe_fused_ffn_combine(ctypes.byref(desc), ctypes.byref(ws), int(phase), _p(x), _p(topk_idx),
+                                        _p(topk_gate), _p(const_mix), _p(expert_offsets), _p(row_of), _p(token_of),
+                                        _p(y), _p(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def moe_layer_host_workspace_size(desc: MoELayerDesc, chunks: int = 0) -> int:

@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
     const int n_ids = const0 + a.n_const;
     __shared__ int s_e[TPB][CMB_MAXK], s_r[TPB][CMB_MAXK];
     __shared__ float s_g[TPB][CMB_MAXK], s_a1[TPB][CMB_MAXK], s_a2[TPB][CMB_MAXK];
+    __shared__ int s_ffn[TPB];                       // the token has an FFN slot (accumulator row written)
     for (long long base = (long long)blockIdx.x * TPB; base < a.T; base += (long long)gridDim.x * TPB) {
         const long long t = base + tib;
         const bool live = t < a.T;
@@ -133,6 +134,11 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
             s_a1[tib][lane] = a1;
             s_a2[tib][lane] = a2;
         }
+        if (live && part == 0) {
+            const bool f = lane < a.k && a.idx[t * a.k + lane] >= 0 && a.idx[t * a.k + lane] < zero0;
+            const unsigned m = __ballot_sync(FULL, f);
+            if (lane == 0) s_ffn[tib] = m != 0u;
+        }
         __syncthreads();
         if (live) {
             // two chunks per lane and step: their row loads are independent
@@ -143,6 +149,10 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
+                if (a.acc_rows && s_ffn[tib]) {      // the FFN slots' sum, formed by the down GEMM
+                    load8<float>(a.ys, t * vecs + i, acc[0]);
+                    if (two) load8<float>(a.ys, t * vecs + i + 32, acc[1]);
+                }
                 for (int s = 0; s < a.n_shared; ++s) {
                     const long long r = (long long)a.offsets[a.n_ffn + s] + t;
                     if (r < a.rows_cap) {
@@ -162,6 +172,7 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
                     const float g = s_g[tib][j];
                     if (e < 0) continue;
                     if (e < zero0) {
+                        if (a.acc_rows) continue;         // already in the accumulator row
                         const long long rb = (long long)s_r[tib][j] * vecs;
                         float w[2][V];
                         load8<float>(a.ys, rb + i, w[0]);

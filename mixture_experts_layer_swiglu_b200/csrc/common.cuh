@@ -337,6 +337,28 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four rows r0..r3 of a 2-D tensor (each one box of the map: 64 elements of
+// K from column c0), gathered into consecutive 128-byte rows of this CTA's
+// shared memory; completion counted on the leader CTA's mbarrier (shared::
+// cluster address).  The map's box is one row high.  No multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int c0,
+                                                 int r0, int r1, int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1),
+          "r"(r2), "r"(r3)
+        : "memory");
+}
+
+// acc[0..3] += v[0..3] with one vector atomic (relaxed, device scope).
+__device__ __forceinline__ void red_add_v4(float* acc, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols)
 {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"

@@ -69,6 +69,14 @@ struct DevArgs {
     long long ldo;
     long long rows_cap;
     int pk_T, pk_dq;
+    // fused permutation / combine (token-column form only)
+    const int32_t* rows;        // row r of the grouped operand is token rows[r] (token_of)
+    int rows_T;                 // tokens (bound of rows[r])
+    float* acc;                 // [rows_T, acc_d] fp32 combine accumulator
+    int acc_d;
+    const int32_t* idx;         // [rows_T, k] routing (gate lookup of the scatter-add epilogue)
+    const float* gate;          // [rows_T, k]
+    int k;
 };
 
 struct TileInfo {
@@ -813,13 +821,23 @@ __device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body)
     }
 }
 
-template <int EPI>
+// MODE: TN_PLAIN, TN_GATHER (SwiGLU only: the token rows of the B operand are
+// gathered from x by `rows` with tile::gather4 loads, and each tile zeroes its
+// share of its tokens' fp32 combine accumulator rows), TN_SCATTER_ADD (fp32
+// only: each output row is scaled by its token's gate for this group's expert
+// and added into the accumulator row of its token with vector atomics).
+enum TnMode { TN_PLAIN = 0, TN_GATHER = 1, TN_SCATTER_ADD = 2 };
+
+template <int EPI, int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW0,
                        const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                        const __grid_constant__ CUtensorMap tmW3, const DevArgs a)
 {
     static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "token-column form: SwiGLU or fp32 epilogue");
+    static_assert(MODE == TN_PLAIN || (MODE == TN_GATHER && EPI == EPI_SWIGLU) ||
+                  (MODE == TN_SCATTER_ADD && EPI == EPI_F32), "fused modes: gather with SwiGLU, scatter-add with fp32");
+    constexpr bool GATHER = MODE == TN_GATHER;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -867,8 +885,10 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (GATHER || lane == 0) {
             // -------------------------------------------- TMA producer (both CTAs)
+            // (gather: all 32 lanes; lane L loads rows 4L .. 4L + 3 of the CTA's
+            // half of the token tile, lane 0 also the weights and the barriers)
             int s = 0;
             uint32_t ph = 0;
             bool bad = false;
@@ -881,22 +901,48 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                                                      : gb * a.N + ti.m * 256 + (int)rank * 128;
                 const CUtensorMap* mw = first ? &tmW0 : &tmW2;
                 const CUtensorMap* mu = first ? &tmW1 : &tmW3;
-                const int xrow = ti.tok0 + (int)rank * (ti.nt >> 1);
-                if (*abort_flag) { bad = true; break; }
+                const int half_n = ti.nt >> 1;
+                const int xrow = ti.tok0 + (int)rank * half_n;
+                int xr[4] = {0, 0, 0, 0};
+                if constexpr (GATHER) {
+                    // token of each of this lane's rows; columns past the tile's
+                    // valid rows repeat its last row (their results are dropped)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int lrow = min((int)rank * half_n + 4 * lane + j, ti.valid - 1);
+                        int t = a.rows[ti.tok0 + lrow];
+                        if (t < 0 || t >= a.rows_T) { set_status(MOE_ERR_DEVICE_BOUNDS); t = 0; }
+                        xr[j] = t;
+                    }
+                }
+                const bool stop = GATHER ? __shfl_sync(0xffffffffu, *abort_flag, 0) != 0 : *abort_flag != 0;
+                if (stop) { bad = true; break; }
                 for (int kb = 0; kb < pnk; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; bad = true; break; }
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
+                    bool ok = lane != 0 || mbar_wait(&empty[s], ph ^ 1);
+                    if constexpr (GATHER) ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) { *abort_flag = 1; bad = true; break; }
+                    // both CTAs' bytes of this stage: A, then B (gathered: half_n rows of 128 B per box)
+                    if (lane == 0 && leader)
+                        mbar_arrive_expect_tx(&full[s], GATHER ? 2 * P_KH * (P_HALF + half_n * 128) : 2 * P_STAGE_BYTES);
 #pragma unroll
                     for (int h = 0; h < P_KH; ++h) {
                         const int k0 = (kb * P_KH + h) * BK;      // past K: zero fill
                         uint8_t* da = sA + s * P_TILE_A + h * P_HALF;
-                        if (EPI == EPI_SWIGLU) {   // 64 gate rows, then the 64 up rows of the same units
-                            tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
-                            tma_load_2d_pair(da + P_HALF / 2, mu, full_leader + 8 * s, k0, wrow);
-                        } else {
-                            tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
+                        uint8_t* db = sB + s * P_TILE_B + h * P_HALF;
+                        if (lane == 0) {
+                            if (EPI == EPI_SWIGLU) {   // 64 gate rows, then the 64 up rows of the same units
+                                tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
+                                tma_load_2d_pair(da + P_HALF / 2, mu, full_leader + 8 * s, k0, wrow);
+                            } else {
+                                tma_load_2d_pair(da, mw, full_leader + 8 * s, k0, wrow);
+                            }
+                            if (!GATHER) tma_load_2d_pair(db, &tmX, full_leader + 8 * s, k0, xrow);
                         }
-                        tma_load_2d_pair(sB + s * P_TILE_B + h * P_HALF, &tmX, full_leader + 8 * s, k0, xrow);
+                        if constexpr (GATHER) {
+                            if (4 * lane < half_n)
+                                tma_gather4_pair(db + 4 * lane * 128, &tmX, full_leader + 8 * s, k0, xr[0], xr[1], xr[2],
+                                                 xr[3]);
+                        }
                     }
                     if (++s == P_STAGES) { s = 0; ph ^= 1; }
                 }
@@ -969,14 +1015,42 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
 #pragma unroll
                     for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = __uint_as_float(v[i]);
                     __syncwarp();
+                    if constexpr (MODE == TN_SCATTER_ADD) {
+                        // lane l: the token of row ch * 32 + l and its gate for this group's expert
+                        int tl = -1;
+                        float gl = 0.f;
+                        const int cl = ch * 32 + lane;
+                        if (cl < ti.valid) {
+                            const int t = a.rows[ti.tok0 + cl];
+                            if (t < 0 || t >= a.rows_T) {
+                                set_status(MOE_ERR_DEVICE_BOUNDS);
+                            } else {
+                                for (int j = 0; j < a.k; ++j)
+                                    if (a.idx[(long long)t * a.k + j] == ti.g) { tl = t; gl = a.gate[(long long)t * a.k + j]; }
+                                if (tl < 0) set_status(MOE_ERR_DEVICE_BOUNDS);
+                            }
+                        }
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const int idx = r * 32 + lane, row = idx >> 3, piece = idx & 7;
-                        const int c = ch * 32 + row;
-                        const long long grow = (long long)ti.tok0 + c;
-                        if (c < ti.valid && grow < a.rows_cap)
-                            *reinterpret_cast<float4*>(out + grow * a.ldo + f0 + piece * 4) =
-                                *reinterpret_cast<const float4*>(stg + row * 32 + piece * 4);
+                        for (int r = 0; r < 8; ++r) {
+                            const int idx = r * 32 + lane, row = idx >> 3, piece = idx & 7;
+                            const int t = __shfl_sync(0xffffffffu, tl, row);
+                            const float gg = __shfl_sync(0xffffffffu, gl, row);
+                            if (t >= 0) {
+                                const float4 w = *reinterpret_cast<const float4*>(stg + row * 32 + piece * 4);
+                                red_add_v4(a.acc + (long long)t * a.acc_d + f0 + piece * 4, gg * w.x, gg * w.y,
+                                           gg * w.z, gg * w.w);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const int idx = r * 32 + lane, row = idx >> 3, piece = idx & 7;
+                            const int c = ch * 32 + row;
+                            const long long grow = (long long)ti.tok0 + c;
+                            if (c < ti.valid && grow < a.rows_cap)
+                                *reinterpret_cast<float4*>(out + grow * a.ldo + f0 + piece * 4) =
+                                    *reinterpret_cast<const float4*>(stg + row * 32 + piece * 4);
+                        }
                     }
                 });
             } else {
@@ -1019,6 +1093,21 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                         finish(g, u, ch * 32 + 16);
                     }
                 });
+                if constexpr (GATHER) {
+                    // this tile's share of zeroing its tokens' combine accumulator rows:
+                    // 16-byte units [m U / ntm, (m + 1) U / ntm) of each row, so the
+                    // ntm weight blocks of a token tile clear its rows between them
+                    const int U = a.acc_d / 4;
+                    const int u0 = (int)((long long)ti.m * U / ntm), u1 = (int)((long long)(ti.m + 1) * U / ntm);
+                    const int c = (int)rank * 128 + (warp - 2) * 32 + lane;
+                    if (c < ti.valid) {
+                        const int t = a.rows[ti.tok0 + c];
+                        if (t >= 0 && t < a.rows_T) {
+                            float4* row = reinterpret_cast<float4*>(a.acc + (long long)t * a.acc_d);
+                            for (int u = u0; u < u1; ++u) row[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -1106,12 +1195,20 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     // warps, which a short mainloop does not hide; measured on B200, K = 1024
     // shared-branch gate/up 72 us row-tiled vs 84 us in this form)
     // (its epilogue writes 16-byte pieces of output rows: row stride and base aligned)
-    const bool tn = MOE_GEMM_TN && (p.pair || p.tn_any) && p.b_kmod == 0 && p.ldo % 8 == 0 &&
+    // (the fused forms exist only in the token-column form, for any K)
+    const bool tn = MOE_GEMM_TN && (p.pair || p.tn_any || p.fuse) && p.b_kmod == 0 && p.ldo % 8 == 0 &&
                     reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
-                    ((EPI == EPI_SWIGLU && p.N % 128 == 0 && p.K >= MOE_TN_SWIGLU_MIN_K) ||
+                    ((EPI == EPI_SWIGLU && p.N % 128 == 0 && (p.K >= MOE_TN_SWIGLU_MIN_K || p.fuse)) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));
+    if (p.fuse && (!tn || (p.fuse == 1) != (EPI == EPI_SWIGLU) || (p.fuse == 2) != (EPI == EPI_F32) ||
+                   !p.rows || !p.acc || p.acc_d % 256 != 0 || p.rows_T <= 0 ||
+                   (p.fuse == 1 && p.K % (BK * P_KH) != 0) || (p.fuse == 2 && (!p.idx || !p.gate || p.k <= 0)) ||
+                   reinterpret_cast<uintptr_t>(p.acc) % 16 != 0))
+        return MOE_ERR_UNSUPPORTED;
     const int wbox = (tn && EPI == EPI_SWIGLU) ? 64 : 128;
-    if (!make_map(&mA, p.A, p.a_rows, p.K) || !make_map(&m0, p.B0, p.b01_rows, kb, wbox) ||
+    // gathered rows: x itself, one-row boxes (tile::gather4 loads)
+    const bool mapA_ok = p.fuse == 1 ? make_map(&mA, p.A, p.rows_T, p.K, 1) : make_map(&mA, p.A, p.a_rows, p.K);
+    if (!mapA_ok || !make_map(&m0, p.B0, p.b01_rows, kb, wbox) ||
         !make_map(&m1, b1, p.b01_rows, kb, wbox) || !make_map(&m2, b2, r23, kb, wbox) ||
         !make_map(&m3, b3, r23, kb, wbox))
         return MOE_ERR_CUDA;
@@ -1131,19 +1228,32 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     a.rows_cap = p.rows_cap;
     a.pk_T = p.pk_T;
     a.pk_dq = p.pk_dq;
+    a.rows = p.rows;
+    a.rows_T = p.rows_T;
+    a.acc = p.acc;
+    a.acc_d = p.acc_d;
+    a.idx = p.idx;
+    a.gate = p.gate;
+    a.k = p.k;
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
     const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
     if constexpr (EPI == EPI_SWIGLU || EPI == EPI_F32) {
         if (tn) {
-            cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI>), P_SMEM_BYTES);
+            constexpr int FM = EPI == EPI_SWIGLU ? TN_GATHER : TN_SCATTER_ADD;
+            const void* fn = p.fuse ? reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI, FM>)
+                                    : reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI, TN_PLAIN>);
+            cudaError_t e = ensure_smem_attr(fn, P_SMEM_BYTES);
             if (e != cudaSuccess) return cuda_status(e);
             // a group of c rows has at most ceil(c / 256) token tiles
             const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
             const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
-            grouped_gemm_tn_kernel<EPI><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+            if (p.fuse) grouped_gemm_tn_kernel<EPI, FM><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+            else grouped_gemm_tn_kernel<EPI, TN_PLAIN><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
             count_launch();
             return cuda_status(cudaGetLastError());
         }
+    } else if (p.fuse) {
+        return MOE_ERR_UNSUPPORTED;
     }
     if (p.pair) {
         cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_pair_kernel<EPI>), P_SMEM_BYTES);

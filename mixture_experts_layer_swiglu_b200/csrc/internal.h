@@ -54,6 +54,19 @@ struct GemmProblem {
     int pair;             // 1: 256-row tiles on CTA pairs (cta_group::2); 0: 128-row tiles per CTA
     int tn_any;           // 1: the token-column pair form may run whatever `pair` says (groups of any size)
     int b_kmod;           // > 0: B has b_kmod columns and is repeated along K (B k = k mod b_kmod)
+    // fused permutation / combine (token-column pair form only; else MOE_ERR_UNSUPPORTED):
+    //   fuse == 1 (SwiGLU): row r of the grouped operand is row rows[r] of A (A = x [rows_T, K]),
+    //             and the tiles zero the rows rows[r] of acc [rows_T, acc_d];
+    //   fuse == 2 (fp32):   out row r is added, scaled by the gate of (token rows[r], the
+    //             group's expert) from idx / gate [rows_T, k], into acc row rows[r].
+    int fuse;
+    const int32_t* rows;
+    int rows_T;
+    float* acc;
+    int acc_d;
+    const int32_t* idx;
+    const float* gate;
+    int k;
 };
 
 moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st);
@@ -148,6 +161,8 @@ struct CombineArgs {
     int T, d, k, n_ffn, n_shared, n_zero, n_copy, n_const;
     long long rows_cap;
     int out_f32;               // y fp32 whatever the input dtype
+    int acc_rows;              // 1: ys is [T, d] fp32 per-token sums of the FFN slots' gated outputs
+                               //    (the fused combine); only the zero-computation slots are added here
 };
 moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st);
 

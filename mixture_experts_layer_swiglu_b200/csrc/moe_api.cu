@@ -137,6 +137,33 @@ size_t scratch_max(const moe_layer_desc* d)
     return std::max(std::max(s.route, s.permute), std::max(s.ffn, (size_t)256));
 }
 
+#ifndef MOE_FUSED_LAYER
+#define MOE_FUSED_LAYER 1     // moe_layer_forward takes the fused expert step where the layer allows it
+#endif
+
+// The fused expert step (gather in the gate/up GEMM's loads, combine in the
+// down GEMM's epilogue): token-column GEMM forms, and at most two FFN
+// contributions per token so that their fp32 sum does not depend on the
+// order the atomics land in.
+bool fused_eligible(const moe_layer_desc* d)
+{
+    return d->kind == MOE_EXPERT_SWIGLU && d->dtype == MOE_BF16 && d->n_ffn > 0 && d->n_shared == 0 &&
+           d->top_k <= 2 && d->d_model % 256 == 0 && d->hidden % 128 == 0;
+}
+
+struct FusedScratch {
+    size_t h, acc, total;     // hidden activation [cap, H] bf16, accumulator [T, d] fp32
+};
+
+FusedScratch fused_scratch(const moe_layer_desc* d)
+{
+    FusedScratch f;
+    f.h = al((size_t)moe_row_capacity(d) * d->hidden * 2);
+    f.acc = al((size_t)d->T * d->d_model * 4);
+    f.total = std::max(f.h + f.acc, (size_t)256);
+    return f;
+}
+
 struct LayerBufs {
     int32_t* idx;
     float* gate;
@@ -165,7 +192,10 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
     b.offsets = reinterpret_cast<int32_t*>(take((moe_num_groups(d) + 1) * 4));
     b.row_of = reinterpret_cast<int32_t*>(take(Tk * 4));
     b.token_of = reinterpret_cast<int32_t*>(take(cap * 4));
-    if (d->kind == MOE_EXPERT_SWIGLU) {
+    if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d)) {
+        b.xs = nullptr;   // the fused step gathers x rows itself and combines into its accumulator
+        b.ys = nullptr;
+    } else if (d->kind == MOE_EXPERT_SWIGLU) {
         b.xs = take((size_t)cap * d->d_model * elt(d));
         b.ys = take((size_t)cap * d->d_model * 4);
     } else {
@@ -173,6 +203,8 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
         b.ys = take(al((size_t)Tk * 4) + (size_t)d->n_shared * d->T * d->d_model * 4);
     }
     b.scratch_bytes = scratch_max(d);
+    if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d))
+        b.scratch_bytes = std::max(b.scratch_bytes, fused_scratch(d).total);
     b.scratch = take(b.scratch_bytes);
     b.total = o;
     return b;
@@ -526,6 +558,104 @@ moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, con
     return launch_combine(d->dtype, a, st);
 }
 
+// One phase of the fused expert step (0: all three).
+moe_status fused_impl(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* x,
+                      const int32_t* idx, const float* gate, const float* cmix, const int32_t* offsets,
+                      const int32_t* row_of, const int32_t* token_of, void* y, void* ws, size_t ws_bytes,
+                      cudaStream_t st)
+{
+    if (!fused_eligible(d)) return MOE_ERR_UNSUPPORTED;
+    if (d->T == 0) return MOE_OK;
+    const FusedScratch fs = fused_scratch(d);
+    if (!ws || ws_bytes < fs.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (!w->w_gate || !w->w_up || !w->w_down || !x || !offsets || !token_of) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[4] = {w->w_gate, w->w_up, w->w_down, x};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    void* h = ws;
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + fs.h);
+    const long long cap = moe_row_capacity(d);
+    moe_status s = MOE_OK;
+    if (phase == 0 || phase == 1) {
+        GemmProblem g{};
+        g.epi = EPI_SWIGLU;
+        g.A = x;
+        g.a_rows = d->T;
+        g.K = d->d_model;
+        g.B0 = w->w_gate;
+        g.B1 = w->w_up;
+        g.b01_rows = (long long)d->n_ffn * d->hidden;
+        g.offsets = offsets;
+        g.n_groups = d->n_ffn;
+        g.n_first = d->n_ffn;
+        g.N = d->hidden;
+        g.out = h;
+        g.ldo = d->hidden;
+        g.rows_cap = cap;
+        g.pair = 1;
+        g.fuse = 1;
+        g.rows = token_of;
+        g.rows_T = d->T;
+        g.acc = acc;
+        g.acc_d = d->d_model;
+        if ((s = launch_grouped_gemm(g, st)) != MOE_OK) return s;
+    }
+    if (phase == 0 || phase == 2) {
+        if (!idx || !gate) return MOE_ERR_INVALID_ARG;
+        GemmProblem g{};
+        g.epi = EPI_F32;
+        g.A = h;
+        g.a_rows = cap;
+        g.K = d->hidden;
+        g.B0 = w->w_down;
+        g.b01_rows = (long long)d->n_ffn * d->d_model;
+        g.offsets = offsets;
+        g.n_groups = d->n_ffn;
+        g.n_first = d->n_ffn;
+        g.N = d->d_model;
+        g.out = acc;
+        g.ldo = d->d_model;
+        g.rows_cap = d->T;
+        g.pair = 1;
+        g.fuse = 2;
+        g.rows = token_of;
+        g.rows_T = d->T;
+        g.acc = acc;
+        g.acc_d = d->d_model;
+        g.idx = idx;
+        g.gate = gate;
+        g.k = d->top_k;
+        if ((s = launch_grouped_gemm(g, st)) != MOE_OK) return s;
+    }
+    if (phase == 0 || phase == 3) {
+        if (!y || !aligned16(y) || !idx || !gate || !row_of) return MOE_ERR_INVALID_ARG;
+        if (d->n_const > 0 && (!cmix || !w->const_vec || !aligned16(w->const_vec))) return MOE_ERR_INVALID_ARG;
+        CombineArgs a{};
+        a.ys = acc;
+        a.offsets = offsets;
+        a.row_of = row_of;
+        a.idx = idx;
+        a.gate = gate;
+        a.const_mix = cmix;
+        a.const_vec = w->const_vec;
+        a.x = x;
+        a.y = y;
+        a.T = d->T;
+        a.d = d->d_model;
+        a.k = d->top_k;
+        a.n_ffn = d->n_ffn;
+        a.n_shared = 0;
+        a.n_zero = d->n_zero;
+        a.n_copy = d->n_copy;
+        a.n_const = d->n_const;
+        a.rows_cap = cap;
+        a.out_f32 = d->out_f32;
+        a.acc_rows = 1;
+        if ((s = launch_combine(d->dtype, a, st)) != MOE_OK) return s;
+    }
+    return MOE_OK;
+}
+
 }  // namespace
 
 moe_status validate_desc(const moe_layer_desc* d) { return check_desc(d); }
@@ -634,6 +764,25 @@ int64_t moe_layer_workspace_size(const moe_layer_desc* d)
     return (int64_t)layer_layout(d, nullptr).total;
 }
 
+int64_t moe_fused_workspace_size(const moe_layer_desc* d)
+{
+    if (check_desc(d) != MOE_OK || !fused_eligible(d)) return -1;
+    return (int64_t)fused_scratch(d).total;
+}
+
+moe_status moe_fused_ffn_combine(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* x,
+                                 const int32_t* topk_idx, const float* topk_gate, const float* const_mix,
+                                 const int32_t* expert_offsets, const int32_t* row_of, const int32_t* token_of,
+                                 void* y, void* workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    t_launches = 0;
+    moe_status s = check_desc(d);
+    if (s != MOE_OK) return s;
+    if (!w || phase < 0 || phase > 3) return MOE_ERR_INVALID_ARG;
+    return fused_impl(d, w, phase, x, topk_idx, topk_gate, const_mix, expert_offsets, row_of, token_of, y,
+                      workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_route(const moe_layer_desc* d, const moe_layer_weights* w, const void* x,
                      const float* prev_logits, float* logits_out, int32_t* topk_idx, float* topk_gate,
                      float* const_mix, void* workspace, size_t ws_bytes, moe_stream_t stream)
@@ -654,8 +803,6 @@ moe_status moe_permute(const moe_layer_desc* d, const int32_t* topk_idx, const v
     moe_status s = check_desc(d);
     if (s != MOE_OK) return s;
     if (!expert_offsets || (d->T > 0 && (!topk_idx || !row_of || !token_of))) return MOE_ERR_INVALID_ARG;
-    if (d->kind == MOE_EXPERT_SWIGLU && d->T > 0 && d->n_ffn + d->n_shared > 0 && !x_sorted)
-        return MOE_ERR_INVALID_ARG;
     return permute_impl(d, topk_idx, x, expert_offsets, row_of, token_of, x_sorted, workspace, ws_bytes,
                         static_cast<cudaStream_t>(stream));
 }
@@ -724,6 +871,9 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const moe_layer_weights* w
         return s;
     if ((s = permute_impl(d, b.idx, x, b.offsets, b.row_of, b.token_of, b.xs, b.scratch, b.scratch_bytes, st)) != MOE_OK)
         return s;
+    if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d))
+        return fused_impl(d, w, 0, x, b.idx, b.gate, b.cmix, b.offsets, b.row_of, b.token_of, y, b.scratch,
+                          b.scratch_bytes, st);
     if ((s = ffn_impl(d, w, b.xs, b.offsets, b.token_of, x, b.gate, b.ys, b.scratch, b.scratch_bytes, st)) != MOE_OK)
         return s;
     return combine_impl(d, w, b.ys, b.offsets, b.row_of, b.idx, b.gate, b.cmix, x, y, st);

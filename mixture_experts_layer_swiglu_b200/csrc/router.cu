@@ -25,6 +25,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <climits>
 
 #include "common.cuh"
@@ -35,6 +36,10 @@ namespace moe {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
+
+#ifndef MOE_ROUTER_STREAM
+#define MOE_ROUTER_STREAM 1       // bf16: the streaming tensor-core router (else router_mma_kernel)
+#endif
 constexpr int R_TPW = 4;         // tokens per warp
 constexpr int R_MAXROWS = 256;   // router rows + constant-mix rows
 
@@ -375,6 +380,208 @@ __global__ void __launch_bounds__(RM_WARPS * 32) router_mma_kernel(const RouterA
     }
 }
 
+// Streaming form of the tensor-core router (bf16 x, d a multiple of 64):
+// x is read once from HBM, so the kernel is built to keep HBM busy.  One
+// persistent block per SM; a producer warp copies each 16-token tile's rows
+// into shared memory with bulk copies (cp.async.bulk, no multicast), chunk
+// by chunk (16 rows x 1024 elements of d per chunk, one copy per row), into a
+// ring of RS_STAGES stages with mbarrier completion, running ahead across
+// tiles; 100-130 KiB are in flight per SM without holding a register.  The
+// 8 consumer warps split each chunk's d: warp w takes the 64-wide slices
+// w, w + 8 of the chunk and computes, for every group of 64 router rows, the
+// m16n8k16 tiles of those slices exactly as router_mma_kernel does (lane
+// (g, q) uses 32 contiguous bytes of token rows g and g + 8 and of router row
+// g of each n8 tile, in the same k order for A and B), reading x from shared
+// memory (rows padded by 16 bytes, so the fragment reads are conflict-free)
+// and the router rows from global memory through L1.  Each warp adds its
+// chunk's partial logits into its own shared-memory buffer; at the tile's
+// end the 8 partials are summed in warp order (fixed, so the logits do not
+// depend on timing) and each warp routes two tokens with route_token.
+constexpr int RS_WARPS = 8;                    // consumer warps
+constexpr int RS_THREADS = (RS_WARPS + 1) * 32;
+constexpr int RS_KC = 1024;                    // d elements per chunk
+constexpr int RS_PITCH = RS_KC * 2 + 16;       // bytes per staged row
+constexpr int RS_STAGE = 16 * RS_PITCH;        // 16 token rows
+constexpr int RS_MAXSTAGES = 4;
+constexpr int RS_SMEM_LIMIT = 227 * 1024;
+
+__host__ __device__ constexpr int rs_zpitch(int R) { return (R + 7) & ~7; }
+__host__ __device__ constexpr int rs_partial_bytes(int R) { return (RS_WARPS + 1) * 16 * rs_zpitch(R) * 4; }
+
+// Consumer-warp barrier (the producer warp never takes part).
+__device__ __forceinline__ void rs_consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(RS_WARPS * 32) : "memory"); }
+
+// Consumer-warp barrier that also returns whether `v` holds in every consumer thread.
+__device__ __forceinline__ bool rs_consumer_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v), "n"(RS_WARPS * 32) : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void lds256(uint32_t saddr, uint32_t (&r)[8])
+{
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%8];\n\t"
+                 "ld.shared.v4.u32 {%4,%5,%6,%7}, [%8+16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(saddr));
+}
+
+// 32-byte read-only global load that may allocate in L1 (router rows: every
+// tile of the block reads them again).
+__device__ __forceinline__ void ld256_l1(const unsigned char* p, uint32_t (&r)[8])
+{
+    asm("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "l"(p));
+}
+
+__global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const RouterArgs a, int stages)
+{
+    extern __shared__ __align__(128) unsigned char rs_smem[];
+    const int R = a.E_r + 2 * a.n_const;
+    const int zpitch = rs_zpitch(R);
+    unsigned char* ring = rs_smem;                                         // [stages][16 rows][RS_PITCH]
+    float* zpart = reinterpret_cast<float*>(rs_smem + (size_t)stages * RS_STAGE);   // [RS_WARPS][16][zpitch]
+    float* zsum = zpart + (size_t)RS_WARPS * 16 * zpitch;                  // [16][zpitch]
+    uint64_t* full = reinterpret_cast<uint64_t*>(zsum + 16 * zpitch);
+    uint64_t* empty = full + RS_MAXSTAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + RS_MAXSTAGES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t rowb = (size_t)a.d * 2;
+    const int nchunk = cdiv(a.d, RS_KC);
+    const int tiles = cdiv(a.T, 16);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], RS_WARPS); }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == RS_WARPS) {
+        // ---------------------------------------------------- producer warp
+        // lanes 0..15 each copy one token row of a chunk; lane 0 arms the stage
+        const unsigned char* xb = static_cast<const unsigned char*>(a.x);
+        int s = 0;
+        uint32_t ph = 0, pend = 0, pend_ph = 0;
+        bool bad = false;
+        for (int tile = blockIdx.x; tile < tiles && !bad; tile += gridDim.x) {
+            const int t0 = tile * 16;
+            const int rows = min(16, a.T - t0);
+            for (int c = 0; c < nchunk; ++c) {
+                const bool ok = *abort_flag == 0 && mbar_wait(&empty[s], ph ^ 1);
+                if (!__all_sync(FULL, ok)) { *abort_flag = 1; bad = true; break; }
+                const int e0 = c * RS_KC;
+                const int bytes = min(RS_KC, a.d - e0) * 2;
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(rows * bytes));
+                __syncwarp();
+                if (lane < rows)
+                    bulk_g2s(ring + (size_t)s * RS_STAGE + (size_t)lane * RS_PITCH,
+                             xb + (size_t)(t0 + lane) * rowb + (size_t)e0 * 2, (uint32_t)bytes, &full[s]);
+                pend |= 1u << s;
+                pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
+                if (++s == stages) { s = 0; ph ^= 1; }
+            }
+        }
+        // copies still in flight land before the block may exit
+        if (lane == 0)
+            for (int i = 0; i < stages; ++i)
+                if ((pend >> i) & 1u) mbar_wait(&full[i], (pend_ph >> i) & 1u);
+        return;
+    }
+
+    // -------------------------------------------------------- consumer warps
+    const int g = lane >> 2, q = lane & 3;
+    const unsigned char* wr = static_cast<const unsigned char*>(a.w_router);
+    const unsigned char* wc = static_cast<const unsigned char*>(a.w_const_mix);
+    float* zw = zpart + (size_t)warp * 16 * zpitch;
+    const uint32_t ring_s = smem_u32(ring);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int t0 = tile * 16;
+        for (int c = 0; c < nchunk; ++c) {
+            if (ok) ok = __all_sync(FULL, mbar_wait(&full[s], ph));   // warp-uniform: the MMAs need every lane
+            const int e0 = c * RS_KC;
+            const int nsl = min(RS_KC, a.d - e0) / 64;           // 64-wide slices in this chunk
+            const uint32_t st = ring_s + (uint32_t)(s * RS_STAGE);
+            for (int n0 = 0; n0 < R && ok; n0 += 8 * RM_NG) {
+                const int ntiles = min(RM_NG, (R - n0 + 7) / 8);
+                float acc[RM_NG][4];
+#pragma unroll
+                for (int nt = 0; nt < RM_NG; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 1
+                for (int sl = warp; sl < nsl; sl += RS_WARPS) {
+                    uint32_t xa[8], xb2[8];
+                    lds256(st + (uint32_t)(g * RS_PITCH + sl * 128 + q * 32), xa);
+                    lds256(st + (uint32_t)((g + 8) * RS_PITCH + sl * 128 + q * 32), xb2);
+                    const size_t off = (size_t)(e0 + sl * 64) * 2 + q * 32;
+#pragma unroll
+                    for (int nt = 0; nt < RM_NG; ++nt) {
+                        if (nt < ntiles) {
+                            const int j = min(n0 + nt * 8 + g, R - 1);   // rows past R repeat the last; never read
+                            const unsigned char* wrow = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
+                            uint32_t w[8];
+                            ld256_l1(wrow + off, w);
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                mma_16816(acc[nt], xa[2 * k4], xb2[2 * k4], xa[2 * k4 + 1], xb2[2 * k4 + 1], w[2 * k4],
+                                          w[2 * k4 + 1]);
+                        }
+                    }
+                }
+                // D fragment: acc[0], acc[1] = token g, rows 2q, 2q+1; acc[2], acc[3] = token g+8
+#pragma unroll
+                for (int nt = 0; nt < RM_NG; ++nt) {
+                    const int col = n0 + nt * 8 + 2 * q;
+                    if (nt < ntiles && col < zpitch) {
+                        float* z0 = zw + g * zpitch + col;
+                        float* z1 = zw + (g + 8) * zpitch + col;
+                        if (c == 0) { z0[0] = acc[nt][0]; z0[1] = acc[nt][1]; z1[0] = acc[nt][2]; z1[1] = acc[nt][3]; }
+                        else { z0[0] += acc[nt][0]; z0[1] += acc[nt][1]; z1[0] += acc[nt][2]; z1[1] += acc[nt][3]; }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);      // this warp is done with the stage
+            if (++s == stages) { s = 0; ph ^= 1; }
+        }
+        // all consumer warps agree to go on (a timed-out wait stops them together)
+        if (!rs_consumer_all(ok)) { *abort_flag = 1; break; }
+        // sum the 8 partials in warp order, then route two tokens per warp
+        for (int i = threadIdx.x; i < 16 * zpitch; i += RS_WARPS * 32) {
+            float v = zpart[i];
+#pragma unroll
+            for (int w2 = 1; w2 < RS_WARPS; ++w2) v += zpart[(size_t)w2 * 16 * zpitch + i];
+            zsum[i] = v;
+        }
+        rs_consumer_sync();
+        for (int tt = warp; tt < 16; tt += RS_WARPS) {
+            const int t = t0 + tt;
+            if (t < a.T) route_token(a, t, zsum + tt * zpitch, lane);
+        }
+        rs_consumer_sync();   // zsum and the partials are free for the next tile
+    }
+}
+
+int router_stream_stages(int R)
+{
+    const int fixed = rs_partial_bytes(R) + 2 * RS_MAXSTAGES * 8 + 16 + 128;
+    return std::min(RS_MAXSTAGES, (RS_SMEM_LIMIT - fixed) / RS_STAGE);
+}
+
+int router_stream_smem(int R, int stages)
+{
+    return stages * RS_STAGE + rs_partial_bytes(R) + 2 * RS_MAXSTAGES * 8 + 16;
+}
+
 // ------------------------------------------------------- product-key selection
 //
 // Every candidate gets one unsigned 64-bit key whose order is the selection
@@ -603,6 +810,19 @@ __global__ void pk_prep_keys_kernel(const __nv_bfloat16* kr, const __nv_bfloat16
 moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
+    if (dtype == MOE_BF16 && a.d % 64 == 0 && MOE_ROUTER_STREAM) {
+        const int R = a.E_r + 2 * a.n_const;
+        const int stages = router_stream_stages(R);
+        if (stages >= 2) {
+            const int smem = router_stream_smem(R, stages);
+            cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(router_stream_kernel), smem);
+            if (e != cudaSuccess) return cuda_status(e);
+            const int grid = std::max(1, std::min(cdiv(a.T, 16), num_sms()));
+            router_stream_kernel<<<grid, RS_THREADS, smem, st>>>(a, stages);
+            count_launch();
+            return cuda_status(cudaGetLastError());
+        }
+    }
     if (dtype == MOE_BF16 && a.d % 64 == 0) {
         const int R = a.E_r + 2 * a.n_const;
         const int smem = RM_WARPS * 16 * ((R + 7) & ~7) * 4;

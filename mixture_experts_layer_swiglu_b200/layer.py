@@ -77,6 +77,8 @@ class StageBuffers:
             c_floats = (T * k * 4 + 255) // 256 * 64
             self.y_sorted = torch.empty((max(c_floats + desc.n_shared * T * d, 1),), dtype=f32, device=device)
         self.workspace = torch.empty((abi.moe_workspace_size(desc),), dtype=torch.uint8, device=device)
+        fw = abi.moe_fused_workspace_size(desc)        # -1: the fused expert step does not apply
+        self.fused_workspace = torch.empty((fw,), dtype=torch.uint8, device=device) if fw > 0 else None
         self.y = torch.empty((T, d), dtype=out_dtype(desc), device=device)
 
 

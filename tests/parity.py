@@ -69,6 +69,33 @@ def run_gpu(cfg, inp_dev: dict, T: int | None = None) -> dict:
     return out
 
 
+def run_gpu_fused(cfg, inp_dev: dict, T: int | None = None) -> dict:
+    """Route, permute without x_sorted, then the fused expert step phase by
+    phase (gather in the gate/up GEMM, combine in the down GEMM's epilogue,
+    the zero-computation terms and the rounding last) with an fp32 output;
+    then phase 3 again with the layer's bf16 output, which must be exactly the
+    round-to-nearest-even of the fp32 one."""
+    desc = moe.desc_from(cfg, T, out_f32=True)
+    b = moe.StageBuffers(desc)
+    assert b.fused_workspace is not None, "the fused expert step does not apply to this layer"
+    x = inp_dev["x"]
+    cm = b.const_mix if desc.n_const > 0 else None
+    moe.moe_route(desc, inp_dev, x, inp_dev.get("z_prev"), b.logits, b.idx, b.gate, cm, b.workspace)
+    moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, None, b.workspace)
+    for phase in (1, 2, 3):
+        moe.moe_fused_ffn_combine(desc, inp_dev, phase, x, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of,
+                                  b.y, b.fused_workspace)
+    d16 = moe.desc_from(cfg, T, out_f32=False)
+    y16 = torch.empty(b.y.shape, dtype=torch.bfloat16, device=b.y.device)
+    moe.moe_fused_ffn_combine(d16, inp_dev, 3, x, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of, y16,
+                              b.fused_workspace)
+    torch.cuda.synchronize()
+    status = moe.moe_get_device_status(reset=True)
+    assert status == moe.MOE_OK, moe.status_string(status)
+    assert torch.equal(y16, b.y.to(torch.bfloat16)), "bf16 output != RNE(fp32 output)"
+    return {"desc": desc, "bufs": b, "y16": y16}
+
+
 def logit_error_bound(cfg, inp: dict, z_abs_max: np.ndarray) -> np.ndarray:
     """Per-token bound of |z_gpu - z_exact| for the SwiGLU router (fp32)."""
     x = inp["x"].double().abs()
@@ -138,10 +165,12 @@ def assert_close(y_gpu: np.ndarray, y_ref: np.ndarray, dtype: str, what: str = "
     return err / rms
 
 
-def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True) -> dict:
-    """Full check of a SwiGLU-kind layer; `tokens` limits the output comparison."""
+def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True, fused: bool = False) -> dict:
+    """Full check of a SwiGLU-kind layer; `tokens` limits the output comparison;
+    `fused` runs the fused expert step (no x_sorted to check)."""
     dev = to_device(inp)
-    r = run_gpu(cfg, dev)
+    r = run_gpu_fused(cfg, dev) if fused else run_gpu(cfg, dev)
+    check_sorted = check_sorted and not fused
     b = r["bufs"]
     T = cfg.T
     logits = b.logits.cpu().numpy().astype(np.float64)

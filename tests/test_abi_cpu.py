@@ -44,9 +44,14 @@ def test_sizes_and_groups(abi):
     assert abi.moe_row_capacity(d) == 8192
     ws = abi.moe_workspace_size(d)
     assert ws >= 8192 * 14336 * 2          # the hidden activation
-    assert abi.moe_layer_workspace_size(d) > ws + 2 * 8192 * 4096 * 2
+    # the layer takes the fused expert step: h and the [T, d] fp32 accumulator, no x_sorted / y_sorted
+    fw = abi.moe_fused_workspace_size(d)
+    assert fw >= 8192 * 14336 * 2 + 4096 * 4096 * 4
+    assert fw <= abi.moe_layer_workspace_size(d) < ws + fw + 2 * 8192 * 4096 * 2
     s = _desc(abi, T=2048, d_model=2048, top_k=6, n_ffn=64, hidden=1408, n_shared=2, hidden_shared=1408)
     assert abi.moe_num_groups(s) == 66 and abi.moe_row_capacity(s) == 2048 * 6 + 2 * 2048
+    assert abi.moe_fused_workspace_size(s) == -1        # shared experts, k = 6: the two-pass combine
+    assert abi.moe_layer_workspace_size(s) > 2 * (2048 * 6 + 2 * 2048) * 2048 * 2
     a = _desc(abi, T=8192, d_model=1024, top_k=64, kind="atomic", pk_rows=512, pk_cols=512,
               pk_topk_half=32, d_query=1024)
     assert abi.moe_num_groups(a) == 512 * 512 and abi.moe_row_capacity(a) == 8192 * 64
