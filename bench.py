@@ -226,8 +226,10 @@ def stage_names(cfg) -> list:
     return ["router", "permute", "gate_up_gemm", "down_gemm", "combine"]
 
 
-def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
-    """Algorithmic work of each stage: ("tensor", FLOPs) or ("hbm", bytes)."""
+def work_model(cfg, R_total: int, R_ffn: int, touched: int, fused: bool = False) -> dict:
+    """Algorithmic work of each stage: ("tensor", FLOPs) or ("hbm", bytes).
+    Fused expert step: the combine stage reads the [T, d] fp32 accumulator
+    the down GEMM formed (no y_sorted)."""
     d, T, k, e = cfg.d, cfg.T, cfg.top_k, cfg.elt_bytes
     if cfg.kind == "atomic":
         dq, N = cfg.d_query, cfg.n_atomic
@@ -251,6 +253,14 @@ def work_model(cfg, R_total: int, R_ffn: int, touched: int) -> dict:
     if cfg.gating_residual:
         router += T * E_r * 4
     zc_x = T * d * e if (cfg.n_copy + cfg.n_const) else 0
+    if fused:
+        return {
+            "router": ("hbm", router),
+            "permute": ("hbm", T * d * e + R_total * d * e + T * k * 12),
+            "gate_up_gemm": ("tensor", 4.0 * R_total * d * H),
+            "down_gemm": ("tensor", 2.0 * R_total * d * H),
+            "combine": ("hbm", T * d * 4 + T * d * e + zc_x + T * k * 12),
+        }
     return {
         "router": ("hbm", router),
         "permute": ("hbm", T * d * e + R_total * d * e + T * k * 12),
@@ -295,13 +305,22 @@ class Workload:
         self.ws = moe.weights_struct(self.w)
         self.b = moe.StageBuffers(self.desc, device=dev)
         self.atomic = cfg.kind == "atomic"
+        # the path moe_layer_forward takes: the fused expert step where it applies
+        self.fused = self.b.fused_workspace is not None
 
-    def calls(self, st):
+    def calls(self, st, fused=None):
         moe, cfg, b, x, ws, desc = self.moe, self.cfg, self.b, self.x, self.ws, self.desc
+        fused = self.fused if fused is None else fused
         cm = b.const_mix if cfg.n_const else None
         c = [lambda: moe.moe_route(desc, ws, x, self.zp, None, b.idx, b.gate, cm, b.workspace, st),
              lambda: moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, b.x_sorted, b.workspace,
                                      st)]
+        if fused:   # the combine in the down GEMM's epilogue, then the finish
+            for ph in (1, 2, 3):
+                c.append(lambda ph=ph: moe.moe_fused_ffn_combine(desc, ws, ph, x, b.x_sorted, b.idx, b.gate, cm,
+                                                                 b.offsets, b.row_of, b.token_of, b.y,
+                                                                 b.fused_workspace, st))
+            return c
         if self.atomic:   # the atomic step alone, then the shared dense branch's two GEMMs (if any)
             c.append(lambda: moe.moe_grouped_ffn(self.desc_atomic, ws, None, b.offsets, b.token_of, x, b.gate,
                                                  b.y_sorted, b.workspace, st))
@@ -317,14 +336,15 @@ class Workload:
         return c
 
 
-def time_workload(wl: Workload, K: int, warmup: int, dist, flush, want_graph: bool) -> dict:
+def time_workload(wl: Workload, K: int, warmup: int, dist, flush, want_graph: bool, fused=None) -> dict:
     """Warm-up, then K timed steps (L2 flushed and a GPU sleep before each,
     outside the events; CUDA events between the stages on the launching
     stream; SM clocks sampled meanwhile); times reduced to their maximum over
     ranks.  Every rank takes the same collective steps."""
     moe, dev = wl.moe, wl.dev
     stream = torch.cuda.current_stream(dev)
-    stage_calls = wl.calls(stream)
+    fused = wl.fused if fused is None else fused
+    stage_calls = wl.calls(stream, fused)
     names = stage_names(wl.cfg)
     nst = len(stage_calls)
 
@@ -371,18 +391,18 @@ def time_workload(wl: Workload, K: int, warmup: int, dist, flush, want_graph: bo
     R_total = int(off[-1].item())
     R_ffn = int(off[wl.cfg.n_ffn].item()) if not wl.atomic else R_total
     touched = int((off[1:] > off[:-1]).sum().item()) if wl.atomic else 0
-    graph_ms = graph_step_ms(wl.calls, stream, flush, sleep_cycles, K) if want_graph else 0.0
+    graph_ms = graph_step_ms(lambda st: wl.calls(st, fused), stream, flush, sleep_cycles, K) if want_graph else 0.0
     assert moe.moe_get_device_status(reset=True) == moe.MOE_OK
     mean = {n: sum(v) / K for n, v in per.items()}
     red = reduce_max_over_ranks(dist, [total_ms, graph_ms] + [mean[n] for n in names], dev)
     return {"names": names, "ms_step": red[0] / K, "graph_ms": red[1],
             "mean": {n: red[2 + j] for j, n in enumerate(names)}, "launches": launches,
-            "clocks": clk.summary(), "R_total": R_total, "R_ffn": R_ffn, "touched": touched}
+            "clocks": clk.summary(), "R_total": R_total, "R_ffn": R_ffn, "touched": touched, "fused": fused}
 
 
 def kernel_table(cfg, t: dict, peaks: Peaks) -> dict:
     """Per-stage time, share of the step and fraction of its roofline."""
-    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"])
+    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"], t["fused"])
     kern = {}
     for n in t["names"]:
         ms = t["mean"][n]
@@ -406,6 +426,7 @@ def workload_line(cfg, t: dict, world: int, peaks: Peaks) -> dict:
             "value": round(job_value(world, cfg.T, t["ms_step"]), 1), "unit": "tokens/s",
             "graph": {"ms_per_step": round(t["graph_ms"], 4),
                       "value": round(job_value(world, cfg.T, t["graph_ms"]), 1)},
+            "expert_step": "fused" if t["fused"] else "two-pass",
             "kernels": kernel_table(cfg, t, peaks), "gpu_launches": t["launches"], "clocks": t["clocks"],
             "rows": {"grouped": t["R_total"], "ffn": t["R_ffn"], "touched_experts": t["touched"]}}
 
@@ -451,6 +472,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     e2e_ms = reduce_max_over_ranks(dist, [e2e_ms / KE], dev)[0]
     del layer
 
+    # the two-pass expert step (x_sorted gather, y_sorted, combine kernel) on the
+    # same workload, for comparison with the fused one the layer takes
+    two_pass = None
+    if wl.fused:
+        two_pass = time_workload(wl, K, args.warmup, dist, flush, want_graph=False, fused=False)
+
     cublas = None
     if wl.atomic is False and cfg.dtype == "bf16" and rank == 0 and not args.no_library_ref:
         cublas = library_reference(cfg, t["R_total"], dev)
@@ -473,7 +500,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         return None
 
     kern = kernel_table(cfg, t, peaks)
-    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"])
+    work = work_model(cfg, t["R_total"], t["R_ffn"], t["touched"], t["fused"])
     ms_step = t["ms_step"]
     value = job_value(world, cfg.T, ms_step)
     names = t["names"]
@@ -512,6 +539,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         "gpu_launches": t["launches"],
         "clocks": t["clocks"],
     }
+    out["config"]["expert_step"] = "fused (combine in the down GEMM's epilogue)" if t["fused"] \
+        else "two-pass (permuted copy, expert GEMMs, combine kernel)"
+    if two_pass:
+        out["two_pass"] = {"ms_per_step": round(two_pass["ms_step"], 4),
+                           "value": round(job_value(world, cfg.T, two_pass["ms_step"]), 1),
+                           "kernels": kernel_table(cfg, two_pass, peaks)}
     if cublas:
         out["library_reference"] = cublas
     if others:
@@ -585,18 +618,27 @@ def library_reference(cfg, R_total: int, dev) -> dict:
 
 
 def _ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if
-    one exists for the current kernel source (else null)."""
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, when
+    the summary was taken from the current source of the file that holds the
+    kernel (its `source:` line names the file and its sha256); else null: a
+    changed kernel has no counters yet."""
+    import hashlib
     f = ROOT / "profiles" / f"{kernel}_{workload}.md"
     if not f.exists():
         return None
+    traffic, src_ok = None, False
     for line in f.read_text().splitlines():
         if line.startswith("dram_bytes_per_launch:"):
             try:
-                return float(line.split(":", 1)[1].split()[0])
+                traffic = float(line.split(":", 1)[1].split()[0])
             except ValueError:
                 return None
-    return None
+        elif line.startswith("source:"):
+            parts = line.split()
+            if len(parts) == 3 and parts[2].startswith("sha256:"):
+                src = ROOT / "mixture_experts_layer_swiglu_b200" / parts[1]
+                src_ok = src.exists() and hashlib.sha256(src.read_bytes()).hexdigest() == parts[2][7:]
+    return traffic if src_ok else None
 
 
 # -------------------------------------------------------------- reference

@@ -168,9 +168,9 @@ MOE_API moe_status moe_route(const moe_layer_desc* desc, const moe_layer_weights
  * token_of [row capacity]: SwiGLU: token of each row; atomic: flat slot id
  *   t*top_k + j of each task.
  * x_sorted [row capacity, d_model]: SwiGLU only, x_sorted[r] = x[token_of[r]];
- *   NULL for the atomic kind, and may be NULL for the SwiGLU kind when the
- *   fused expert step (moe_fused_ffn_combine) gathers the rows itself.  Rows
- *   past expert_offsets[groups] are untouched.
+ *   NULL for the atomic kind, and may be NULL for the SwiGLU kind (no copy
+ *   made) when the fused expert step gathers the rows itself.  Rows past
+ *   expert_offsets[groups] are untouched.
  * An id outside [0, n_ffn + n_zero + n_copy + n_const) (or the atomic grid)
  * sets MOE_ERR_DEVICE_BOUNDS in the device status and is skipped.
  */
@@ -243,9 +243,13 @@ MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weigh
  * assembled per token).  Same result as moe_grouped_ffn + moe_combine, with no
  * x_sorted and no y_sorted in memory:
  *   phase 1: h[r] = silu(W_gate[e] x[token_of[r]]) * (W_up[e] x[token_of[r]])
- *            for the rows r of expert e's group; the token rows are gathered
- *            by the GEMM's own loads (tile::gather4, no x_sorted); the same
- *            kernel zeroes the fp32 accumulator rows of the groups' tokens;
+ *            for the rows r of expert e's group, the token rows read from
+ *            moe_permute's x_sorted, or, with x_sorted NULL, gathered from x
+ *            by the GEMM's own loads (tile::gather4 of single rows; each row
+ *            is then fetched once per weight block, which measured 3x slower
+ *            than the gather copy on the Mixtral-shaped layer, so the layer
+ *            path passes x_sorted); the same kernel zeroes the fp32
+ *            accumulator rows of the groups' tokens;
  *   phase 2: acc[t] += g(t, e) * (W_down[e] h[r]) for t = token_of[r], by
  *            the GEMM's epilogue with vector atomics.  A token has at most
  *            two FFN slots, and two fp32 additions into zero give the same sum
@@ -259,8 +263,9 @@ MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weigh
  * of 256, hidden a multiple of 128.  moe_layer_forward uses this step for
  * every such layer.
  * Arguments as moe_route / moe_permute produce them (expert_offsets [n_ffn +
- * 1], row_of [T, top_k], token_of [T * top_k]); x [T, d_model]; y [T,
- * d_model] (bf16, or fp32 if desc->out_f32).  workspace: at least
+ * 1], row_of [T, top_k], token_of [T * top_k], x_sorted [row capacity,
+ * d_model] or NULL); x [T, d_model]; y [T, d_model] (bf16, or fp32 if
+ * desc->out_f32).  workspace: at least
  * moe_fused_workspace_size(desc) bytes (h, then the accumulator at byte
  * align256(cap * hidden * 2)); phases 1-3 called one by one must share it.
  * moe_fused_workspace_size returns -1 for a descriptor the step does not
@@ -268,7 +273,8 @@ MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weigh
  */
 MOE_API int64_t moe_fused_workspace_size(const moe_layer_desc* desc);
 MOE_API moe_status moe_fused_ffn_combine(const moe_layer_desc* desc, const moe_layer_weights* w, int phase,
-                                         const void* x, const int32_t* topk_idx, const float* topk_gate,
+                                         const void* x, const void* x_sorted, const int32_t* topk_idx,
+                                         const float* topk_gate,
                                          const float* const_mix, const int32_t* expert_offsets,
                                          const int32_t* row_of, const int32_t* token_of, void* y,
                                          void* workspace, size_t ws_bytes, moe_stream_t stream);

@@ -74,7 +74,7 @@ def load(path: Path | str | None = None):
     L.moe_layer_forward.argtypes = [D, W, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_fused_workspace_size.argtypes = [D]
     L.moe_fused_workspace_size.restype = I64
-    L.moe_fused_ffn_combine.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
+    L.moe_fused_ffn_combine.argtypes = [D, W, ctypes.c_int, VP, VP, VP, VP, VP, VP, VP, VP, VP, VP, SZ, VP]
     L.moe_layer_host_workspace_size.argtypes = [D, ctypes.c_int]
     L.moe_layer_host_workspace_size.restype = I64
     L.moe_layer_forward_host.argtypes = [D, W, VP, VP, VP, ctypes.c_int, VP, SZ, VP]
@@ -227,11 +227,13 @@ def moe_fused_workspace_size(desc: MoELayerDesc) -> int:
     return int(load().moe_fused_workspace_size(ctypes.byref(desc)))
 
 
-def moe_fused_ffn_combine(desc, weights, phase, x, topk_idx, topk_gate, const_mix, expert_offsets, row_of,
-                          token_of, y, workspace, stream=None) -> None:
+def moe_fused_ffn_combine(desc, weights, phase, x, x_sorted, topk_idx, topk_gate, const_mix, expert_offsets,
+                          row_of, token_of, y, workspace, stream=None) -> None:
+    """x_sorted None: phase 1 gathers the token rows from x by its own loads."""
     ws = weights if isinstance(weights, MoELayerWeights) else weights_struct(weights)
     _check("moe_fused_ffn_combine",
-           load().moe_fused_ffn_combine(ctypes.byref(desc), ctypes.byref(ws), int(phase), _p(x), _p(topk_idx),
+           load().moe_fused_ffn_combine(ctypes.byref(desc), ctypes.byref(ws), int(phase), _p(x), _p(x_sorted),
+                                        _p(topk_idx),
                                         _p(topk_gate), _p(const_mix), _p(expert_offsets), _p(row_of), _p(token_of),
                                         _p(y), _p(workspace), _nbytes(workspace), _stream(stream)))
 

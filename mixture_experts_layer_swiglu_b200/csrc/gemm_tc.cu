@@ -821,12 +821,13 @@ __device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body)
     }
 }
 
-// MODE: TN_PLAIN, TN_GATHER (SwiGLU only: the token rows of the B operand are
-// gathered from x by `rows` with tile::gather4 loads, and each tile zeroes its
-// share of its tokens' fp32 combine accumulator rows), TN_SCATTER_ADD (fp32
-// only: each output row is scaled by its token's gate for this group's expert
-// and added into the accumulator row of its token with vector atomics).
-enum TnMode { TN_PLAIN = 0, TN_GATHER = 1, TN_SCATTER_ADD = 2 };
+// MODE flags: TN_GATHER (SwiGLU: the token rows of the B operand are gathered
+// from x by `rows` with tile::gather4 loads instead of read from x_sorted),
+// TN_ZERO_ACC (SwiGLU: each tile zeroes its share of its tokens' fp32 combine
+// accumulator rows), TN_SCATTER_ADD (fp32: each output row is scaled by its
+// token's gate for this group's expert and added into the accumulator row of
+// its token with vector atomics).
+enum TnMode { TN_PLAIN = 0, TN_GATHER = 1, TN_SCATTER_ADD = 2, TN_ZERO_ACC = 4 };
 
 template <int EPI, int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
@@ -835,9 +836,10 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                        const __grid_constant__ CUtensorMap tmW3, const DevArgs a)
 {
     static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "token-column form: SwiGLU or fp32 epilogue");
-    static_assert(MODE == TN_PLAIN || (MODE == TN_GATHER && EPI == EPI_SWIGLU) ||
-                  (MODE == TN_SCATTER_ADD && EPI == EPI_F32), "fused modes: gather with SwiGLU, scatter-add with fp32");
-    constexpr bool GATHER = MODE == TN_GATHER;
+    static_assert(MODE == TN_PLAIN || (EPI == EPI_SWIGLU && (MODE == TN_ZERO_ACC || MODE == (TN_GATHER | TN_ZERO_ACC))) ||
+                  (EPI == EPI_F32 && MODE == TN_SCATTER_ADD), "fused modes: gather / zeroing with SwiGLU, scatter-add with fp32");
+    constexpr bool GATHER = (MODE & TN_GATHER) != 0;
+    constexpr bool ZERO_ACC = (MODE & TN_ZERO_ACC) != 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -1093,7 +1095,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                         finish(g, u, ch * 32 + 16);
                     }
                 });
-                if constexpr (GATHER) {
+                if constexpr (ZERO_ACC) {
                     // this tile's share of zeroing its tokens' combine accumulator rows:
                     // 16-byte units [m U / ntm, (m + 1) U / ntm) of each row, so the
                     // ntm weight blocks of a token tile clear its rows between them
@@ -1200,7 +1202,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
                     reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
                     ((EPI == EPI_SWIGLU && p.N % 128 == 0 && (p.K >= MOE_TN_SWIGLU_MIN_K || p.fuse)) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));
-    if (p.fuse && (!tn || (p.fuse == 1) != (EPI == EPI_SWIGLU) || (p.fuse == 2) != (EPI == EPI_F32) ||
+    // fuse: 1 = gathered B rows + zeroing, 3 = zeroing (B from x_sorted) -- SwiGLU; 2 = scatter-add -- fp32
+    const bool swiglu_fuse = p.fuse == 1 || p.fuse == 3;
+    if (p.fuse && (!tn || swiglu_fuse != (EPI == EPI_SWIGLU) || (p.fuse == 2) != (EPI == EPI_F32) ||
                    !p.rows || !p.acc || p.acc_d % 256 != 0 || p.rows_T <= 0 ||
                    (p.fuse == 1 && p.K % (BK * P_KH) != 0) || (p.fuse == 2 && (!p.idx || !p.gate || p.k <= 0)) ||
                    reinterpret_cast<uintptr_t>(p.acc) % 16 != 0))
@@ -1239,18 +1243,23 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
     if constexpr (EPI == EPI_SWIGLU || EPI == EPI_F32) {
         if (tn) {
-            constexpr int FM = EPI == EPI_SWIGLU ? TN_GATHER : TN_SCATTER_ADD;
-            const void* fn = p.fuse ? reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI, FM>)
-                                    : reinterpret_cast<const void*>(grouped_gemm_tn_kernel<EPI, TN_PLAIN>);
-            cudaError_t e = ensure_smem_attr(fn, P_SMEM_BYTES);
-            if (e != cudaSuccess) return cuda_status(e);
             // a group of c rows has at most ceil(c / 256) token tiles
             const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
             const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
-            if (p.fuse) grouped_gemm_tn_kernel<EPI, FM><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
-            else grouped_gemm_tn_kernel<EPI, TN_PLAIN><<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
-            count_launch();
-            return cuda_status(cudaGetLastError());
+            auto go = [&](auto kernel) {
+                cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), P_SMEM_BYTES);
+                if (e != cudaSuccess) return cuda_status(e);
+                kernel<<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+                count_launch();
+                return cuda_status(cudaGetLastError());
+            };
+            if constexpr (EPI == EPI_SWIGLU) {
+                if (p.fuse == 1) return go(grouped_gemm_tn_kernel<EPI, TN_GATHER | TN_ZERO_ACC>);
+                if (p.fuse == 3) return go(grouped_gemm_tn_kernel<EPI, TN_ZERO_ACC>);
+            } else {
+                if (p.fuse == 2) return go(grouped_gemm_tn_kernel<EPI, TN_SCATTER_ADD>);
+            }
+            return go(grouped_gemm_tn_kernel<EPI, TN_PLAIN>);
         }
     } else if (p.fuse) {
         return MOE_ERR_UNSUPPORTED;

@@ -57,6 +57,7 @@ struct GemmProblem {
     // fused permutation / combine (token-column pair form only; else MOE_ERR_UNSUPPORTED):
     //   fuse == 1 (SwiGLU): row r of the grouped operand is row rows[r] of A (A = x [rows_T, K]),
     //             and the tiles zero the rows rows[r] of acc [rows_T, acc_d];
+    //   fuse == 3 (SwiGLU): A is x_sorted as usual; the tiles zero the rows rows[r] of acc;
     //   fuse == 2 (fp32):   out row r is added, scaled by the gate of (token rows[r], the
     //             group's expert) from idx / gate [rows_T, k], into acc row rows[r].
     int fuse;

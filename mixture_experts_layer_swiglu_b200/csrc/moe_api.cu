@@ -193,8 +193,8 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
     b.row_of = reinterpret_cast<int32_t*>(take(Tk * 4));
     b.token_of = reinterpret_cast<int32_t*>(take(cap * 4));
     if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d)) {
-        b.xs = nullptr;   // the fused step gathers x rows itself and combines into its accumulator
-        b.ys = nullptr;
+        b.xs = take((size_t)cap * d->d_model * elt(d));
+        b.ys = nullptr;   // the fused step combines into its own accumulator
     } else if (d->kind == MOE_EXPERT_SWIGLU) {
         b.xs = take((size_t)cap * d->d_model * elt(d));
         b.ys = take((size_t)cap * d->d_model * 4);
@@ -560,7 +560,7 @@ moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, con
 
 // One phase of the fused expert step (0: all three).
 moe_status fused_impl(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* x,
-                      const int32_t* idx, const float* gate, const float* cmix, const int32_t* offsets,
+                      const void* xs, const int32_t* idx, const float* gate, const float* cmix, const int32_t* offsets,
                       const int32_t* row_of, const int32_t* token_of, void* y, void* ws, size_t ws_bytes,
                       cudaStream_t st)
 {
@@ -577,10 +577,12 @@ moe_status fused_impl(const moe_layer_desc* d, const moe_layer_weights* w, int p
     const long long cap = moe_row_capacity(d);
     moe_status s = MOE_OK;
     if (phase == 0 || phase == 1) {
+        // B rows from x_sorted, or (x_sorted NULL) gathered from x by the GEMM's own loads
+        if (xs && !aligned16(xs)) return MOE_ERR_INVALID_ARG;
         GemmProblem g{};
         g.epi = EPI_SWIGLU;
-        g.A = x;
-        g.a_rows = d->T;
+        g.A = xs ? xs : x;
+        g.a_rows = xs ? cap : d->T;
         g.K = d->d_model;
         g.B0 = w->w_gate;
         g.B1 = w->w_up;
@@ -593,7 +595,7 @@ moe_status fused_impl(const moe_layer_desc* d, const moe_layer_weights* w, int p
         g.ldo = d->hidden;
         g.rows_cap = cap;
         g.pair = 1;
-        g.fuse = 1;
+        g.fuse = xs ? 3 : 1;
         g.rows = token_of;
         g.rows_T = d->T;
         g.acc = acc;
@@ -771,15 +773,16 @@ int64_t moe_fused_workspace_size(const moe_layer_desc* d)
 }
 
 moe_status moe_fused_ffn_combine(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* x,
-                                 const int32_t* topk_idx, const float* topk_gate, const float* const_mix,
-                                 const int32_t* expert_offsets, const int32_t* row_of, const int32_t* token_of,
-                                 void* y, void* workspace, size_t ws_bytes, moe_stream_t stream)
+                                 const void* x_sorted, const int32_t* topk_idx, const float* topk_gate,
+                                 const float* const_mix, const int32_t* expert_offsets, const int32_t* row_of,
+                                 const int32_t* token_of, void* y, void* workspace, size_t ws_bytes,
+                                 moe_stream_t stream)
 {
     t_launches = 0;
     moe_status s = check_desc(d);
     if (s != MOE_OK) return s;
     if (!w || phase < 0 || phase > 3) return MOE_ERR_INVALID_ARG;
-    return fused_impl(d, w, phase, x, topk_idx, topk_gate, const_mix, expert_offsets, row_of, token_of, y,
+    return fused_impl(d, w, phase, x, x_sorted, topk_idx, topk_gate, const_mix, expert_offsets, row_of, token_of, y,
                       workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -872,7 +875,7 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const moe_layer_weights* w
     if ((s = permute_impl(d, b.idx, x, b.offsets, b.row_of, b.token_of, b.xs, b.scratch, b.scratch_bytes, st)) != MOE_OK)
         return s;
     if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d))
-        return fused_impl(d, w, 0, x, b.idx, b.gate, b.cmix, b.offsets, b.row_of, b.token_of, y, b.scratch,
+        return fused_impl(d, w, 0, x, b.xs, b.idx, b.gate, b.cmix, b.offsets, b.row_of, b.token_of, y, b.scratch,
                           b.scratch_bytes, st);
     if ((s = ffn_impl(d, w, b.xs, b.offsets, b.token_of, x, b.gate, b.ys, b.scratch, b.scratch_bytes, st)) != MOE_OK)
         return s;

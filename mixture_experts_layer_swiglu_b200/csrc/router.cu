@@ -380,33 +380,36 @@ __global__ void __launch_bounds__(RM_WARPS * 32) router_mma_kernel(const RouterA
     }
 }
 
-// Streaming form of the tensor-core router (bf16 x, d a multiple of 64):
-// x is read once from HBM, so the kernel is built to keep HBM busy.  One
-// persistent block per SM; a producer warp copies each 16-token tile's rows
-// into shared memory with bulk copies (cp.async.bulk, no multicast), chunk
-// by chunk (16 rows x 1024 elements of d per chunk, one copy per row), into a
-// ring of RS_STAGES stages with mbarrier completion, running ahead across
-// tiles; 100-130 KiB are in flight per SM without holding a register.  The
-// 8 consumer warps split each chunk's d: warp w takes the 64-wide slices
-// w, w + 8 of the chunk and computes, for every group of 64 router rows, the
-// m16n8k16 tiles of those slices exactly as router_mma_kernel does (lane
-// (g, q) uses 32 contiguous bytes of token rows g and g + 8 and of router row
-// g of each n8 tile, in the same k order for A and B), reading x from shared
-// memory (rows padded by 16 bytes, so the fragment reads are conflict-free)
-// and the router rows from global memory through L1.  Each warp adds its
-// chunk's partial logits into its own shared-memory buffer; at the tile's
-// end the 8 partials are summed in warp order (fixed, so the logits do not
-// depend on timing) and each warp routes two tokens with route_token.
-constexpr int RS_WARPS = 8;                    // consumer warps
+// Streaming form of the tensor-core router (bf16 x, d a multiple of 64, at
+// most 64 router + mixing rows): x is read once from HBM, so the kernel is
+// built to keep HBM busy.  One persistent block per SM; a producer warp
+// copies each 16-token tile's rows into shared memory with bulk copies
+// (cp.async.bulk, no multicast), chunk by chunk (16 rows x 1024 elements of d
+// per chunk, one copy per row), into a ring of stages with mbarrier
+// completion, running ahead across tiles (100-130 KiB in flight per SM).
+// The router rows are copied into shared memory once per block when they fit
+// (else read through L1).  The 16 consumer warps split each chunk's d: warp w
+// takes the 64-wide slices w, w + 16 of the chunk and accumulates, in
+// registers across the tile's chunks, the m16n8k16 tiles of those slices as
+// router_mma_kernel does (lane (g, q) uses 32 contiguous bytes of token rows g
+// and g + 8 and of router row g of each n8 tile, in the same k order for A and
+// B); rows are padded by 16 bytes in shared memory so the fragment reads are
+// conflict-free.  At the tile's end the 16 partial logits are summed in warp
+// order (fixed, so the logits do not depend on timing) and each warp routes
+// one token with route_token, while the producer already streams the next
+// tile.
+constexpr int RS_WARPS = 16;                   // consumer warps
 constexpr int RS_THREADS = (RS_WARPS + 1) * 32;
 constexpr int RS_KC = 1024;                    // d elements per chunk
 constexpr int RS_PITCH = RS_KC * 2 + 16;       // bytes per staged row
 constexpr int RS_STAGE = 16 * RS_PITCH;        // 16 token rows
 constexpr int RS_MAXSTAGES = 4;
+constexpr int RS_MAXROWS = 8 * RM_NG;          // router + mixing rows (one group of n8 tiles)
 constexpr int RS_SMEM_LIMIT = 227 * 1024;
 
 __host__ __device__ constexpr int rs_zpitch(int R) { return (R + 7) & ~7; }
 __host__ __device__ constexpr int rs_partial_bytes(int R) { return (RS_WARPS + 1) * 16 * rs_zpitch(R) * 4; }
+__host__ __device__ constexpr int rs_wpitch(int d) { return d * 2 + 16; }
 
 // Consumer-warp barrier (the producer warp never takes part).
 __device__ __forceinline__ void rs_consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(RS_WARPS * 32) : "memory"); }
@@ -441,21 +444,52 @@ __device__ __forceinline__ void ld256_l1(const unsigned char* p, uint32_t (&r)[8
         : "l"(p));
 }
 
-__global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const RouterArgs a, int stages)
+struct RsLayout {
+    int stages;
+    bool w_smem;      // router rows staged in shared memory
+    int w_off, z_off, bar_off, bytes;
+};
+
+__host__ __device__ inline RsLayout rs_layout(int R, int d)
+{
+    RsLayout L;
+    const int part = rs_partial_bytes(R);
+    const int wbytes = ((R * rs_wpitch(d)) + 127) & ~127;
+    const int fixed = part + 2 * RS_MAXSTAGES * 8 + 16;
+    L.w_smem = RS_SMEM_LIMIT - fixed - wbytes >= 3 * RS_STAGE;
+    const int avail = RS_SMEM_LIMIT - fixed - (L.w_smem ? wbytes : 0);
+    L.stages = avail / RS_STAGE < RS_MAXSTAGES ? avail / RS_STAGE : RS_MAXSTAGES;
+    L.w_off = L.stages * RS_STAGE;
+    L.z_off = L.w_off + (L.w_smem ? wbytes : 0);
+    L.bar_off = L.z_off + part;
+    L.bytes = L.bar_off + 2 * RS_MAXSTAGES * 8 + 16;
+    return L;
+}
+
+// NT: n8 tiles of router + mixing rows (R <= 8 NT); the accumulators of
+// exactly those tiles live in registers.
+template <int NT>
+__global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const RouterArgs a)
 {
     extern __shared__ __align__(128) unsigned char rs_smem[];
     const int R = a.E_r + 2 * a.n_const;
     const int zpitch = rs_zpitch(R);
-    unsigned char* ring = rs_smem;                                         // [stages][16 rows][RS_PITCH]
-    float* zpart = reinterpret_cast<float*>(rs_smem + (size_t)stages * RS_STAGE);   // [RS_WARPS][16][zpitch]
-    float* zsum = zpart + (size_t)RS_WARPS * 16 * zpitch;                  // [16][zpitch]
-    uint64_t* full = reinterpret_cast<uint64_t*>(zsum + 16 * zpitch);
+    const RsLayout L = rs_layout(R, a.d);
+    const int stages = L.stages;
+    unsigned char* ring = rs_smem;                                          // [stages][16 rows][RS_PITCH]
+    unsigned char* wsm = rs_smem + L.w_off;                                 // [R][wpitch] (if w_smem)
+    float* zpart = reinterpret_cast<float*>(rs_smem + L.z_off);             // [RS_WARPS][16][zpitch]
+    float* zsum = zpart + (size_t)RS_WARPS * 16 * zpitch;                   // [16][zpitch]
+    uint64_t* full = reinterpret_cast<uint64_t*>(rs_smem + L.bar_off);
     uint64_t* empty = full + RS_MAXSTAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + RS_MAXSTAGES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t rowb = (size_t)a.d * 2;
+    const int wpitch = rs_wpitch(a.d);
     const int nchunk = cdiv(a.d, RS_KC);
     const int tiles = cdiv(a.T, 16);
+    const unsigned char* wr = static_cast<const unsigned char*>(a.w_router);
+    const unsigned char* wc = static_cast<const unsigned char*>(a.w_const_mix);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], RS_WARPS); }
@@ -497,65 +531,72 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
     }
 
     // -------------------------------------------------------- consumer warps
+    if (L.w_smem) {   // router rows (then mixing rows) into shared memory, once
+        const int vpr = a.d / 8;                                  // 16-byte vectors per row
+        for (int i = threadIdx.x; i < R * vpr; i += RS_WARPS * 32) {
+            const int j = i / vpr, v = i - j * vpr;
+            const unsigned char* src = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
+            *reinterpret_cast<uint4*>(wsm + (size_t)j * wpitch + v * 16) =
+                __ldg(reinterpret_cast<const uint4*>(src) + v);
+        }
+        rs_consumer_sync();
+    }
     const int g = lane >> 2, q = lane & 3;
-    const unsigned char* wr = static_cast<const unsigned char*>(a.w_router);
-    const unsigned char* wc = static_cast<const unsigned char*>(a.w_const_mix);
     float* zw = zpart + (size_t)warp * 16 * zpitch;
-    const uint32_t ring_s = smem_u32(ring);
+    const uint32_t ring_s = smem_u32(ring), wsm_s = smem_u32(wsm);
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int t0 = tile * 16;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         for (int c = 0; c < nchunk; ++c) {
             if (ok) ok = __all_sync(FULL, mbar_wait(&full[s], ph));   // warp-uniform: the MMAs need every lane
             const int e0 = c * RS_KC;
             const int nsl = min(RS_KC, a.d - e0) / 64;           // 64-wide slices in this chunk
             const uint32_t st = ring_s + (uint32_t)(s * RS_STAGE);
-            for (int n0 = 0; n0 < R && ok; n0 += 8 * RM_NG) {
-                const int ntiles = min(RM_NG, (R - n0 + 7) / 8);
-                float acc[RM_NG][4];
-#pragma unroll
-                for (int nt = 0; nt < RM_NG; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll 1
-                for (int sl = warp; sl < nsl; sl += RS_WARPS) {
-                    uint32_t xa[8], xb2[8];
-                    lds256(st + (uint32_t)(g * RS_PITCH + sl * 128 + q * 32), xa);
-                    lds256(st + (uint32_t)((g + 8) * RS_PITCH + sl * 128 + q * 32), xb2);
-                    const size_t off = (size_t)(e0 + sl * 64) * 2 + q * 32;
+            for (int sl = warp; sl < nsl && ok; sl += RS_WARPS) {
+                uint32_t xa[8], xb2[8];
+                lds256(st + (uint32_t)(g * RS_PITCH + sl * 128 + q * 32), xa);
+                lds256(st + (uint32_t)((g + 8) * RS_PITCH + sl * 128 + q * 32), xb2);
+                const int off = (e0 + sl * 64) * 2 + q * 32;      // byte offset in a router row
 #pragma unroll
-                    for (int nt = 0; nt < RM_NG; ++nt) {
-                        if (nt < ntiles) {
-                            const int j = min(n0 + nt * 8 + g, R - 1);   // rows past R repeat the last; never read
-                            const unsigned char* wrow = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
-                            uint32_t w[8];
-                            ld256_l1(wrow + off, w);
-#pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4)
-                                mma_16816(acc[nt], xa[2 * k4], xb2[2 * k4], xa[2 * k4 + 1], xb2[2 * k4 + 1], w[2 * k4],
-                                          w[2 * k4 + 1]);
-                        }
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int j = min(nt * 8 + g, R - 1);          // rows past R repeat the last; never read
+                    uint32_t w[8];
+                    if (L.w_smem) {
+                        lds256(wsm_s + (uint32_t)(j * wpitch + off), w);
+                    } else {
+                        const unsigned char* wrow = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
+                        ld256_l1(wrow + off, w);
                     }
-                }
-                // D fragment: acc[0], acc[1] = token g, rows 2q, 2q+1; acc[2], acc[3] = token g+8
 #pragma unroll
-                for (int nt = 0; nt < RM_NG; ++nt) {
-                    const int col = n0 + nt * 8 + 2 * q;
-                    if (nt < ntiles && col < zpitch) {
-                        float* z0 = zw + g * zpitch + col;
-                        float* z1 = zw + (g + 8) * zpitch + col;
-                        if (c == 0) { z0[0] = acc[nt][0]; z0[1] = acc[nt][1]; z1[0] = acc[nt][2]; z1[1] = acc[nt][3]; }
-                        else { z0[0] += acc[nt][0]; z0[1] += acc[nt][1]; z1[0] += acc[nt][2]; z1[1] += acc[nt][3]; }
-                    }
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        mma_16816(acc[nt], xa[2 * k4], xb2[2 * k4], xa[2 * k4 + 1], xb2[2 * k4 + 1], w[2 * k4],
+                                  w[2 * k4 + 1]);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);      // this warp is done with the stage
             if (++s == stages) { s = 0; ph ^= 1; }
         }
+        // D fragment: acc[0], acc[1] = token g, rows 2q, 2q+1; acc[2], acc[3] = token g+8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int col = nt * 8 + 2 * q;
+            if (col < zpitch) {
+                zw[g * zpitch + col] = acc[nt][0];
+                zw[g * zpitch + col + 1] = acc[nt][1];
+                zw[(g + 8) * zpitch + col] = acc[nt][2];
+                zw[(g + 8) * zpitch + col + 1] = acc[nt][3];
+            }
+        }
         // all consumer warps agree to go on (a timed-out wait stops them together)
         if (!rs_consumer_all(ok)) { *abort_flag = 1; break; }
-        // sum the 8 partials in warp order, then route two tokens per warp
+        // sum the partials in warp order, then route one token per warp
         for (int i = threadIdx.x; i < 16 * zpitch; i += RS_WARPS * 32) {
             float v = zpart[i];
 #pragma unroll
@@ -563,23 +604,18 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
             zsum[i] = v;
         }
         rs_consumer_sync();
-        for (int tt = warp; tt < 16; tt += RS_WARPS) {
-            const int t = t0 + tt;
-            if (t < a.T) route_token(a, t, zsum + tt * zpitch, lane);
-        }
+        if (t0 + warp < a.T) route_token(a, t0 + warp, zsum + warp * zpitch, lane);
         rs_consumer_sync();   // zsum and the partials are free for the next tile
     }
 }
 
-int router_stream_stages(int R)
+// Shared-memory bytes of router_stream_kernel, or 0 if the layer does not
+// fit its limits (more than 64 rows, or fewer than 2 stages).
+int router_stream_smem(int R, int d)
 {
-    const int fixed = rs_partial_bytes(R) + 2 * RS_MAXSTAGES * 8 + 16 + 128;
-    return std::min(RS_MAXSTAGES, (RS_SMEM_LIMIT - fixed) / RS_STAGE);
-}
-
-int router_stream_smem(int R, int stages)
-{
-    return stages * RS_STAGE + rs_partial_bytes(R) + 2 * RS_MAXSTAGES * 8 + 16;
+    if (R > RS_MAXROWS) return 0;
+    const RsLayout L = rs_layout(R, d);
+    return L.stages >= 2 ? L.bytes : 0;
 }
 
 // ------------------------------------------------------- product-key selection
@@ -812,15 +848,22 @@ moe_status launch_router(int dtype, const RouterArgs& a, cudaStream_t st)
     if (a.T == 0) return MOE_OK;
     if (dtype == MOE_BF16 && a.d % 64 == 0 && MOE_ROUTER_STREAM) {
         const int R = a.E_r + 2 * a.n_const;
-        const int stages = router_stream_stages(R);
-        if (stages >= 2) {
-            const int smem = router_stream_smem(R, stages);
-            cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(router_stream_kernel), smem);
-            if (e != cudaSuccess) return cuda_status(e);
+        const int smem = router_stream_smem(R, a.d);
+        if (smem > 0) {
             const int grid = std::max(1, std::min(cdiv(a.T, 16), num_sms()));
-            router_stream_kernel<<<grid, RS_THREADS, smem, st>>>(a, stages);
-            count_launch();
-            return cuda_status(cudaGetLastError());
+            auto go = [&](auto kernel) {
+                cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem);
+                if (e != cudaSuccess) return cuda_status(e);
+                kernel<<<grid, RS_THREADS, smem, st>>>(a);
+                count_launch();
+                return cuda_status(cudaGetLastError());
+            };
+            const int nt = (R + 7) / 8;
+            if (nt <= 1) return go(router_stream_kernel<1>);
+            if (nt <= 2) return go(router_stream_kernel<2>);
+            if (nt <= 3) return go(router_stream_kernel<3>);
+            if (nt <= 4) return go(router_stream_kernel<4>);
+            return go(router_stream_kernel<8>);
         }
     }
     if (dtype == MOE_BF16 && a.d % 64 == 0) {

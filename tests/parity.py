@@ -69,25 +69,27 @@ def run_gpu(cfg, inp_dev: dict, T: int | None = None) -> dict:
     return out
 
 
-def run_gpu_fused(cfg, inp_dev: dict, T: int | None = None) -> dict:
-    """Route, permute without x_sorted, then the fused expert step phase by
-    phase (gather in the gate/up GEMM, combine in the down GEMM's epilogue,
-    the zero-computation terms and the rounding last) with an fp32 output;
-    then phase 3 again with the layer's bf16 output, which must be exactly the
-    round-to-nearest-even of the fp32 one."""
+def run_gpu_fused(cfg, inp_dev: dict, T: int | None = None, gather: bool = False) -> dict:
+    """Route, permute, then the fused expert step phase by phase (gate/up
+    GEMM reading x_sorted -- or, with `gather`, gathering the token rows from
+    x by its own loads, no x_sorted made -- combine in the down GEMM's
+    epilogue, the zero-computation terms and the rounding last) with an fp32
+    output; then phase 3 again with the layer's bf16 output, which must be
+    exactly the round-to-nearest-even of the fp32 one."""
     desc = moe.desc_from(cfg, T, out_f32=True)
     b = moe.StageBuffers(desc)
     assert b.fused_workspace is not None, "the fused expert step does not apply to this layer"
     x = inp_dev["x"]
     cm = b.const_mix if desc.n_const > 0 else None
     moe.moe_route(desc, inp_dev, x, inp_dev.get("z_prev"), b.logits, b.idx, b.gate, cm, b.workspace)
-    moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, None, b.workspace)
+    xs = None if gather else b.x_sorted
+    moe.moe_permute(desc, b.idx, x, b.offsets, b.row_of, b.token_of, xs, b.workspace)
     for phase in (1, 2, 3):
-        moe.moe_fused_ffn_combine(desc, inp_dev, phase, x, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of,
+        moe.moe_fused_ffn_combine(desc, inp_dev, phase, x, xs, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of,
                                   b.y, b.fused_workspace)
     d16 = moe.desc_from(cfg, T, out_f32=False)
     y16 = torch.empty(b.y.shape, dtype=torch.bfloat16, device=b.y.device)
-    moe.moe_fused_ffn_combine(d16, inp_dev, 3, x, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of, y16,
+    moe.moe_fused_ffn_combine(d16, inp_dev, 3, x, xs, b.idx, b.gate, cm, b.offsets, b.row_of, b.token_of, y16,
                               b.fused_workspace)
     torch.cuda.synchronize()
     status = moe.moe_get_device_status(reset=True)
@@ -165,12 +167,14 @@ def assert_close(y_gpu: np.ndarray, y_ref: np.ndarray, dtype: str, what: str = "
     return err / rms
 
 
-def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True, fused: bool = False) -> dict:
+def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True, fused: bool = False,
+                       gather: bool = False) -> dict:
     """Full check of a SwiGLU-kind layer; `tokens` limits the output comparison;
-    `fused` runs the fused expert step (no x_sorted to check)."""
+    `fused` runs the fused expert step (`gather`: with its own row gather, no
+    x_sorted to check)."""
     dev = to_device(inp)
-    r = run_gpu_fused(cfg, dev) if fused else run_gpu(cfg, dev)
-    check_sorted = check_sorted and not fused
+    r = run_gpu_fused(cfg, dev, gather=gather) if fused else run_gpu(cfg, dev)
+    check_sorted = check_sorted and not (fused and gather)
     b = r["bufs"]
     T = cfg.T
     logits = b.logits.cpu().numpy().astype(np.float64)

@@ -1,9 +1,10 @@
 """The expert-parallel layer on one GPU through NCCL (a group of one rank).
 
 With one rank every expert is local, so the exchange reduces to local copies,
-and the layer must equal moe_layer_forward bit for bit: the same permutation,
-the same grouped GEMMs over the received rows (the owned experts as groups),
-the same combine.  Several ranks need several GPUs; their exchange logic is
+and the layer must equal the two-pass path (moe_route, moe_permute,
+moe_grouped_ffn, moe_combine) bit for bit: the same permutation, the same
+grouped GEMMs over the received rows (the owned experts as groups), the same
+combine.  Several ranks need several GPUs; their exchange logic is
 covered by the gloo tests (test_ep_ranks.py).
 """
 
@@ -42,12 +43,14 @@ def nccl_group():
 
 
 @pytest.mark.parametrize("name,T", [("mixtral", 600), ("moepp", 700)])
-def test_expert_parallel_one_rank_equals_layer_forward(nccl_group, name, T):
+def test_expert_parallel_one_rank_equals_two_pass_layer(nccl_group, name, T):
     base = get_config(name)
     cfg = scaled(base, T=T, d=2048 if name == "mixtral" else 256, hidden=512 if name == "mixtral" else 256)
     inp = to_device(make_inputs(cfg))
     desc = moe.desc_from(cfg)
-    y_ref = moe.MoELayer(desc, inp).forward(inp["x"], prev_logits=inp.get("z_prev"))
+    stages = moe.StageBuffers(desc)
+    moe.run_stages(desc, inp, inp["x"], stages, prev_logits=inp.get("z_prev"))
+    y_ref = stages.y
     lo, hi = moe.moe_ep_expert_range(1, cfg.n_ffn, 0)
     assert (lo, hi) == (0, cfg.n_ffn)
     layer = ep.ExpertParallelMoELayer(desc, ep.local_expert_weights(inp, lo, hi))

@@ -1,8 +1,8 @@
 """The fused expert step (moe_fused_ffn_combine) through the C ABI vs the
-fp64 oracle, element by element: token rows gathered by the gate/up GEMM's
-own loads (no x_sorted), the gate-weighted combine done by the down GEMM's
-epilogue into an fp32 accumulator (no y_sorted), then the zero-computation
-terms and one rounding.  Routing and the permutation are checked as for the
+fp64 oracle, element by element: the gate/up GEMM on x_sorted (or, `gather`,
+on token rows it gathers from x with its own loads), the gate-weighted
+combine done by the down GEMM's epilogue into an fp32 accumulator (no
+y_sorted), then the zero-computation terms and one rounding.  Routing and the permutation are checked as for the
 two-pass path; the bf16 output must be the round-to-nearest-even of the fp32
 result.  moe_layer_forward takes this step for every layer it applies to.
 """
@@ -35,18 +35,20 @@ def _sample(T: int, n: int, seed: int = 0) -> np.ndarray:
     return np.array(sorted(s), dtype=np.int32)
 
 
+@pytest.mark.parametrize("gather", [False, True])
 @pytest.mark.parametrize("T,d,H,E", [(333, 256, 384, 4), (600, 2048, 512, 2), (1100, 2048, 1024, 4),
                                      (513, 512, 256, 2)])
-def test_fused_mixtral_shaped_ragged(T, d, H, E):
+def test_fused_mixtral_shaped_ragged(T, d, H, E, gather):
     cfg = scaled(get_config("mixtral"), T=T, d=d, hidden=H, n_ffn=E)
-    rep = check_swiglu_layer(cfg, make_inputs(cfg), fused=True)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg), fused=True, gather=gather)
     assert rep["R"] == T * 2
 
 
+@pytest.mark.parametrize("gather", [False, True])
 @pytest.mark.parametrize("T", [1, 2, 127, 129])
-def test_fused_token_counts_across_tile_edges(T):
+def test_fused_token_counts_across_tile_edges(T, gather):
     cfg = scaled(get_config("mixtral"), T=T, d=256, hidden=384, n_ffn=4)
-    check_swiglu_layer(cfg, make_inputs(cfg), fused=True)
+    check_swiglu_layer(cfg, make_inputs(cfg), fused=True, gather=gather)
 
 
 def test_fused_moepp_zero_copy_const_and_tokens_without_ffn_slots():
@@ -57,6 +59,7 @@ def test_fused_moepp_zero_copy_const_and_tokens_without_ffn_slots():
     inp = make_inputs(cfg)
     rep = check_swiglu_layer(cfg, inp, fused=True)
     assert rep["R"] < 300 * 2
+    check_swiglu_layer(cfg, inp, fused=True, gather=True)
     idx = rep["idx_oracle"]
     assert ((idx >= cfg.n_ffn).all(axis=1)).any(), "the case should hold a token with no FFN slot"
 
@@ -99,8 +102,8 @@ def test_fused_step_refuses_layers_it_does_not_cover():
     assert moe.moe_fused_workspace_size(desc) == -1
     b = moe.StageBuffers(desc)
     with pytest.raises(moe.MoEError) as e:
-        moe.moe_fused_ffn_combine(desc, inp, 0, inp["x"], b.idx, b.gate, None, b.offsets, b.row_of, b.token_of,
-                                  b.y, b.workspace)
+        moe.moe_fused_ffn_combine(desc, inp, 0, inp["x"], b.x_sorted, b.idx, b.gate, None, b.offsets, b.row_of,
+                                  b.token_of, b.y, b.workspace)
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED
 
 
