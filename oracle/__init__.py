@@ -66,6 +66,15 @@ def lib():
             ctypes.c_int, _I32P, _I32P, _F64P, _F64P]
         L.orc_omni_tokens.argtypes = [ctypes.c_int] * 3 + [_VP] * 3 + [ctypes.c_int] * 2 + [_VP] * 3 + [
             ctypes.c_int, _I32P, _I32P, _F64P, _F64P]
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_round.argtypes = [ctypes.c_double]
+        L.orc_e4m3_round.restype = ctypes.c_double
+        L.orc_pow2_scale.argtypes = [ctypes.c_double]
+        L.orc_pow2_scale.restype = ctypes.c_double
+        L.orc_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _VP, _F64P, _F64P]
+        L.orc_fp8_moe_tokens.argtypes = [ctypes.POINTER(_Layer)] + [_VP] * 18 + [
+            ctypes.c_int, _I32P, _I32P, _F64P, _I32P, _F64P, _F64P]
         _lib = L
     return _lib
 
@@ -258,3 +267,77 @@ def atomic_tokens(x, u, v, tokens, idx, gate, shared=None) -> np.ndarray:
         lib().orc_omni_tokens(d, K, _dt(x, u, v, sg, su, sd), _vp(x), _vp(u), _vp(v), S, Hs, _vp(sg), _vp(su),
                               _vp(sd), n, _i32(tokens), _i32(idx), _f64(gate), _f64(y))
     return y
+
+
+# ------------------------------------------------------------- FP8 experts
+
+def e4m3_decode(code: int) -> float:
+    """Value of one e4m3 code (NaN for the NaN codes)."""
+    return float(lib().orc_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_round(v: float) -> float:
+    """Nearest e4m3 value (ties to even), saturated at +-448."""
+    return float(lib().orc_e4m3_round(float(v)))
+
+
+def pow2_scale(amax: float) -> float:
+    """The smallest power of two s with 448 s >= amax (1 for amax == 0)."""
+    return float(lib().orc_pow2_scale(float(amax)))
+
+
+def quantize_rows(x):
+    """Each row divided by its power-of-two scale and rounded to e4m3:
+    (values [n, d] float64 on the e4m3 grid, scales [n])."""
+    x = _cpu(x)
+    n, d = x.shape
+    q = np.empty((n, d), np.float64)
+    sc = np.empty((n,), np.float64)
+    lib().orc_quantize_rows(n, d, _dt(x), _vp(x), _f64(q), _f64(sc))
+    return q, sc
+
+
+def _u8(t):
+    if t is None:
+        return None
+    t = _cpu(t)
+    if t.dtype != torch.uint8:
+        t = t.view(torch.uint8)
+    return t
+
+
+def fp8_moe_tokens(cfg, inp: dict, tokens, idx_in=None):
+    """Layer output (fp64) for the listed tokens with FP8 experts: ``inp`` holds
+    the e4m3 codes (w_gate8, w_up8, w_down8 and ws_*8 for shared experts, as
+    uint8 or float8_e4m3fn tensors) and their fp32 row scales (s_gate, s_up,
+    s_down, ss_*), plus x, the router and MoE++ tensors as for moe_tokens.
+    Returns (y, idx, gate, margin)."""
+    tokens = _np_i32(tokens).reshape(-1)
+    n = tokens.shape[0]
+    x = _cpu(inp["x"])
+    g = {k_: _cpu(inp.get(k_)) for k_ in ("w_router", "w_const_mix", "const_vec")}
+    codes = {k_: _u8(inp.get(k_)) for k_ in ("w_gate8", "w_up8", "w_down8", "ws_gate8", "ws_up8", "ws_down8")}
+    scales = {k_: (None if inp.get(k_) is None else _cpu(inp[k_]).to(torch.float32).contiguous())
+              for k_ in ("s_gate", "s_up", "s_down", "ss_gate", "ss_up", "ss_down")}
+    bias = inp.get("router_bias")
+    bias = None if bias is None else _cpu(bias).to(torch.float32).contiguous()
+    zp = inp.get("z_prev")
+    zp = None if zp is None else _cpu(zp).to(torch.float32).contiguous()
+    dt = _dt(x, *[v for v in g.values() if v is not None])
+    L = _Layer(T=x.shape[0], d=cfg.d, top_k=cfg.top_k, dt=dt, n_ffn=cfg.n_ffn,
+               hidden=cfg.hidden, n_shared=cfg.n_shared, hidden_shared=cfg.hidden_shared,
+               n_zero=cfg.n_zero, n_copy=cfg.n_copy, n_const=cfg.n_const)
+    k = cfg.top_k
+    y = np.empty((n, cfg.d), np.float64)
+    idx = np.empty((n, k), np.int32)
+    gate = np.empty((n, k), np.float64)
+    margin = np.empty((n,), np.float64)
+    ii = None if idx_in is None else _np_i32(idx_in).reshape(n, k)
+    lib().orc_fp8_moe_tokens(ctypes.byref(L), _vp(x), _vp(g["w_router"]), _vp(bias), _vp(zp),
+                             _vp(codes["w_gate8"]), _vp(scales["s_gate"]), _vp(codes["w_up8"]), _vp(scales["s_up"]),
+                             _vp(codes["w_down8"]), _vp(scales["s_down"]),
+                             _vp(codes["ws_gate8"]), _vp(scales["ss_gate"]), _vp(codes["ws_up8"]),
+                             _vp(scales["ss_up"]), _vp(codes["ws_down8"]), _vp(scales["ss_down"]),
+                             _vp(g["w_const_mix"]), _vp(g["const_vec"]),
+                             n, _i32(tokens), _i32(ii), _f64(y), _i32(idx), _f64(gate), _f64(margin))
+    return y, idx, gate, margin

@@ -458,3 +458,203 @@ void orc_omni_tokens(int d, int K, int dt, const void* x, const void* u, const v
         free(h);
     }
 }
+
+/* ---------------------------------------------------------- FP8 experts */
+/*
+ * "PCoMoE" summary, "Improvements", 3 (Mixed Precision Execution): the
+ * expert computation in FP8, the gating in BF16.  FP8 here is E4M3: sign, 4
+ * exponent bits (bias 7), 3 mantissa bits; largest finite value 448,
+ * smallest normal 2^-6, subnormals spaced 2^-9; the code with all exponent
+ * and mantissa bits set is NaN.
+ *   stored expert weights: an e4m3 code per element and an fp32 scale per
+ *     output row; the weight is code value * scale (read exactly here);
+ *   activations (x, then the hidden h): each row is divided by the smallest
+ *     power of two s with 448 s >= max|row| and rounded to the nearest e4m3
+ *     value (ties to even); the row is then s * codes.  A power-of-two scale
+ *     makes the division exact, so the rounding decisions are those of the
+ *     definition whatever the precision of the arithmetic;
+ *   the hidden activation is rounded to bf16 (nearest, ties to even) before
+ *     its quantization: it is stored so between the two expert GEMMs.
+ */
+
+double orc_e4m3_decode(uint8_t b)
+{
+    const int e = (b >> 3) & 15, m = b & 7;
+    const double s = (b & 0x80) ? -1.0 : 1.0;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) return s * ldexp((double)m, -9);
+    return s * ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* Nearest e4m3 value to v, ties to even mantissa; |v| >= 448 gives +-448. */
+double orc_e4m3_round(double v)
+{
+    if (v != v) return v;
+    const double a = fabs(v), sg = v < 0 ? -1.0 : 1.0;
+    if (a >= 448.0) return sg * 448.0;
+    double q;                                   /* spacing of the e4m3 values around a */
+    if (a < ldexp(1.0, -6)) {
+        q = ldexp(1.0, -9);
+    } else {
+        int ex;
+        frexp(a, &ex);                          /* a in [2^(ex-1), 2^ex) */
+        q = ldexp(1.0, ex - 1 - 3);
+    }
+    return sg * nearbyint(a / q) * q;           /* a / q exact; nearbyint: ties to even */
+}
+
+/* Nearest bf16 value to v (8 significant bits), ties to even. */
+static double bf16_round(double v)
+{
+    if (v == 0.0 || v != v || isinf(v)) return v;
+    int ex;
+    frexp(fabs(v), &ex);
+    if (ex - 1 < -126) ex = -125;               /* subnormal range: fixed spacing 2^-133 */
+    const double q = ldexp(1.0, ex - 1 - 7);
+    return nearbyint(v / q) * q;
+}
+
+/* The smallest power of two s with 448 s >= amax (1 for amax == 0). */
+double orc_pow2_scale(double amax)
+{
+    if (!(amax > 0.0)) return 1.0;
+    int ex;
+    frexp(amax, &ex);                           /* amax in [2^(ex-1), 2^ex) */
+    int e = ex - 9;                             /* 448 * 2^(ex-9) = 0.875 * 2^ex: at or near amax */
+    while (448.0 * ldexp(1.0, e) < amax) ++e;
+    while (448.0 * ldexp(1.0, e - 1) >= amax) --e;
+    return ldexp(1.0, e);
+}
+
+/* One row of n values quantized: codes (as values) q[i] and the scale. */
+static double quantize_row(const double* v, int n, double* q)
+{
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i)
+        if (fabs(v[i]) > amax) amax = fabs(v[i]);
+    const double s = orc_pow2_scale(amax);
+    for (int i = 0; i < n; ++i) q[i] = orc_e4m3_round(v[i] / s);
+    return s;
+}
+
+/* Rows of x (n rows of d, dtype dt) quantized: q [n, d] (e4m3 values), scale [n]. */
+void orc_quantize_rows(int n, int d, int dt, const void* x, double* q, double* scale)
+{
+    double* row = (double*)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
+    for (int r = 0; r < n; ++r) {
+        widen_row(x, (size_t)r, d, dt, row);
+        scale[r] = quantize_row(row, d, q + (size_t)r * d);
+    }
+    free(row);
+}
+
+/* sum_i a[i] * W[row, i] with W an e4m3 code matrix (row-major, ld = n). */
+static double dot_row_e4m3(const double* a, const uint8_t* W, size_t row, int n)
+{
+    double s = 0.0;
+    const uint8_t* w = W + row * (size_t)n;
+    for (int i = 0; i < n; ++i) s += a[i] * orc_e4m3_decode(w[i]);
+    return s;
+}
+
+/*
+ * One FP8 SwiGLU expert on one token, y += w * out:
+ *   x quantized (sx, x8);  g_i = sx sg_i (x8 . Wg8_i),  u_i = sx su_i (x8 . Wu8_i);
+ *   h_i = bf16(silu(g_i) u_i);  h quantized (sh, h8);  out_o = sh sd_o (h8 . Wd8_o).
+ * Wg8, Wu8 [H, d], Wd8 [d, H] codes; sg, su [H], sd [d] row scales.
+ */
+static void swiglu_fp8_acc(int d, int H, const uint8_t* Wg, const float* sg, const uint8_t* Wu, const float* su,
+                           const uint8_t* Wd, const float* sd, const double* x8, double sx, double w, double* y,
+                           double* h, double* h8)
+{
+    for (int i = 0; i < H; ++i) {
+        const double g = sx * (double)sg[i] * dot_row_e4m3(x8, Wg, (size_t)i, d);
+        const double u = sx * (double)su[i] * dot_row_e4m3(x8, Wu, (size_t)i, d);
+        h[i] = bf16_round(silu(g) * u);
+    }
+    const double sh = quantize_row(h, H, h8);
+    for (int o = 0; o < d; ++o) y[o] += w * sh * (double)sd[o] * dot_row_e4m3(h8, Wd, (size_t)o, H);
+}
+
+/*
+ * The layer output for the listed tokens with FP8 experts: routing, zero /
+ * copy / constant experts and the combine exactly as orc_moe_tokens (bf16
+ * or fp32 x, router and MoE++ tensors of type L->dt); every FFN and shared
+ * expert is swiglu_fp8_acc with its codes and row scales (routed [n_ffn, ...],
+ * shared [n_shared, ...]).
+ */
+void orc_fp8_moe_tokens(const orc_layer* L, const void* x, const void* w_router, const float* bias,
+                        const float* zprev, const uint8_t* wg8, const float* sg, const uint8_t* wu8,
+                        const float* su, const uint8_t* wd8, const float* sd, const uint8_t* sg8,
+                        const float* ssg, const uint8_t* su8, const float* ssu, const uint8_t* sd8,
+                        const float* ssd, const void* w_const_mix, const void* const_vec, int n_tok,
+                        const int32_t* tokens, const int32_t* idx_in, double* y, int32_t* idx, double* gate,
+                        double* margin)
+{
+    const int d = L->d, k = L->top_k, H = L->hidden, Hs = L->hidden_shared;
+    const int E = L->n_ffn + L->n_zero + L->n_copy + L->n_const;
+    const int zero0 = L->n_ffn, copy0 = zero0 + L->n_zero, const0 = copy0 + L->n_copy;
+    const int hmax = H > Hs ? H : Hs;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < n_tok; ++n) {
+        const int t = tokens[n];
+        double* xt = (double*)malloc(sizeof(double) * (size_t)d);
+        double* x8 = (double*)malloc(sizeof(double) * (size_t)d);
+        double* z = (double*)malloc(sizeof(double) * (size_t)E);
+        double* h = (double*)malloc(sizeof(double) * (size_t)(hmax > 0 ? hmax : 1));
+        double* h8 = (double*)malloc(sizeof(double) * (size_t)(hmax > 0 ? hmax : 1));
+        unsigned char* taken = (unsigned char*)malloc((size_t)E);
+        double* yt = y + (size_t)n * d;
+        int32_t* it = idx + (size_t)n * k;
+        double* gt = gate + (size_t)n * k;
+        widen_row(x, (size_t)t, d, L->dt, xt);
+        for (int e = 0; e < E; ++e) {
+            z[e] = dot_row(xt, w_router, (size_t)e, d, L->dt);
+            if (bias) z[e] += (double)bias[e];
+            if (zprev) z[e] += (double)zprev[(size_t)t * E + e];
+        }
+        if (idx_in) {
+            double zmax = -INFINITY, s = 0.0;
+            for (int j = 0; j < k; ++j) {
+                it[j] = idx_in[(size_t)n * k + j];
+                if (z[it[j]] > zmax) zmax = z[it[j]];
+            }
+            for (int j = 0; j < k; ++j) s += exp(z[it[j]] - zmax);
+            for (int j = 0; j < k; ++j) gt[j] = exp(z[it[j]] - zmax) / s;
+            if (margin) margin[n] = NAN;
+        } else {
+            topk_one(E, k, z, it, gt, margin ? margin + n : NULL, taken);
+        }
+        const double sx = quantize_row(xt, d, x8);
+        for (int o = 0; o < d; ++o) yt[o] = 0.0;
+        for (int s = 0; s < L->n_shared; ++s) {
+            const size_t wo = (size_t)s * Hs * d;
+            swiglu_fp8_acc(d, Hs, sg8 + wo, ssg + (size_t)s * Hs, su8 + wo, ssu + (size_t)s * Hs, sd8 + wo,
+                           ssd + (size_t)s * d, x8, sx, 1.0, yt, h, h8);
+        }
+        for (int j = 0; j < k; ++j) {
+            const int e = it[j];
+            const double g = gt[j];
+            if (e < zero0) {
+                const size_t wo = (size_t)e * H * d;
+                swiglu_fp8_acc(d, H, wg8 + wo, sg + (size_t)e * H, wu8 + wo, su + (size_t)e * H, wd8 + wo,
+                               sd + (size_t)e * d, x8, sx, g, yt, h, h8);
+            } else if (e < copy0) {
+                /* zero expert: contributes nothing */
+            } else if (e < const0) {
+                for (int o = 0; o < d; ++o) yt[o] += g * xt[o];
+            } else {
+                const int c = e - const0;
+                double l0 = dot_row(xt, w_const_mix, (size_t)(2 * c), d, L->dt);
+                double l1 = dot_row(xt, w_const_mix, (size_t)(2 * c + 1), d, L->dt);
+                double m = l0 > l1 ? l0 : l1;
+                double a1 = exp(l0 - m), a2 = exp(l1 - m), sa = a1 + a2;
+                a1 /= sa;
+                a2 /= sa;
+                for (int o = 0; o < d; ++o)
+                    yt[o] += g * (a1 * xt[o] + a2 * ld(const_vec, (size_t)c * d + o, L->dt));
+            }
+        }
+        free(xt); free(x8); free(z); free(h); free(h8); free(taken);
+    }
+}
