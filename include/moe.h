@@ -97,6 +97,17 @@ typedef struct moe_layer_desc {
     int32_t out_f32;       /* 0: y is `dtype`; 1: y is fp32 (the fp32 combine     *
                             * before its final rounding; the dtype output is its *
                             * round-to-nearest-even)                              */
+    int32_t expert_fp8;    /* 1: FP8 experts ("PCoMoE" summary, Improvements 3,  *
+                            * Mixed Precision Execution): the SwiGLU experts'     *
+                            * weights are e4m3 codes with an fp32 scale per      *
+                            * output row (moe_layer_weights s_*), the expert     *
+                            * GEMMs run on e4m3 activations (each row divided by *
+                            * the smallest power of two s with 448 s >= its      *
+                            * max |value| and rounded to nearest, s kept); the  *
+                            * router and the combine stay in `dtype` (bf16,     *
+                            * required), as do h between its rounding to bf16   *
+                            * and its quantization.  d_model a multiple of 256, *
+                            * hidden of 128.  0: weights in `dtype`.             */
 } moe_layer_desc;
 
 /* Device pointers to the layer's parameters (NULL where the layer has none). */
@@ -116,6 +127,14 @@ typedef struct moe_layer_weights {
     const void* subkeys_col;  /* atomic: [pk_cols, d_query / 2]                          */
     const void* u;            /* atomic: [pk_rows * pk_cols, d_model] input vectors      */
     const void* v;            /* atomic: [pk_rows * pk_cols, d_model] output vectors     */
+    /* expert_fp8: w_gate, w_up, w_down (and ws_*) hold e4m3 codes; these are
+     * the fp32 scales of their rows (the weight is code * scale):            */
+    const float* s_gate;      /* [n_ffn, hidden]                                         */
+    const float* s_up;        /* [n_ffn, hidden]                                         */
+    const float* s_down;      /* [n_ffn, d_model]                                        */
+    const float* ss_gate;     /* [n_shared, hidden_shared]                               */
+    const float* ss_up;       /* [n_shared, hidden_shared]                               */
+    const float* ss_down;     /* [n_shared, d_model]                                     */
 } moe_layer_weights;
 
 /* Number of expert groups of the grouped step: n_ffn + n_shared (SwiGLU) or
@@ -167,7 +186,9 @@ MOE_API moe_status moe_route(const moe_layer_desc* desc, const moe_layer_weights
  * row_of [T*top_k]: row of slot (t, j), -1 for a zero-computation expert.
  * token_of [row capacity]: SwiGLU: token of each row; atomic: flat slot id
  *   t*top_k + j of each task.
- * x_sorted [row capacity, d_model]: SwiGLU only, x_sorted[r] = x[token_of[r]];
+ * x_sorted [row capacity, d_model]: SwiGLU only, x_sorted[r] = x[token_of[r]]
+ *   (expert_fp8: the rows' e4m3 codes [row capacity, d_model] bytes, then at
+ *   byte offset align256(capacity * d_model) their fp32 scales [row capacity]);
  *   NULL for the atomic kind, and may be NULL for the SwiGLU kind (no copy
  *   made) when the fused expert step gathers the rows itself.  Rows past
  *   expert_offsets[groups] are untouched.

@@ -37,13 +37,14 @@ class MoEError(RuntimeError):
 class MoELayerDesc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "T", "d_model", "top_k", "dtype", "kind", "n_ffn", "hidden", "n_shared", "hidden_shared",
-        "n_zero", "n_copy", "n_const", "pk_rows", "pk_cols", "pk_topk_half", "d_query", "out_f32")]
+        "n_zero", "n_copy", "n_const", "pk_rows", "pk_cols", "pk_topk_half", "d_query", "out_f32", "expert_fp8")]
 
 
 class MoELayerWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_router", "router_bias", "w_const_mix", "const_vec", "w_gate", "w_up", "w_down",
-        "ws_gate", "ws_up", "ws_down", "w_query", "subkeys_row", "subkeys_col", "u", "v")]
+        "ws_gate", "ws_up", "ws_down", "w_query", "subkeys_row", "subkeys_col", "u", "v",
+        "s_gate", "s_up", "s_down", "ss_gate", "ss_up", "ss_down")]
 
 
 _lib = None

@@ -77,6 +77,12 @@ struct DevArgs {
     const int32_t* idx;         // [rows_T, k] routing (gate lookup of the scatter-add epilogue)
     const float* gate;          // [rows_T, k]
     int k;
+    // e4m3 operands (token-column form): out = acc * sa[weight row] * sb[token row]
+    const float* sa0;           // row scales of B0 (gate / down), B1 (up), B2, B3 (shared experts)
+    const float* sa1;
+    const float* sa2;
+    const float* sa3;
+    const float* sb;            // [rows] row scales of the token-row operand
 };
 
 struct TileInfo {
@@ -829,7 +835,9 @@ __device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body)
 // its token with vector atomics).
 enum TnMode { TN_PLAIN = 0, TN_GATHER = 1, TN_SCATTER_ADD = 2, TN_ZERO_ACC = 4 };
 
-template <int EPI, int MODE>
+// FP8: both operands e4m3 (kind::f8f6f4); a 128-byte box row holds 128
+// elements of K instead of 64, and the epilogue applies the row scales.
+template <int EPI, int MODE, bool FP8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW0,
                        const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
@@ -838,8 +846,10 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "token-column form: SwiGLU or fp32 epilogue");
     static_assert(MODE == TN_PLAIN || (EPI == EPI_SWIGLU && (MODE == TN_ZERO_ACC || MODE == (TN_GATHER | TN_ZERO_ACC))) ||
                   (EPI == EPI_F32 && MODE == TN_SCATTER_ADD), "fused modes: gather / zeroing with SwiGLU, scatter-add with fp32");
+    static_assert(!FP8 || MODE == TN_PLAIN, "e4m3 operands: the plain form");
     constexpr bool GATHER = (MODE & TN_GATHER) != 0;
     constexpr bool ZERO_ACC = (MODE & TN_ZERO_ACC) != 0;
+    constexpr int BKE = FP8 ? 2 * BK : BK;        // K elements per 128-byte box row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -881,7 +891,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
 
     const uint32_t tmem_base = *tmem_slot;
     const int total = tile_start[a.n_groups];
-    const int pnk = cdiv(a.K, BK * P_KH);
+    const int pnk = cdiv(a.K, BKE * P_KH);
     const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     const uint32_t full_leader = mapa_shared(smem_u32(&full[0]), 0);
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
@@ -928,7 +938,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                         mbar_arrive_expect_tx(&full[s], GATHER ? 2 * P_KH * (P_HALF + half_n * 128) : 2 * P_STAGE_BYTES);
 #pragma unroll
                     for (int h = 0; h < P_KH; ++h) {
-                        const int k0 = (kb * P_KH + h) * BK;      // past K: zero fill
+                        const int k0 = (kb * P_KH + h) * BKE;     // past K: zero fill
                         uint8_t* da = sA + s * P_TILE_A + h * P_HALF;
                         uint8_t* db = sB + s * P_TILE_B + h * P_HALF;
                         if (lane == 0) {
@@ -964,7 +974,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
                 const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
-                const uint32_t idesc = idesc_bf16_f32(P_BM, ti.nt);
+                const uint32_t idesc = FP8 ? idesc_e4m3_f32(P_BM, ti.nt) : idesc_bf16_f32(P_BM, ti.nt);
                 if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
@@ -972,12 +982,18 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                     if (!mbar_wait(&full[s], ph)) { *abort_flag = 1; bad = true; break; }
                     const uint64_t ad = ad0 + (uint64_t)((s * P_TILE_A) >> 4);
                     const uint64_t bd = bd0 + (uint64_t)((s * P_TILE_B) >> 4);
+                    // four 32-byte K steps per 128-byte row (16 bf16 or 32 e4m3 elements each)
 #pragma unroll
                     for (int h = 0; h < P_KH; ++h)
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            tc_mma_bf16_pair(d_tmem, ad + (h * P_HALF >> 4) + 2 * kk, bd + (h * P_HALF >> 4) + 2 * kk,
-                                             idesc, (kb | h | kk) != 0);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            if constexpr (FP8)
+                                tc_mma_e4m3_pair(d_tmem, ad + (h * P_HALF >> 4) + 2 * kk,
+                                                 bd + (h * P_HALF >> 4) + 2 * kk, idesc, (kb | h | kk) != 0);
+                            else
+                                tc_mma_bf16_pair(d_tmem, ad + (h * P_HALF >> 4) + 2 * kk,
+                                                 bd + (h * P_HALF >> 4) + 2 * kk, idesc, (kb | h | kk) != 0);
+                        }
                     tc_commit_pair(&empty[s], 0x3);
                     if (++s == P_STAGES) { s = 0; ph ^= 1; }
                 }
@@ -1012,10 +1028,24 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                 float* out = reinterpret_cast<float*>(a.out);
                 float* stg = mine;                        // [32 tokens][32 features]
                 const int f0 = ti.m * 256 + (int)rank * 128 + q * 32;
+                float s_lane = 1.f;                       // e4m3: this lane's weight-row scale
+                if constexpr (FP8) {
+                    const bool first = ti.g < a.n_first;
+                    const int gb = first ? ti.g : ti.g - a.n_first;
+                    s_lane = (first ? a.sa0 : a.sa2)[(long long)gb * a.N + f0 + lane];
+                }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     __syncwarp();                         // the previous chunk has been read
+                    if constexpr (FP8) {                  // out = acc * s_weight_row * s_token_row
+                        const int cl = ch * 32 + lane;
+                        const float sl = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = __uint_as_float(v[i]);
+                        for (int i = 0; i < 32; ++i)
+                            stg[i * 32 + lane] = __uint_as_float(v[i]) * s_lane * __shfl_sync(0xffffffffu, sl, i);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = __uint_as_float(v[i]);
+                    }
                     __syncwarp();
                     if constexpr (MODE == TN_SCATTER_ADD) {
                         // lane l: the token of row ch * 32 + l and its gate for this group's expert
@@ -1076,22 +1106,40 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                                 *reinterpret_cast<const uint4*>(stg + row * 32 + piece * 8);
                     }
                 };
+                float s_lane = 1.f;                       // e4m3: this lane's gate or up row scale
+                if constexpr (FP8) {
+                    const bool first = ti.g < a.n_first;
+                    const int gb = first ? ti.g : ti.g - a.n_first;
+                    const float* sa = gate_warp ? (first ? a.sa0 : a.sa2) : (first ? a.sa1 : a.sa3);
+                    s_lane = sa[(long long)gb * a.N + unit0 + lane];
+                }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     team_sync(team);                      // the partner has read the previous chunk
+                    float vv[32];                         // (e4m3: acc * s_weight_row * s_token_row)
+                    if constexpr (FP8) {
+                        const int cl = ch * 32 + lane;
+                        const float sl = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            vv[i] = __uint_as_float(v[i]) * s_lane * __shfl_sync(0xffffffffu, sl, i);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) vv[i] = __uint_as_float(v[i]);
+                    }
                     float g[16], u[16];
                     if (gate_warp) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = __uint_as_float(v[16 + i]);
+                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = vv[16 + i];
                         team_sync(team);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) { g[i] = __uint_as_float(v[i]); u[i] = theirs[i * 32 + lane]; }
+                        for (int i = 0; i < 16; ++i) { g[i] = vv[i]; u[i] = theirs[i * 32 + lane]; }
                         finish(g, u, ch * 32);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = __uint_as_float(v[i]);
+                        for (int i = 0; i < 16; ++i) mine[i * 32 + lane] = vv[i];
                         team_sync(team);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) { g[i] = theirs[i * 32 + lane]; u[i] = __uint_as_float(v[16 + i]); }
+                        for (int i = 0; i < 16; ++i) { g[i] = theirs[i * 32 + lane]; u[i] = vv[16 + i]; }
                         finish(g, u, ch * 32 + 16);
                     }
                 });
@@ -1147,19 +1195,22 @@ EncodeTiledFn get_encode()
     return fn;
 }
 
-// bf16 [rows, K] row-major, box {64 (K), box_rows}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows = 128)
+// bf16 [rows, K] row-major, box {64 (K), box_rows}, 128-byte swizzle; or
+// (e4m3) bytes [rows, K], box {128 (K), box_rows}: 128-byte box rows either way.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows = 128, bool e4m3 = false)
 {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
     if (rows <= 0 || base == nullptr) {   // unused operand: point at something valid
         rows = 128;
     }
+    const int esz = e4m3 ? 1 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * esz};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+    CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -1204,6 +1255,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
                      (EPI == EPI_F32 && p.N % 256 == 0));
     // fuse: 1 = gathered B rows + zeroing, 3 = zeroing (B from x_sorted) -- SwiGLU; 2 = scatter-add -- fp32
     const bool swiglu_fuse = p.fuse == 1 || p.fuse == 3;
+    if (p.fp8 && (!tn || p.fuse || p.K % 128 != 0 || !p.sb || !p.sa0 || (EPI == EPI_SWIGLU && !p.sa1) ||
+                  (p.n_first < p.n_groups && (!p.sa2 || (EPI == EPI_SWIGLU && !p.sa3)))))
+        return MOE_ERR_UNSUPPORTED;
     if (p.fuse && (!tn || swiglu_fuse != (EPI == EPI_SWIGLU) || (p.fuse == 2) != (EPI == EPI_F32) ||
                    !p.rows || !p.acc || p.acc_d % 256 != 0 || p.rows_T <= 0 ||
                    (p.fuse == 1 && p.K % (BK * P_KH) != 0) || (p.fuse == 2 && (!p.idx || !p.gate || p.k <= 0)) ||
@@ -1211,10 +1265,12 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
         return MOE_ERR_UNSUPPORTED;
     const int wbox = (tn && EPI == EPI_SWIGLU) ? 64 : 128;
     // gathered rows: x itself, one-row boxes (tile::gather4 loads)
-    const bool mapA_ok = p.fuse == 1 ? make_map(&mA, p.A, p.rows_T, p.K, 1) : make_map(&mA, p.A, p.a_rows, p.K);
-    if (!mapA_ok || !make_map(&m0, p.B0, p.b01_rows, kb, wbox) ||
-        !make_map(&m1, b1, p.b01_rows, kb, wbox) || !make_map(&m2, b2, r23, kb, wbox) ||
-        !make_map(&m3, b3, r23, kb, wbox))
+    const bool f8 = p.fp8 != 0;
+    const bool mapA_ok = p.fuse == 1 ? make_map(&mA, p.A, p.rows_T, p.K, 1)
+                                     : make_map(&mA, p.A, p.a_rows, p.K, 128, f8);
+    if (!mapA_ok || !make_map(&m0, p.B0, p.b01_rows, kb, wbox, f8) ||
+        !make_map(&m1, b1, p.b01_rows, kb, wbox, f8) || !make_map(&m2, b2, r23, kb, wbox, f8) ||
+        !make_map(&m3, b3, r23, kb, wbox, f8))
         return MOE_ERR_CUDA;
     if (EPI == EPI_PK_SPLIT) mo = mA;   // direct stores; the map is unused
     else if (!make_out_map(&mo, p.out, std::min<long long>(p.rows_cap, 1ll << 31), p.N, p.ldo, EPI == EPI_F32))
@@ -1239,6 +1295,11 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     a.idx = p.idx;
     a.gate = p.gate;
     a.k = p.k;
+    a.sa0 = p.sa0;
+    a.sa1 = p.sa1;
+    a.sa2 = p.sa2;
+    a.sa3 = p.sa3;
+    a.sb = p.sb;
     const int ntn = (EPI == EPI_SWIGLU) ? cdiv(p.N, 128) : cdiv(p.N, 256);
     const long long rows = std::min<long long>(p.rows_cap, 1ll << 30);
     if constexpr (EPI == EPI_SWIGLU || EPI == EPI_F32) {
@@ -1253,6 +1314,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
                 count_launch();
                 return cuda_status(cudaGetLastError());
             };
+            if (p.fp8) return go(grouped_gemm_tn_kernel<EPI, TN_PLAIN, true>);
             if constexpr (EPI == EPI_SWIGLU) {
                 if (p.fuse == 1) return go(grouped_gemm_tn_kernel<EPI, TN_GATHER | TN_ZERO_ACC>);
                 if (p.fuse == 3) return go(grouped_gemm_tn_kernel<EPI, TN_ZERO_ACC>);
@@ -1261,7 +1323,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
             }
             return go(grouped_gemm_tn_kernel<EPI, TN_PLAIN>);
         }
-    } else if (p.fuse) {
+    } else if (p.fuse || p.fp8) {
         return MOE_ERR_UNSUPPORTED;
     }
     if (p.pair) {

@@ -68,6 +68,15 @@ struct GemmProblem {
     const int32_t* idx;
     const float* gate;
     int k;
+    // e4m3 operands (token-column pair form only; else MOE_ERR_UNSUPPORTED): A and B hold
+    // e4m3 codes, K a multiple of 128; out = acc * sa[weight row] * sb[token row], with
+    // sa0 / sa1 the row scales of B0 / B1 and sa2 / sa3 those of B2 / B3.
+    int fp8;
+    const float* sa0;
+    const float* sa1;
+    const float* sa2;
+    const float* sa3;
+    const float* sb;
 };
 
 moe_status launch_grouped_gemm(const GemmProblem& p, cudaStream_t st);
@@ -110,11 +119,20 @@ struct PermuteArgs {
     int32_t* ws_counts;   // [n_blocks, n_ffn] (SwiGLU) or [N] (atomic)
     int32_t* ws_blocksum; // atomic scan: [scan blocks]
     int T, k, d, n_ffn, n_shared, n_ids, elt_bytes;
+    float* xs_scale;      // non-null: x_sorted gets e4m3 codes of the rows and these their scales
 };
 moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st);
 moe_status launch_permute_atomic(const PermuteArgs& a, cudaStream_t st);
 int permute_blocks(int T);
 int atomic_scan_blocks(int N);
+
+// ------------------------------------------------------------ e4m3 activations
+// codes[r] = e4m3(x[token_of[r]] / scale[r]) for r < offsets[n_last] (x bf16 [T, d], d % 256 == 0)
+moe_status launch_gather_quant(const int32_t* token_of, const int32_t* offsets, int n_last, const void* x, int d,
+                               int T, void* codes, float* scale, long long rows_cap, cudaStream_t st);
+// codes[r] = e4m3(h[r] / scale[r]) for r < offsets[n_last] (h bf16 [rows, H])
+moe_status launch_quant_rows(const void* h, const int32_t* offsets, int n_last, int H, void* codes, float* scale,
+                             long long rows_cap, cudaStream_t st);
 
 // ------------------------------------------------------------ experts
 struct FfnF32Args {

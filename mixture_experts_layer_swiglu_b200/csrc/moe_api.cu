@@ -64,6 +64,10 @@ moe_status check_desc(const moe_layer_desc* d)
     if (d->T < 0 || d->d_model <= 0 || d->top_k <= 0) return MOE_ERR_INVALID_ARG;
     if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (d->out_f32 != 0 && d->out_f32 != 1) return MOE_ERR_INVALID_ARG;
+    if (d->expert_fp8 != 0 && d->expert_fp8 != 1) return MOE_ERR_INVALID_ARG;
+    if (d->expert_fp8 && (d->kind != MOE_EXPERT_SWIGLU || d->dtype != MOE_BF16 || d->d_model % 256 != 0 ||
+                          (d->n_ffn + d->n_shared > 0 && d->hidden % 128 != 0)))
+        return MOE_ERR_UNSUPPORTED;
     if (d->kind == MOE_EXPERT_SWIGLU) {
         if (d->n_ffn < 0 || d->n_shared < 0 || d->n_zero < 0 || d->n_copy < 0 || d->n_const < 0)
             return MOE_ERR_INVALID_ARG;
@@ -120,6 +124,8 @@ Scratch scratch_sizes(const moe_layer_desc* d)
     if (d->kind == MOE_EXPERT_SWIGLU) {
         s.permute = al((size_t)permute_blocks(d->T) * std::max(d->n_ffn, 1) * 4);
         s.ffn = (d->n_ffn + d->n_shared > 0) ? al((size_t)cap * d->hidden * elt(d)) : 0;
+        if (d->expert_fp8 && s.ffn)   // h (bf16), then its e4m3 codes and row scales
+            s.ffn += al((size_t)cap * d->hidden) + al((size_t)cap * 4);
     } else {
         const size_t half = d->d_query / 2;
         s.route = al((size_t)2 * d->T * 3 * half * 2) + al((size_t)(d->pk_rows + d->pk_cols) * 3 * half * 2) +
@@ -147,7 +153,7 @@ size_t scratch_max(const moe_layer_desc* d)
 // order the atomics land in.
 bool fused_eligible(const moe_layer_desc* d)
 {
-    return d->kind == MOE_EXPERT_SWIGLU && d->dtype == MOE_BF16 && d->n_ffn > 0 && d->n_shared == 0 &&
+    return d->kind == MOE_EXPERT_SWIGLU && d->dtype == MOE_BF16 && !d->expert_fp8 && d->n_ffn > 0 && d->n_shared == 0 &&
            d->top_k <= 2 && d->d_model % 256 == 0 && d->hidden % 128 == 0;
 }
 
@@ -196,7 +202,8 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
         b.xs = take((size_t)cap * d->d_model * elt(d));
         b.ys = nullptr;   // the fused step combines into its own accumulator
     } else if (d->kind == MOE_EXPERT_SWIGLU) {
-        b.xs = take((size_t)cap * d->d_model * elt(d));
+        // (FP8 experts: the rows' e4m3 codes, then their fp32 scales)
+        b.xs = take(d->expert_fp8 ? al((size_t)cap * d->d_model) + (size_t)cap * 4 : (size_t)cap * d->d_model * elt(d));
         b.ys = take((size_t)cap * d->d_model * 4);
     } else {
         b.xs = nullptr;
@@ -338,6 +345,8 @@ moe_status permute_impl(const moe_layer_desc* d, const int32_t* idx, const void*
     a.elt_bytes = elt(d);
     if (d->kind == MOE_EXPERT_SWIGLU) {
         if (xs && (!x || !aligned16(x) || !aligned16(xs))) return MOE_ERR_INVALID_ARG;
+        if (xs && d->expert_fp8)   // e4m3 codes of the rows, then their scales
+            a.xs_scale = reinterpret_cast<float*>(static_cast<char*>(xs) + al((size_t)moe_row_capacity(d) * d->d_model));
         a.ws_counts = static_cast<int32_t*>(ws);
         a.n_ffn = d->n_ffn;
         a.n_shared = d->n_shared;
@@ -403,6 +412,68 @@ moe_status atomic_shared_phase(const moe_layer_desc* d, const moe_layer_weights*
     return launch_grouped_gemm(g, st);
 }
 
+// The SwiGLU step with FP8 experts.  Phase 1: h = SwiGLU on the e4m3 rows of
+// x_sorted (epilogue: acc * weight-row scale * row scale), h rounded to bf16,
+// then each h row quantized to e4m3 with its power-of-two scale.  Phase 2:
+// y_sorted = (h8 W_down8^T) * weight-row scale * row scale.  Workspace: h
+// [cap, H] bf16, h8 [cap, H], s_h [cap].
+moe_status ffn_phase_fp8(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* xs,
+                         const int32_t* offsets, void* ys, void* ws, long long cap, cudaStream_t st)
+{
+    if ((d->n_ffn && (!w->s_gate || !w->s_up || !w->s_down)) ||
+        (d->n_shared && (!w->ss_gate || !w->ss_up || !w->ss_down)))
+        return MOE_ERR_INVALID_ARG;
+    char* h = static_cast<char*>(ws);
+    char* h8 = h + al((size_t)cap * d->hidden * 2);
+    float* s_h = reinterpret_cast<float*>(h8 + al((size_t)cap * d->hidden));
+    const float* s_x = reinterpret_cast<const float*>(static_cast<const char*>(xs) + al((size_t)cap * d->d_model));
+    GemmProblem g{};
+    g.offsets = offsets;
+    g.n_groups = d->n_ffn + d->n_shared;
+    g.n_first = d->n_ffn;
+    g.rows_cap = cap;
+    g.pair = 1;
+    g.tn_any = 1;
+    g.fp8 = 1;
+    g.a_rows = cap;
+    if (phase == 1) {
+        g.epi = EPI_SWIGLU;
+        g.A = xs;
+        g.K = d->d_model;
+        g.B0 = d->n_ffn ? w->w_gate : w->ws_gate;
+        g.B1 = d->n_ffn ? w->w_up : w->ws_up;
+        g.sa0 = d->n_ffn ? w->s_gate : w->ss_gate;
+        g.sa1 = d->n_ffn ? w->s_up : w->ss_up;
+        g.b01_rows = (long long)std::max(d->n_ffn, 1) * d->hidden;
+        g.B2 = w->ws_gate;
+        g.B3 = w->ws_up;
+        g.sa2 = w->ss_gate;
+        g.sa3 = w->ss_up;
+        g.b23_rows = (long long)d->n_shared * d->hidden;
+        g.N = d->hidden;
+        g.sb = s_x;
+        g.out = h;
+        g.ldo = d->hidden;
+        moe_status s = launch_grouped_gemm(g, st);
+        if (s != MOE_OK) return s;
+        return launch_quant_rows(h, offsets, d->n_ffn + d->n_shared, d->hidden, h8, s_h, cap, st);
+    }
+    g.epi = EPI_F32;
+    g.A = h8;
+    g.K = d->hidden;
+    g.B0 = d->n_ffn ? w->w_down : w->ws_down;
+    g.sa0 = d->n_ffn ? w->s_down : w->ss_down;
+    g.b01_rows = (long long)std::max(d->n_ffn, 1) * d->d_model;
+    g.B2 = w->ws_down;
+    g.sa2 = w->ss_down;
+    g.b23_rows = (long long)d->n_shared * d->d_model;
+    g.N = d->d_model;
+    g.sb = s_h;
+    g.out = ys;
+    g.ldo = d->d_model;
+    return launch_grouped_gemm(g, st);
+}
+
 moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, int phase, const void* xs,
                           const int32_t* offsets, void* ys, void* ws, size_t ws_bytes, cudaStream_t st)
 {
@@ -434,6 +505,7 @@ moe_status ffn_phase_impl(const moe_layer_desc* d, const moe_layer_weights* w, i
     const void* ptrs[8] = {xs, ys, w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (d->expert_fp8) return ffn_phase_fp8(d, w, phase, xs, offsets, ys, ws, cap, st);
     GemmProblem g{};
     g.offsets = offsets;
     g.n_groups = d->n_ffn + d->n_shared;

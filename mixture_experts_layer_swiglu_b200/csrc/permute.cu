@@ -307,7 +307,12 @@ moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
     if (a.T > 0) {
         perm_scatter_kernel<<<nb, P_TOK, 0, st>>>(a);
         count_launch();
-        if (a.x_sorted) {
+        if (a.x_sorted && a.xs_scale) {   // e4m3 codes of the rows and their scales
+            const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
+            moe_status s = launch_gather_quant(a.token_of, a.offsets, a.n_ffn + a.n_shared, a.x, a.d, a.T, a.x_sorted,
+                                               a.xs_scale, rows_cap, st);
+            if (s != MOE_OK) return s;
+        } else if (a.x_sorted) {
             const int vecs = a.d * a.elt_bytes / 16;
             const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
             const int grid = (int)std::max<long long>(1, std::min<long long>((rows_cap + 7) / 8, num_sms() * 16));

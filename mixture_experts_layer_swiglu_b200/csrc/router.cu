@@ -455,14 +455,14 @@ __host__ __device__ inline RsLayout rs_layout(int R, int d)
     RsLayout L;
     const int part = rs_partial_bytes(R);
     const int wbytes = ((R * rs_wpitch(d)) + 127) & ~127;
-    const int fixed = part + 2 * RS_MAXSTAGES * 8 + 16;
+    const int fixed = part + (2 * RS_MAXSTAGES + 1) * 8 + 16;
     L.w_smem = RS_SMEM_LIMIT - fixed - wbytes >= 3 * RS_STAGE;
     const int avail = RS_SMEM_LIMIT - fixed - (L.w_smem ? wbytes : 0);
     L.stages = avail / RS_STAGE < RS_MAXSTAGES ? avail / RS_STAGE : RS_MAXSTAGES;
     L.w_off = L.stages * RS_STAGE;
     L.z_off = L.w_off + (L.w_smem ? wbytes : 0);
     L.bar_off = L.z_off + part;
-    L.bytes = L.bar_off + 2 * RS_MAXSTAGES * 8 + 16;
+    L.bytes = L.bar_off + (2 * RS_MAXSTAGES + 1) * 8 + 16;
     return L;
 }
 
@@ -482,7 +482,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
     float* zsum = zpart + (size_t)RS_WARPS * 16 * zpitch;                   // [16][zpitch]
     uint64_t* full = reinterpret_cast<uint64_t*>(rs_smem + L.bar_off);
     uint64_t* empty = full + RS_MAXSTAGES;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + RS_MAXSTAGES);
+    uint64_t* wbar = empty + RS_MAXSTAGES;                                  // router rows landed
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(wbar + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t rowb = (size_t)a.d * 2;
     const int wpitch = rs_wpitch(a.d);
@@ -493,6 +494,7 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], RS_WARPS); }
+        mbar_init(wbar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -500,6 +502,16 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
 
     if (warp == RS_WARPS) {
         // ---------------------------------------------------- producer warp
+        // first the router rows (then the mixing rows) into shared memory, one
+        // bulk copy per row, landing while the first x chunks are in flight
+        if (L.w_smem) {
+            if (lane == 0) mbar_arrive_expect_tx(wbar, (uint32_t)(R * a.d * 2));
+            __syncwarp();
+            for (int j = lane; j < R; j += 32) {
+                const unsigned char* src = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
+                bulk_g2s(wsm + (size_t)j * wpitch, src, (uint32_t)(a.d * 2), wbar);
+            }
+        }
         // lanes 0..15 each copy one token row of a chunk; lane 0 arms the stage
         const unsigned char* xb = static_cast<const unsigned char*>(a.x);
         int s = 0;
@@ -524,29 +536,21 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
             }
         }
         // copies still in flight land before the block may exit
-        if (lane == 0)
+        if (lane == 0) {
             for (int i = 0; i < stages; ++i)
                 if ((pend >> i) & 1u) mbar_wait(&full[i], (pend_ph >> i) & 1u);
+            if (L.w_smem) mbar_wait(wbar, 0);
+        }
         return;
     }
 
     // -------------------------------------------------------- consumer warps
-    if (L.w_smem) {   // router rows (then mixing rows) into shared memory, once
-        const int vpr = a.d / 8;                                  // 16-byte vectors per row
-        for (int i = threadIdx.x; i < R * vpr; i += RS_WARPS * 32) {
-            const int j = i / vpr, v = i - j * vpr;
-            const unsigned char* src = j < a.E_r ? wr + (size_t)j * rowb : wc + (size_t)(j - a.E_r) * rowb;
-            *reinterpret_cast<uint4*>(wsm + (size_t)j * wpitch + v * 16) =
-                __ldg(reinterpret_cast<const uint4*>(src) + v);
-        }
-        rs_consumer_sync();
-    }
+    bool ok = !L.w_smem || __all_sync(FULL, mbar_wait(wbar, 0));   // the router rows are in shared memory
     const int g = lane >> 2, q = lane & 3;
     float* zw = zpart + (size_t)warp * 16 * zpitch;
     const uint32_t ring_s = smem_u32(ring), wsm_s = smem_u32(wsm);
     int s = 0;
     uint32_t ph = 0;
-    bool ok = true;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int t0 = tile * 16;
         float acc[NT][4];

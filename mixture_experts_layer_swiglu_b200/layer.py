@@ -17,13 +17,13 @@ _TORCH_DT = {abi.MOE_F32: torch.float32, abi.MOE_BF16: torch.bfloat16}
 def make_desc(T: int, d_model: int, top_k: int, dtype="bf16", kind: str = "swiglu", n_ffn: int = 0,
               hidden: int = 0, n_shared: int = 0, hidden_shared: int = 0, n_zero: int = 0, n_copy: int = 0,
               n_const: int = 0, pk_rows: int = 0, pk_cols: int = 0, pk_topk_half: int = 0,
-              d_query: int = 0, out_f32: bool = False) -> abi.MoELayerDesc:
+              d_query: int = 0, out_f32: bool = False, expert_fp8: bool = False) -> abi.MoELayerDesc:
     return abi.MoELayerDesc(
         T=T, d_model=d_model, top_k=top_k, dtype=_DT[dtype],
         kind=abi.MOE_EXPERT_SWIGLU if kind == "swiglu" else abi.MOE_EXPERT_ATOMIC_GELU,
         n_ffn=n_ffn, hidden=hidden, n_shared=n_shared, hidden_shared=hidden_shared, n_zero=n_zero,
         n_copy=n_copy, n_const=n_const, pk_rows=pk_rows, pk_cols=pk_cols, pk_topk_half=pk_topk_half,
-        d_query=d_query, out_f32=int(bool(out_f32)))
+        d_query=d_query, out_f32=int(bool(out_f32)), expert_fp8=int(bool(expert_fp8)))
 
 
 def desc_from(cfg, T: int | None = None, out_f32: bool = False) -> abi.MoELayerDesc:
@@ -33,7 +33,8 @@ def desc_from(cfg, T: int | None = None, out_f32: bool = False) -> abi.MoELayerD
                      kind=cfg.kind, n_ffn=g("n_ffn"), hidden=g("hidden"), n_shared=g("n_shared"),
                      hidden_shared=g("hidden_shared"), n_zero=g("n_zero"), n_copy=g("n_copy"),
                      n_const=g("n_const"), pk_rows=g("pk_rows"), pk_cols=g("pk_cols"),
-                     pk_topk_half=g("pk_topk_half"), d_query=g("d_query"), out_f32=out_f32)
+                     pk_topk_half=g("pk_topk_half"), d_query=g("d_query"), out_f32=out_f32,
+                     expert_fp8=bool(g("expert_fp8")))
 
 
 def torch_dtype(desc: abi.MoELayerDesc) -> torch.dtype:
@@ -68,7 +69,12 @@ class StageBuffers:
         self.offsets = torch.empty((groups + 1,), dtype=i32, device=device)
         self.row_of = torch.empty((T, k), dtype=i32, device=device)
         self.token_of = torch.empty((max(cap, 1),), dtype=i32, device=device)
-        if desc.kind == abi.MOE_EXPERT_SWIGLU:
+        if desc.kind == abi.MOE_EXPERT_SWIGLU and desc.expert_fp8:
+            # the rows' e4m3 codes, then (at a 256-byte boundary) their fp32 scales
+            codes = (max(cap, 1) * d + 255) // 256 * 256
+            self.x_sorted = torch.empty((codes + max(cap, 1) * 4,), dtype=torch.uint8, device=device)
+            self.y_sorted = torch.empty((max(cap, 1), d), dtype=f32, device=device)
+        elif desc.kind == abi.MOE_EXPERT_SWIGLU:
             self.x_sorted = torch.empty((max(cap, 1), d), dtype=dt, device=device)
             self.y_sorted = torch.empty((max(cap, 1), d), dtype=f32, device=device)
         else:

@@ -23,6 +23,10 @@ shapes and distributions follow the workloads the pages study:
                       page, 2.1 "Shared Dense MLP"), a SwiGLU FFN of hidden
                       width 2816 (8/3 d rounded up to a multiple of 128; the
                       page gives no size).
+* ``mixtral_fp8``, ``longtail_fp8``, ``moepp_fp8``: the same layers with FP8
+                      experts (PCoMoE page, "Improvements", 3: FP8 for the
+                      expert computation, BF16 for the gating): each expert
+                      weight row stored as e4m3 codes with an fp32 scale.
 """
 
 from __future__ import annotations
@@ -54,6 +58,7 @@ class MoEConfig:
     pk_cols: int = 0
     pk_topk_half: int = 0
     d_query: int = 0
+    expert_fp8: bool = False         # expert weights stored as e4m3 codes + fp32 row scales
 
     @property
     def n_routed(self) -> int:
@@ -91,8 +96,11 @@ CONFIGS: dict[str, MoEConfig] = {
         name="omnimoe", T=8192, d=1024, top_k=64, dtype="bf16", kind="atomic",
         pk_rows=512, pk_cols=512, pk_topk_half=32, d_query=1024, n_shared=1, hidden_shared=2816),
 }
+for _base in ("mixtral", "longtail", "moepp"):
+    CONFIGS[_base + "_fp8"] = dataclasses.replace(CONFIGS[_base], name=_base + "_fp8", expert_fp8=True)
 
-ORDER = ["tiny_f32", "mixtral", "longtail", "moepp", "atomic", "omnimoe"]
+ORDER = ["tiny_f32", "mixtral", "longtail", "moepp", "atomic", "omnimoe", "mixtral_fp8", "longtail_fp8",
+         "moepp_fp8"]
 
 
 def get_config(name: str) -> MoEConfig:

@@ -13,7 +13,10 @@ Recipe (the same for the CUDA path and the oracle):
   expert vectors u and v; sub-keys and the constant vectors v are N(0, 1);
   x is N(0, x_std^2); the previous layer's logits are N(0, 1) in fp32;
 * the long-tail and MoE++ router biases are stored numbers (fp32), fitted by a
-  script that uses only the oracle; they are loaded, not computed, here.
+  script that uses only the oracle; they are loaded, not computed, here;
+* FP8-expert workloads store each expert weight row (drawn as above, in bf16)
+  as e4m3 codes of row / s with s = max|row| / 448 (fp32; torch's float8
+  cast, nearest) and the row scale s: the stored weight is code * s.
 """
 
 from __future__ import annotations
@@ -78,6 +81,15 @@ def _fill_parallel(jobs, seed: int, dt: torch.dtype) -> None:
             list(ex.map(one, jobs))
     finally:
         torch.set_num_threads(prev)
+
+
+def _to_e4m3_rows(w: torch.Tensor):
+    """[..., K] weights -> (e4m3 codes as uint8, fp32 row scales [...])."""
+    wf = w.to(torch.float32)
+    s = wf.abs().amax(dim=-1) / 448.0
+    s = torch.where(s > 0, s, torch.ones_like(s))
+    codes = (wf / s.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), s.contiguous()
 
 
 def _dt(cfg: MoEConfig) -> torch.dtype:
@@ -164,6 +176,11 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
     if cfg.n_const:
         w["w_const_mix"] = _normal((cfg.n_const, 2, d), d ** -0.5, seed, _WC, dt)
         w["const_vec"] = _normal((cfg.n_const, d), 1.0, seed, _CV, dt)
+    if cfg.expert_fp8:
+        for name, sname in (("w_gate", "s_gate"), ("w_up", "s_up"), ("w_down", "s_down"),
+                            ("ws_gate", "ss_gate"), ("ws_up", "ss_up"), ("ws_down", "ss_down")):
+            if name in w:
+                w[name], w[sname] = _to_e4m3_rows(w[name])
     return w
 
 

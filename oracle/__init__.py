@@ -308,15 +308,20 @@ def _u8(t):
 
 def fp8_moe_tokens(cfg, inp: dict, tokens, idx_in=None):
     """Layer output (fp64) for the listed tokens with FP8 experts: ``inp`` holds
-    the e4m3 codes (w_gate8, w_up8, w_down8 and ws_*8 for shared experts, as
-    uint8 or float8_e4m3fn tensors) and their fp32 row scales (s_gate, s_up,
-    s_down, ss_*), plus x, the router and MoE++ tensors as for moe_tokens.
-    Returns (y, idx, gate, margin)."""
+    the e4m3 codes (w_gate8, w_up8, w_down8 and ws_*8 for shared experts, or
+    under w_gate, ... themselves; uint8 or float8_e4m3fn tensors) and their
+    fp32 row scales (s_gate, s_up, s_down, ss_*), plus x, the router and MoE++
+    tensors as for moe_tokens.  Returns (y, idx, gate, margin)."""
     tokens = _np_i32(tokens).reshape(-1)
     n = tokens.shape[0]
     x = _cpu(inp["x"])
     g = {k_: _cpu(inp.get(k_)) for k_ in ("w_router", "w_const_mix", "const_vec")}
-    codes = {k_: _u8(inp.get(k_)) for k_ in ("w_gate8", "w_up8", "w_down8", "ws_gate8", "ws_up8", "ws_down8")}
+    def codes_of(name):   # the codes under name + "8", or under name itself when it holds codes
+        c = inp.get(name + "8")
+        if c is None and inp.get(name) is not None and inp[name].dtype in (torch.uint8, torch.float8_e4m3fn):
+            c = inp[name]
+        return _u8(c)
+    codes = {k_ + "8": codes_of(k_) for k_ in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")}
     scales = {k_: (None if inp.get(k_) is None else _cpu(inp[k_]).to(torch.float32).contiguous())
               for k_ in ("s_gate", "s_up", "s_down", "ss_gate", "ss_up", "ss_down")}
     bias = inp.get("router_bias")

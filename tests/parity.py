@@ -185,7 +185,19 @@ def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True, f
     R = check_permutation(cfg, idx, b.offsets.cpu().numpy(), b.row_of.cpu().numpy(),
                           b.token_of.cpu().numpy(), cfg.n_ffn, n_ids, cfg.n_shared, T)
     total = R + cfg.n_shared * T
-    if check_sorted and total:
+    fp8 = getattr(cfg, "expert_fp8", False)
+    if check_sorted and total and fp8:
+        # e4m3 codes and power-of-two scales of the permuted rows: bit-exact with
+        # the oracle's quantization of the same rows (a power-of-two division is exact)
+        cap = b.y_sorted.shape[0]
+        off = (cap * cfg.d + 255) // 256 * 256
+        codes = b.x_sorted[:total * cfg.d].view(total, cfg.d).cpu()
+        scales = b.x_sorted[off:off + cap * 4].view(torch.float32)[:total].cpu().double().numpy()
+        q_ref, s_ref = oracle.quantize_rows(inp["x"][b.token_of[:total].long().cpu()])
+        np.testing.assert_array_equal(scales, s_ref, err_msg="x_sorted row scales")
+        np.testing.assert_array_equal(codes.view(torch.float8_e4m3fn).double().numpy(), q_ref,
+                                      err_msg="x_sorted e4m3 codes")
+    elif check_sorted and total:
         tok = b.token_of[:total].long()
         assert torch.equal(b.x_sorted[:total], dev["x"][tok]), "x_sorted rows"
     if cfg.n_const:
@@ -195,7 +207,8 @@ def check_swiglu_layer(cfg, inp: dict, tokens=None, check_sorted: bool = True, f
         tokens = np.arange(T)
     tokens = np.asarray(tokens, dtype=np.int32)
     y_gpu = b.y.float().cpu().numpy()[tokens].astype(np.float64)
-    y_ref, _, _, _ = oracle.moe_tokens(cfg, inp, tokens, idx_in=idx[tokens])
+    layer_ref = oracle.fp8_moe_tokens if fp8 else oracle.moe_tokens
+    y_ref, _, _, _ = layer_ref(cfg, inp, tokens, idx_in=idx[tokens])
     rel = assert_close(y_gpu, y_ref, cfg.dtype)
     rep.update(rel_err=rel, R=R, n_tokens=len(tokens), rel_err_out=_out_err(r, tokens, y_ref))
     return rep
