@@ -281,8 +281,10 @@ MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weigh
  *   phase 0: the three in order.
  * Layers it applies to (else MOE_ERR_UNSUPPORTED, nothing enqueued): SwiGLU
  * kind, bf16, n_ffn > 0, no shared experts, top_k <= 2, d_model a multiple
- * of 256, hidden a multiple of 128.  moe_layer_forward uses this step for
- * every such layer.
+ * of 256, hidden a multiple of 128.  moe_layer_forward keeps the two-pass
+ * step (moe_grouped_ffn + moe_combine): on B200 it measured faster on the
+ * Mixtral-shaped and MoE++ layers, because zeroing the accumulator and the
+ * atomic epilogue cost more inside the GEMMs than the y_sorted round trip.
  * Arguments as moe_route / moe_permute produce them (expert_offsets [n_ffn +
  * 1], row_of [T, top_k], token_of [T * top_k], x_sorted [row capacity,
  * d_model] or NULL); x [T, d_model]; y [T, d_model] (bf16, or fp32 if

@@ -1248,10 +1248,10 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     // warps, which a short mainloop does not hide; measured on B200, K = 1024
     // shared-branch gate/up 72 us row-tiled vs 84 us in this form)
     // (its epilogue writes 16-byte pieces of output rows: row stride and base aligned)
-    // (the fused forms exist only in the token-column form, for any K)
+    // (the fused and e4m3 forms exist only in the token-column form, for any K)
     const bool tn = MOE_GEMM_TN && (p.pair || p.tn_any || p.fuse) && p.b_kmod == 0 && p.ldo % 8 == 0 &&
                     reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
-                    ((EPI == EPI_SWIGLU && p.N % 128 == 0 && (p.K >= MOE_TN_SWIGLU_MIN_K || p.fuse)) ||
+                    ((EPI == EPI_SWIGLU && p.N % 128 == 0 && (p.K >= MOE_TN_SWIGLU_MIN_K || p.fuse || p.fp8)) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));
     // fuse: 1 = gathered B rows + zeroing, 3 = zeroing (B from x_sorted) -- SwiGLU; 2 = scatter-add -- fp32
     const bool swiglu_fuse = p.fuse == 1 || p.fuse == 3;

@@ -143,8 +143,14 @@ size_t scratch_max(const moe_layer_desc* d)
     return std::max(std::max(s.route, s.permute), std::max(s.ffn, (size_t)256));
 }
 
+// moe_layer_forward's expert step: the two-pass one (gather copy, GEMMs, combine
+// kernel).  The fused step was measured on B200 alongside it, interleaved, and
+// is slower on the Mixtral-shaped and MoE++ layers (2.203 vs 2.158 ms and 1.398
+// vs 1.377 ms): zeroing the accumulator in the gate/up epilogue costs ~40 us
+// and the atomic epilogue ~15 us more than plain stores, against the ~15-20 us
+// the finish kernel saves over the combine.  1 makes the layer take it.
 #ifndef MOE_FUSED_LAYER
-#define MOE_FUSED_LAYER 1     // moe_layer_forward takes the fused expert step where the layer allows it
+#define MOE_FUSED_LAYER 0
 #endif
 
 // The fused expert step (gather in the gate/up GEMM's loads, combine in the

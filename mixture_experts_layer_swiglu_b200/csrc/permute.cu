@@ -16,14 +16,19 @@
 //               one warp per row.
 // Shared experts get groups n_ffn.. holding every token in order.
 //
-// Atomic kind (N up to millions of experts, ~2 tasks each):
-//   histogram with integer atomics, a three-kernel exclusive scan (no
-//   cross-block waits), placement through per-expert cursors, then each
-//   expert's short segment is sorted by slot id (= token order), which fixes
-//   the order whatever order the atomics took.
+// Atomic kind (N up to millions of experts, ~2 tasks each), two launches:
+//   a kernel zeroes the counts and a barrier counter; one cooperative kernel
+//   (every block resident) then runs histogram (integer atomics) -> per-block
+//   totals -> exclusive scan -> placement through per-expert cursors ->
+//   per-expert sort of each short segment by slot id (= token order), which
+//   fixes the order whatever order the atomics took; the phases are separated
+//   by a grid barrier whose waits are bounded (2 s, then MOE_ERR_TIMEOUT).
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -34,7 +39,6 @@ namespace {
 
 constexpr int P_TOK = 256;        // tokens per count / scatter block
 constexpr int P_MAXE = 1024;      // max FFN experts of the mask kernels
-constexpr int SCAN_ELEMS = 4096;  // elements per block of the atomic-kind scan
 
 __device__ __forceinline__ bool build_masks(const PermuteArgs& a, uint32_t (*mask)[8], int b)
 {
@@ -184,115 +188,144 @@ __global__ void zero_i32_kernel(int32_t* p, long long n)
         p[i] = 0;
 }
 
-__global__ void atomic_count_kernel(const PermuteArgs a)
+// ---- the atomic-kind permutation in one cooperative kernel
+
+constexpr int AP_THREADS = 256;
+constexpr int AP_MAX_BLOCKS = 4096;    // blocksum entries in the workspace
+
+// Grid barrier number `phase` (1, 2, ...) on a counter zeroed before the
+// launch: every block adds one and waits for phase * gridDim.x arrivals.
+// The cooperative launch makes every block resident, so the wait ends; it is
+// still bounded.  Returns false (MOE_ERR_TIMEOUT recorded) if it gave up.
+__device__ __forceinline__ bool ap_grid_sync(unsigned* bar, unsigned phase, int* s_ok)
 {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();                                    // this block's writes before its arrival
+        atomicAdd(bar, 1u);
+        const unsigned target = phase * gridDim.x;
+        bool ok = true;
+        const uint64_t t0 = globaltimer();
+        unsigned v;
+        for (uint32_t i = 0;; ++i) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= target) break;
+            if ((i & 255u) == 255u && globaltimer() - t0 > kWaitLimitNs) { ok = false; break; }
+        }
+        if (!ok) set_status(MOE_ERR_TIMEOUT);
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+// Sum of v over the block (all threads get it).
+__device__ __forceinline__ int ap_block_sum(int v, int* red)
+{
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    int t = 0;
+#pragma unroll
+    for (int i = 0; i < AP_THREADS / 32; ++i) t += red[i];
+    return t;
+}
+
+__global__ void __launch_bounds__(AP_THREADS) atomic_permute_kernel(const PermuteArgs a, unsigned* bar)
+{
+    __shared__ int red[AP_THREADS / 32];
+    __shared__ int s_ok;
     const long long n = (long long)a.T * a.k;
-    for (long long s = blockIdx.x * (long long)blockDim.x + threadIdx.x; s < n;
-         s += (long long)gridDim.x * blockDim.x) {
+    const int N = a.n_ids;
+    const long long gstride = (long long)gridDim.x * blockDim.x;
+    const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    // 1. histogram
+    for (long long s = gtid; s < n; s += gstride) {
         const int e = a.idx[s];
-        if (e < 0 || e >= a.n_ids) { set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
+        if (e < 0 || e >= N) { set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
         atomicAdd(&a.ws_counts[e], 1);
     }
-}
-
-__device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int w = warp_tot[lane];
-        int wi = w;
+    if (!ap_grid_sync(bar, 1, &s_ok)) return;
+    // 2. this block's chunk of experts and its total
+    const int chunk = cdiv(N, gridDim.x);
+    const int lo = min(N, (int)blockIdx.x * chunk), hi = min(N, lo + chunk);
+    int part = 0;
+    for (int e = lo + threadIdx.x; e < hi; e += AP_THREADS) part += a.ws_counts[e];
+    const int total = ap_block_sum(part, red);
+    if (threadIdx.x == 0) a.ws_blocksum[blockIdx.x] = total;
+    if (!ap_grid_sync(bar, 2, &s_ok)) return;
+    // 3. exclusive scan: the totals of the blocks before this one, then the chunk
+    int pre = 0;
+    for (int b = threadIdx.x; b < (int)blockIdx.x; b += AP_THREADS) pre += a.ws_blocksum[b];
+    int run = ap_block_sum(pre, red);
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int base = lo; base < hi; base += AP_THREADS) {
+        const int e = base + threadIdx.x;
+        const int c = e < hi ? a.ws_counts[e] : 0;
+        int incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += u;
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
         }
-        warp_tot[lane] = wi - w;
-        if (lane == 31) *total = wi;
+        __syncthreads();
+        if (lane == 31) red[w] = incl;
+        __syncthreads();
+        int wpre = 0;
+        for (int i = 0; i < w; ++i) wpre += red[i];
+        int step = 0;
+#pragma unroll
+        for (int i = 0; i < AP_THREADS / 32; ++i) step += red[i];
+        if (e < hi) a.offsets[e] = run + wpre + incl - c;
+        run += step;
     }
-    __syncthreads();
-    const int r = warp_tot[warp] + incl - v;
-    __syncthreads();
-    return r;
-}
-
-// pass 1: per-block totals of SCAN_ELEMS counts
-__global__ void __launch_bounds__(1024) atomic_scan1_kernel(const int32_t* counts, int N, int32_t* blocksum)
-{
-    __shared__ int wt[32];
-    __shared__ int tot;
-    const long long base = (long long)blockIdx.x * SCAN_ELEMS + threadIdx.x * 4;
-    int s = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) if (base + i < N) s += counts[base + i];
-    block_excl_scan_1024(s, wt, &tot);
-    if (threadIdx.x == 0) blocksum[blockIdx.x] = tot;
-}
-
-// pass 2: offsets[e] = (sum of the totals of the blocks before this one) +
-// exclusive scan inside the block; each block sums the preceding totals
-// itself (nb <= 4096), so no third pass is needed.
-__global__ void __launch_bounds__(1024) atomic_scan2_kernel(const int32_t* counts, int N,
-                                                            const int32_t* blocksum, int32_t* offsets)
-{
-    __shared__ int wt[32];
-    __shared__ int tot;
-    int pre = 0;
-    for (int i = threadIdx.x; i < (int)blockIdx.x; i += blockDim.x) pre += blocksum[i];
-    block_excl_scan_1024(pre, wt, &tot);
-    const int base_sum = tot;                  // sum of all preceding block totals
-    const long long base = (long long)blockIdx.x * SCAN_ELEMS + threadIdx.x * 4;
-    int v[4], s = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) { v[i] = (base + i < N) ? counts[base + i] : 0; s += v[i]; }
-    int run = base_sum + block_excl_scan_1024(s, wt, &tot);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (base + i < N) offsets[base + i] = run;
-        run += v[i];
-        if (base + i == N - 1) offsets[N] = run;
-    }
-}
-
-__global__ void atomic_place_kernel(const PermuteArgs a)
-{
-    const long long n = (long long)a.T * a.k;
-    for (long long s = blockIdx.x * (long long)blockDim.x + threadIdx.x; s < n;
-         s += (long long)gridDim.x * blockDim.x) {
+    if (hi == N && lo < hi && threadIdx.x == 0) a.offsets[N] = run;
+    if (!ap_grid_sync(bar, 3, &s_ok)) return;
+    // 4. placement through per-expert cursors (any order; sorted next)
+    for (long long s = gtid; s < n; s += gstride) {
         const int e = a.idx[s];
-        if (e < 0 || e >= a.n_ids) { a.row_of[s] = -1; continue; }
-        const int pos = a.offsets[e] + atomicSub(&a.ws_counts[e], 1) - 1;   // any order; sorted next
+        if (e < 0 || e >= N) { a.row_of[s] = -1; continue; }
+        const int pos = a.offsets[e] + atomicSub(&a.ws_counts[e], 1) - 1;
         a.token_of[pos] = (int)s;
     }
-}
-
-// Sort each expert's segment by slot id and record row_of.
-__global__ void atomic_sort_kernel(const PermuteArgs a)
-{
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < a.n_ids;
-         e += (long long)gridDim.x * blockDim.x) {
-        const int lo = a.offsets[e], hi = a.offsets[e + 1];
-        for (int i = lo + 1; i < hi; ++i) {
+    if (!ap_grid_sync(bar, 4, &s_ok)) return;
+    // 5. each expert's segment sorted by slot id, and row_of
+    for (long long e = gtid; e < N; e += gstride) {
+        const int s0 = a.offsets[e], s1 = a.offsets[e + 1];
+        for (int i = s0 + 1; i < s1; ++i) {
             const int v = a.token_of[i];
             int j = i - 1;
-            while (j >= lo && a.token_of[j] > v) { a.token_of[j + 1] = a.token_of[j]; --j; }
+            while (j >= s0 && a.token_of[j] > v) { a.token_of[j + 1] = a.token_of[j]; --j; }
             a.token_of[j + 1] = v;
         }
-        for (int i = lo; i < hi; ++i) a.row_of[a.token_of[i]] = i;
+        for (int i = s0; i < s1; ++i) a.row_of[a.token_of[i]] = i;
     }
+}
+
+int ap_grid(int N)
+{
+    static std::atomic<int> per_sm[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    int b = per_sm[dev].load(std::memory_order_relaxed);
+    if (b == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, atomic_permute_kernel, AP_THREADS, 0) != cudaSuccess ||
+            b <= 0)
+            b = 1;
+        per_sm[dev].store(b, std::memory_order_relaxed);
+    }
+    (void)N;
+    return std::max(1, std::min(b * num_sms(), AP_MAX_BLOCKS));
 }
 
 }  // namespace
 
 int permute_blocks(int T) { return std::max(1, cdiv(T, P_TOK)); }
-int atomic_scan_blocks(int N) { return std::max(1, cdiv(N, SCAN_ELEMS)); }
+// ints after the counts in the atomic kind's workspace: the block totals, then the barrier counter
+int atomic_scan_blocks(int N) { (void)N; return AP_MAX_BLOCKS + 64; }
 
 moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
 {
@@ -328,18 +361,19 @@ moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
 moe_status launch_permute_atomic(const PermuteArgs& a, cudaStream_t st)
 {
     const int N = a.n_ids;
-    const int grid_n = std::max(1, std::min(cdiv(N, 256), num_sms() * 8));
-    zero_i32_kernel<<<std::max(1, std::min(cdiv(N, 1024), num_sms() * 4)), 256, 0, st>>>(a.ws_counts, N);
-    const long long n = (long long)a.T * a.k;
-    const int grid_t = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, num_sms() * 8));
-    atomic_count_kernel<<<grid_t, 256, 0, st>>>(a);
-    const int nb = atomic_scan_blocks(N);
-    if (nb > 4096) return MOE_ERR_UNSUPPORTED;
-    atomic_scan1_kernel<<<nb, 1024, 0, st>>>(a.ws_counts, N, a.ws_blocksum);
-    atomic_scan2_kernel<<<nb, 1024, 0, st>>>(a.ws_counts, N, a.ws_blocksum, a.offsets);
-    atomic_place_kernel<<<grid_t, 256, 0, st>>>(a);
-    atomic_sort_kernel<<<grid_n, 256, 0, st>>>(a);
-    count_launch(6);
+    unsigned* bar = reinterpret_cast<unsigned*>(a.ws_blocksum + AP_MAX_BLOCKS);
+    // counts, block totals and the barrier counter are one contiguous zeroed
+    // range (the counts' 256-byte padding included)
+    int32_t* zero_end = a.ws_blocksum + AP_MAX_BLOCKS + 64;
+    const long long nz = zero_end - a.ws_counts;
+    zero_i32_kernel<<<std::max(1, (int)std::min<long long>((nz + 1023) / 1024, num_sms() * 4)), 256, 0, st>>>(a.ws_counts, nz);
+    count_launch();
+    PermuteArgs args = a;
+    void* params[2] = {&args, &bar};
+    cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(atomic_permute_kernel), dim3(ap_grid(N)),
+                                                dim3(AP_THREADS), params, 0, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    count_launch();
     return cuda_status(cudaGetLastError());
 }
 

@@ -108,7 +108,9 @@ def expert_ids(cfg: MoEConfig) -> dict:
 def load_router_bias(cfg: MoEConfig) -> torch.Tensor | None:
     if cfg.router_bias is None:
         return None
-    path = GOLDEN_DIR / f"{cfg.name}_router_bias.txt"
+    # an FP8-expert workload has the router (and so the bias) of its bf16 layer
+    base = cfg.name[:-len("_fp8")] if cfg.expert_fp8 and cfg.name.endswith("_fp8") else cfg.name
+    path = GOLDEN_DIR / f"{base}_router_bias.txt"
     vals = [float(l.split()[0]) for l in path.read_text().splitlines()
             if l.strip() and not l.lstrip().startswith("#")]
     if len(vals) != cfg.n_routed:
