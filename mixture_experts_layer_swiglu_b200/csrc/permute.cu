@@ -190,7 +190,7 @@ __global__ void zero_i32_kernel(int32_t* p, long long n)
 
 // ---- the atomic-kind permutation in one cooperative kernel
 
-constexpr int AP_THREADS = 256;
+constexpr int AP_THREADS = 1024;       // one block per SM: few spinners at each grid barrier
 constexpr int AP_MAX_BLOCKS = 4096;    // blocksum entries in the workspace
 
 // Grid barrier number `phase` (1, 2, ...) on a counter zeroed before the
@@ -210,7 +210,8 @@ __device__ __forceinline__ bool ap_grid_sync(unsigned* bar, unsigned phase, int*
         for (uint32_t i = 0;; ++i) {
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
             if (v >= target) break;
-            if ((i & 255u) == 255u && globaltimer() - t0 > kWaitLimitNs) { ok = false; break; }
+            __nanosleep(64);                                // back off: every block polls one line
+            if ((i & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) { ok = false; break; }
         }
         if (!ok) set_status(MOE_ERR_TIMEOUT);
         *s_ok = ok;
@@ -318,7 +319,7 @@ int ap_grid(int N)
         per_sm[dev].store(b, std::memory_order_relaxed);
     }
     (void)N;
-    return std::max(1, std::min(b * num_sms(), AP_MAX_BLOCKS));
+    return std::max(1, std::min(std::min(b, 1) * num_sms(), AP_MAX_BLOCKS));
 }
 
 }  // namespace
