@@ -101,14 +101,31 @@ constexpr int R_SMEM = R_STAGES * R_TILE * R_CHUNK_BYTES + 2 * R_W_BYTES + R_WAR
 // bias and the previous layer's logits, writes logits_out, selects the k
 // largest (value desc, ties to the lower id) with a warp argmax, softmax gates
 // over the selected, and the constant experts' (a1, a2).
-__device__ __forceinline__ void route_token(const RouterArgs& a, int t, float* z, int lane)
+// (E_r <= 64 and `pre` given: the bias and previous-layer logits of experts
+// lane and lane + 32, loaded ahead by the caller; the sum order is the same.)
+__device__ __forceinline__ void route_token(const RouterArgs& a, int t, float* z, int lane,
+                                            const float (*pre)[2] = nullptr)
 {
-    for (int e = lane; e < a.E_r; e += 32) {
-        float v = z[e];
-        if (a.bias) v += a.bias[e];
-        if (a.prev) v += a.prev[(long long)t * a.E_r + e];
-        z[e] = v;
-        if (a.logits_out) a.logits_out[(long long)t * a.E_r + e] = v;
+    if (pre) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int e = lane + 32 * i;
+            if (e < a.E_r) {
+                float v = z[e];
+                if (a.bias) v += pre[i][0];
+                if (a.prev) v += pre[i][1];
+                z[e] = v;
+                if (a.logits_out) a.logits_out[(long long)t * a.E_r + e] = v;
+            }
+        }
+    } else {
+        for (int e = lane; e < a.E_r; e += 32) {
+            float v = z[e];
+            if (a.bias) v += a.bias[e];
+            if (a.prev) v += a.prev[(long long)t * a.E_r + e];
+            z[e] = v;
+            if (a.logits_out) a.logits_out[(long long)t * a.E_r + e] = v;
+        }
     }
     __syncwarp();
     uint32_t taken = 0;   // bit i: expert lane + 32 i already selected
@@ -384,23 +401,24 @@ __global__ void __launch_bounds__(RM_WARPS * 32) router_mma_kernel(const RouterA
 // most 64 router + mixing rows): x is read once from HBM, so the kernel is
 // built to keep HBM busy.  One persistent block per SM; a producer warp
 // copies each 16-token tile's rows into shared memory with bulk copies
-// (cp.async.bulk, no multicast), chunk by chunk (16 rows x 1024 elements of d
+// (cp.async.bulk, no multicast), chunk by chunk (16 rows x 960 elements of d
 // per chunk, one copy per row), into a ring of stages with mbarrier
 // completion, running ahead across tiles (100-130 KiB in flight per SM).
 // The router rows are copied into shared memory once per block when they fit
-// (else read through L1).  The 16 consumer warps split each chunk's d: warp w
-// takes the 64-wide slices w, w + 16 of the chunk and accumulates, in
+// (else read through L1).  The 15 consumer warps split each chunk's d: warp w
+// takes the 64-wide slice w of the chunk and accumulates, in
 // registers across the tile's chunks, the m16n8k16 tiles of those slices as
 // router_mma_kernel does (lane (g, q) uses 32 contiguous bytes of token rows g
 // and g + 8 and of router row g of each n8 tile, in the same k order for A and
 // B); rows are padded by 16 bytes in shared memory so the fragment reads are
-// conflict-free.  At the tile's end the 16 partial logits are summed in warp
-// order (fixed, so the logits do not depend on timing) and each warp routes
-// one token with route_token, while the producer already streams the next
-// tile.
-constexpr int RS_WARPS = 16;                   // consumer warps
+// conflict-free.  At the tile's end the 15 partial logits are summed in warp
+// order (fixed, so the logits do not depend on timing) and the warps route
+// the 16 tokens with route_token (the bias and previous-layer logits of
+// their tokens loaded before the MMAs), while the producer already streams
+// the next tile.
+constexpr int RS_WARPS = 15;                   // consumer warps (16 warps in all: 4 per SM sub-partition)
 constexpr int RS_THREADS = (RS_WARPS + 1) * 32;
-constexpr int RS_KC = 1024;                    // d elements per chunk
+constexpr int RS_KC = 64 * RS_WARPS;           // d elements per chunk: one 64-wide slice per consumer warp
 constexpr int RS_PITCH = RS_KC * 2 + 16;       // bytes per staged row
 constexpr int RS_STAGE = 16 * RS_PITCH;        // 16 token rows
 constexpr int RS_MAXSTAGES = 4;
@@ -553,6 +571,20 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
     uint32_t ph = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int t0 = tile * 16;
+        // the bias and previous-layer logits of this warp's token, loaded now so
+        // that routing it after the MMAs does not wait on them
+        float pre[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        if (t0 + warp < a.T) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int e = lane + 32 * i;
+                if (e < a.E_r) {
+                    if (a.bias) pre[i][0] = a.bias[e];
+                    if (a.prev) pre[i][1] = a.prev[(long long)(t0 + warp) * a.E_r + e];
+                }
+            }
+        }
+        // (warp 0 also routes token 15, whose values it loads when routing it)
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
@@ -608,7 +640,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
             zsum[i] = v;
         }
         rs_consumer_sync();
-        if (t0 + warp < a.T) route_token(a, t0 + warp, zsum + warp * zpitch, lane);
+        if (t0 + warp < a.T) route_token(a, t0 + warp, zsum + warp * zpitch, lane, pre);
+        if (warp == 0 && t0 + 15 < a.T) route_token(a, t0 + 15, zsum + 15 * zpitch, lane);
         rs_consumer_sync();   // zsum and the partials are free for the next tile
     }
 }
