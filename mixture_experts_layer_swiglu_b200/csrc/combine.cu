@@ -597,9 +597,10 @@ __global__ void __launch_bounds__(PB_WARPS * 32, 1) atomic_phase_b_kernel(const 
 // token adding only the slots whose expert lies in range p: the rows a range
 // touches (~56 MiB) are read from DRAM once and then served from L2, and the
 // token's fp32 accumulator row (the [T, d] buffer, 32 MiB, also L2-resident)
-// carries the sum from pass to pass.  Sum order: range, then slot.  The last
-// pass adds the slots of its range and writes y (the shared dense branch's
-// output, when present, is the accumulator's starting value).
+// carries the sum from pass to pass.  Sum order: range, then slot.  The first
+// pass starts from the shared dense branch's output when there is one (read
+// only, so the call can be repeated on the same inputs); the last pass adds
+// the slots of its range and writes y.
 constexpr int PR_WARPS = 8;
 constexpr int PR_GROUP = 4;          // v rows loaded together
 
@@ -621,10 +622,11 @@ __global__ void __launch_bounds__(PR_WARPS * 32) atomic_phase_b_range_kernel(con
             for (int v = 0; v < NV; ++v)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) sum[v][i] = 0.f;
-        } else {   // the previous passes' sum (or the shared branch's output)
+        } else {   // the previous passes' sum, or (first pass) the shared branch's output
+            const float4* srow = first ? reinterpret_cast<const float4*>(a.shared_out + (long long)t * a.d) : arow;
 #pragma unroll
             for (int v = 0; v < NV; ++v) {
-                const float4 p0 = arow[(v * 32 + lane) * 2], p1 = arow[(v * 32 + lane) * 2 + 1];
+                const float4 p0 = srow[(v * 32 + lane) * 2], p1 = srow[(v * 32 + lane) * 2 + 1];
                 sum[v][0] = p0.x; sum[v][1] = p0.y; sum[v][2] = p0.z; sum[v][3] = p0.w;
                 sum[v][4] = p1.x; sum[v][5] = p1.y; sum[v][6] = p1.z; sum[v][7] = p1.w;
             }
