@@ -210,15 +210,13 @@ MOE_API moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_i
  * Atomic: c[s] = topk_gate[s] * GELU(u_e . x_t) for each task s = t*K + j of
  *   expert e, over the expert-sorted task order in units of 16 tasks whose
  *   dot products are one tensor-core tile (each touched u_e read once per
- *   unit); y_sorted is float c[T*K] in slot order, followed at byte offset
- *   align256(T*K*4) by n_shared [T, d_model] fp32 rows of the shared branch
- *   and then a [T, d_model] fp32 accumulator that moe_combine uses
- *   (y_sorted: align256(T*K*4) + (n_shared + 1)*T*d_model*4 bytes).
- *   x_sorted unused.  The workspace holds the expert of each task (T*top_k
- *   int32).  With a shared dense branch ("OmniMoE" 2.1, Shared Dense MLP;
- *   n_shared = 1) the call also computes ys = Ws_down (silu(Ws_gate x_t) *
- *   (Ws_up x_t)) for every token (two grouped GEMMs, the hidden activation
- *   rounded to bf16 in the workspace) into the shared rows after c.
+ *   unit); y_sorted is float c[T*K] in slot order.  x_sorted unused.  The
+ *   workspace holds the expert of each task (T*top_k int32).  With a shared
+ *   dense branch ("OmniMoE" 2.1, Shared Dense MLP; n_shared = 1) the call
+ *   also computes ys = Ws_down (silu(Ws_gate x_t) * (Ws_up x_t)) for every
+ *   token (two grouped GEMMs, the hidden activation rounded to bf16 in the
+ *   workspace) into y_sorted after c, at byte offset align256(T*K*4), as
+ *   [T, d_model] fp32.
  */
 MOE_API moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_layer_weights* w,
                            const void* x_sorted, const int32_t* expert_offsets,
@@ -250,11 +248,7 @@ MOE_API moe_status moe_grouped_ffn_phase(const moe_layer_desc* desc, const moe_l
  *   a1 x_t + a2 v_c for constant expert c (const_mix, w->const_vec);
  *   accumulated in fp32 in slot order, rounded once to dtype.
  * Atomic: y_t = sum_j c[t*K + j] * v_{topk_idx[t, j]} (+ the shared branch's
- *   row of y_sorted when n_shared = 1), fp32, rounded once.  The experts are
- *   taken in contiguous id ranges of ~64 MiB of v, one pass over the tokens
- *   per range, summing in (range, slot) order in y_sorted's fp32 accumulator
- *   (which it overwrites; c and the shared rows are only read, so the call
- *   can be repeated): a range's rows stay in L2 across the tokens.
+ *   row of y_sorted when n_shared = 1), fp32, rounded once.
  * y [T, d_model] in dtype, or fp32 if desc->out_f32.
  */
 MOE_API moe_status moe_combine(const moe_layer_desc* desc, const moe_layer_weights* w,

@@ -97,7 +97,7 @@ __device__ __forceinline__ void store8(void* p, long long i8, const float (&v)[8
 constexpr int CMB_SPLIT = 4;
 
 template <typename T, typename TO>
-__global__ void __launch_bounds__(256, 2) combine_kernel(const CombineArgs a)
+__global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
 {
     constexpr int V = 8;
     constexpr int WPB = 256 / 32;                    // warps per block
@@ -165,20 +165,6 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const CombineArgs a)
                             for (int v = 0; v < V; ++v) acc[u][v] += w[u][v];
                     }
                 }
-                // the rows of the first two FFN slots are loaded together, before
-                // any is used (the slot loop below adds every slot in order)
-                float pw[2][2][V];
-                bool pre[2] = {false, false};
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int e = j < a.k ? s_e[tib][j] : -1;
-                    if (!a.acc_rows && e >= 0 && e < zero0) {
-                        const long long rb = (long long)s_r[tib][j] * vecs;
-                        load8<float>(a.ys, rb + i, pw[j][0]);
-                        if (two) load8<float>(a.ys, rb + i + 32, pw[j][1]);
-                        pre[j] = true;
-                    }
-                }
                 bool have_x = false;
                 float xv[2][V];
                 for (int j = 0; j < a.k; ++j) {
@@ -187,20 +173,6 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const CombineArgs a)
                     if (e < 0) continue;
                     if (e < zero0) {
                         if (a.acc_rows) continue;         // already in the accumulator row
-                        if (j == 0 && pre[0]) {
-#pragma unroll
-                            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, pw[0][u][v], acc[u][v]);
-                            continue;
-                        }
-                        if (j == 1 && pre[1]) {
-#pragma unroll
-                            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, pw[1][u][v], acc[u][v]);
-                            continue;
-                        }
                         const long long rb = (long long)s_r[tib][j] * vecs;
                         float w[2][V];
                         load8<float>(a.ys, rb + i, w[0]);
@@ -588,117 +560,6 @@ __global__ void __launch_bounds__(PB_WARPS * 32, 1) atomic_phase_b_kernel(const 
     }
 }
 
-// ---- phase B by expert-id ranges: the touched v rows of a range stay in L2.
-//
-// The token-centric gather above reads each slot's v row (2 KiB) from wherever
-// it is, and v (512 MiB) is far larger than L2, so a row used by two tokens is
-// mostly read from DRAM twice.  Here the N experts are cut into n_pass
-// contiguous id ranges of about 64 MiB of v each, and pass p goes over every
-// token adding only the slots whose expert lies in range p: the rows a range
-// touches (~56 MiB) are read from DRAM once and then served from L2, and the
-// token's fp32 accumulator row (the [T, d] buffer, 32 MiB, also L2-resident)
-// carries the sum from pass to pass.  Sum order: range, then slot.  The first
-// pass starts from the shared dense branch's output when there is one (read
-// only, so the call can be repeated on the same inputs); the last pass adds
-// the slots of its range and writes y.
-constexpr int PR_WARPS = 8;
-constexpr int PR_GROUP = 4;          // v rows loaded together
-
-template <int NV>
-__global__ void __launch_bounds__(PR_WARPS * 32) atomic_phase_b_range_kernel(const AtomicArgs a, float* acc,
-                                                                             int pass, int n_pass)
-{
-    const int lane = threadIdx.x & 31;
-    const long long lo = (long long)pass * a.N / n_pass, hi = (long long)(pass + 1) * a.N / n_pass;
-    const bool first = pass == 0, last = pass == n_pass - 1;
-    const int vecs = a.d / 8;                          // 8-element vectors per row
-    const uint4* vb = static_cast<const uint4*>(a.v);
-    const int nw = gridDim.x * PR_WARPS;
-    for (int t = blockIdx.x * PR_WARPS + (threadIdx.x >> 5); t < a.T; t += nw) {
-        float sum[NV][8];
-        float4* arow = reinterpret_cast<float4*>(acc + (long long)t * a.d);
-        if (first && !a.shared_out) {
-#pragma unroll
-            for (int v = 0; v < NV; ++v)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) sum[v][i] = 0.f;
-        } else {   // the previous passes' sum, or (first pass) the shared branch's output
-            const float4* srow = first ? reinterpret_cast<const float4*>(a.shared_out + (long long)t * a.d) : arow;
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                const float4 p0 = srow[(v * 32 + lane) * 2], p1 = srow[(v * 32 + lane) * 2 + 1];
-                sum[v][0] = p0.x; sum[v][1] = p0.y; sum[v][2] = p0.z; sum[v][3] = p0.w;
-                sum[v][4] = p1.x; sum[v][5] = p1.y; sum[v][6] = p1.z; sum[v][7] = p1.w;
-            }
-        }
-        // the token's slots in this range, in slot order (K <= 128: four per lane)
-        for (int j0 = 0; j0 < a.K; j0 += 32) {
-            const int j = j0 + lane;
-            int e = -1;
-            float c = 0.f;
-            if (j < a.K) {
-                e = a.idx[(long long)t * a.K + j];
-                if (e < 0 || e >= a.N) { if (first) set_status(MOE_ERR_DEVICE_BOUNDS); e = -1; }
-                else c = a.c[(long long)t * a.K + j];
-            }
-            unsigned m = __ballot_sync(FULL, e >= lo && e < hi);
-            while (m) {
-                int src[PR_GROUP];
-                int n = 0;
-#pragma unroll
-                for (int g = 0; g < PR_GROUP; ++g) {
-                    src[g] = m ? __ffs(m) - 1 : -1;
-                    if (m) { m &= m - 1; ++n; }
-                }
-                uint4 w[PR_GROUP][NV];
-#pragma unroll
-                for (int g = 0; g < PR_GROUP; ++g) {
-                    const int eg = __shfl_sync(FULL, e, src[g] < 0 ? 0 : src[g]);
-                    if (g < n) {
-#pragma unroll
-                        for (int v = 0; v < NV; ++v) w[g][v] = __ldg(vb + (long long)eg * vecs + v * 32 + lane);
-                    }
-                }
-#pragma unroll
-                for (int g = 0; g < PR_GROUP; ++g) {
-                    const float cg = __shfl_sync(FULL, c, src[g] < 0 ? 0 : src[g]);
-                    if (g < n) {
-#pragma unroll
-                        for (int v = 0; v < NV; ++v) {
-                            fma2(sum[v][0], sum[v][1], cg, bf16_lo(w[g][v].x), bf16_hi(w[g][v].x));
-                            fma2(sum[v][2], sum[v][3], cg, bf16_lo(w[g][v].y), bf16_hi(w[g][v].y));
-                            fma2(sum[v][4], sum[v][5], cg, bf16_lo(w[g][v].z), bf16_hi(w[g][v].z));
-                            fma2(sum[v][6], sum[v][7], cg, bf16_lo(w[g][v].w), bf16_hi(w[g][v].w));
-                        }
-                    }
-                }
-            }
-        }
-        if (!last) {
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                arow[(v * 32 + lane) * 2] = make_float4(sum[v][0], sum[v][1], sum[v][2], sum[v][3]);
-                arow[(v * 32 + lane) * 2 + 1] = make_float4(sum[v][4], sum[v][5], sum[v][6], sum[v][7]);
-            }
-        } else if (a.out_f32) {
-            float4* y = reinterpret_cast<float4*>(a.y);
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                const long long o = ((long long)t * vecs + v * 32 + lane) * 2;
-                y[o] = make_float4(sum[v][0], sum[v][1], sum[v][2], sum[v][3]);
-                y[o + 1] = make_float4(sum[v][4], sum[v][5], sum[v][6], sum[v][7]);
-            }
-        } else {
-            uint4* y = reinterpret_cast<uint4*>(a.y);
-#pragma unroll
-            for (int v = 0; v < NV; ++v)
-                y[(long long)t * vecs + v * 32 + lane] =
-                    make_uint4(pack_bf16(sum[v][0], sum[v][1]), pack_bf16(sum[v][2], sum[v][3]),
-                               pack_bf16(sum[v][4], sum[v][5]), pack_bf16(sum[v][6], sum[v][7]));
-        }
-    }
-}
-
 template <template <int> class K, typename... Args>
 moe_status launch_nv(int nv, int grid, cudaStream_t st, const AtomicArgs& a)
 {
@@ -757,42 +618,10 @@ moe_status launch_atomic_phase_a(const AtomicArgs& a, cudaStream_t st)
     return cuda_status(cudaGetLastError());
 }
 
-#ifndef MOE_PB_RANGES
-#define MOE_PB_RANGES 1       // phase B by expert-id ranges (0: one token-centric pass)
-#endif
-
-template <int NV> struct PhaseBRange {
-    static cudaError_t launch(int grid, cudaStream_t st, const AtomicArgs& a, float* acc, int pass, int n_pass)
-    {
-        atomic_phase_b_range_kernel<NV><<<grid, PR_WARPS * 32, 0, st>>>(a, acc, pass, n_pass);
-        return cudaSuccess;
-    }
-};
-
 moe_status launch_atomic_phase_b(const AtomicArgs& a, cudaStream_t st)
 {
     if (a.T == 0) return MOE_OK;
     if (a.K > 128) return MOE_ERR_UNSUPPORTED;
-    if (MOE_PB_RANGES && a.acc) {
-        // ranges of about 64 MiB of v, so that a range's touched rows and the
-        // accumulator fit in L2 together
-        const long long vbytes = (long long)a.N * a.d * 2;
-        const int n_pass = (int)std::max(1LL, std::min(16LL, (vbytes + (64LL << 20) - 1) / (64LL << 20)));
-        const int grid = std::max(1, std::min(cdiv(a.T, PR_WARPS), num_sms() * 8));
-        for (int p = 0; p < n_pass; ++p) {
-            cudaError_t e;
-            switch (a.d / 256) {
-                case 1: e = PhaseBRange<1>::launch(grid, st, a, a.acc, p, n_pass); break;
-                case 2: e = PhaseBRange<2>::launch(grid, st, a, a.acc, p, n_pass); break;
-                case 4: e = PhaseBRange<4>::launch(grid, st, a, a.acc, p, n_pass); break;
-                case 8: e = PhaseBRange<8>::launch(grid, st, a, a.acc, p, n_pass); break;
-                default: return MOE_ERR_UNSUPPORTED;
-            }
-            if (e != cudaSuccess) return cuda_status(e);
-            count_launch();
-        }
-        return cuda_status(cudaGetLastError());
-    }
     const int grid = std::max(1, std::min(cdiv(a.T, PB_WARPS), num_sms()));
     return launch_nv<PhaseB>(a.d / 256, grid, st, a);
 }

@@ -159,7 +159,6 @@ struct AtomicArgs {
     const float* gate;         // [T, K]
     float* c;                  // [T*K]
     const float* shared_out;   // [T, d] fp32 output of the shared dense branch, nullable
-    float* acc;                // [T, d] fp32 accumulator of the expert-range passes (shared_out's buffer)
     void* y;                   // [T, d] bf16, or fp32 if out_f32
     int T, d, K, N;
     int out_f32;

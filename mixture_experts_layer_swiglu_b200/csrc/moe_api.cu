@@ -213,8 +213,7 @@ LayerBufs layer_layout(const moe_layer_desc* d, void* base)
         b.ys = take((size_t)cap * d->d_model * 4);
     } else {
         b.xs = nullptr;
-        // c, the shared branch's [T, d] fp32 output (full layer), the combine's [T, d] fp32 accumulator
-        b.ys = take(al((size_t)Tk * 4) + (size_t)(d->n_shared + 1) * d->T * d->d_model * 4);
+        b.ys = take(al((size_t)Tk * 4) + (size_t)d->n_shared * d->T * d->d_model * 4);   // c, then the shared rows
     }
     b.scratch_bytes = scratch_max(d);
     if (d->kind == MOE_EXPERT_SWIGLU && MOE_FUSED_LAYER && fused_eligible(d))
@@ -600,10 +599,9 @@ moe_status combine_impl(const moe_layer_desc* d, const moe_layer_weights* w, con
         a.v = w->v;
         a.idx = idx;
         a.c = const_cast<float*>(static_cast<const float*>(ys));
-        float* after_c = reinterpret_cast<float*>(const_cast<char*>(static_cast<const char*>(ys)) +
-                                                  al((size_t)d->T * d->top_k * 4));
-        a.shared_out = d->n_shared ? after_c : nullptr;
-        a.acc = after_c + (size_t)d->n_shared * d->T * d->d_model;
+        a.shared_out = d->n_shared ? reinterpret_cast<const float*>(static_cast<const char*>(ys) +
+                                                                     al((size_t)d->T * d->top_k * 4))
+                                   : nullptr;
         a.y = y;
         a.T = d->T;
         a.d = d->d_model;

@@ -401,22 +401,21 @@ __global__ void __launch_bounds__(RM_WARPS * 32) router_mma_kernel(const RouterA
 // most 64 router + mixing rows): x is read once from HBM, so the kernel is
 // built to keep HBM busy.  One persistent block per SM; a producer warp
 // copies each 16-token tile's rows into shared memory with bulk copies
-// (cp.async.bulk, no multicast), chunk by chunk (16 rows x 960 elements of d
+// (cp.async.bulk, no multicast), chunk by chunk (16 rows x 1024 elements of d
 // per chunk, one copy per row), into a ring of stages with mbarrier
 // completion, running ahead across tiles (100-130 KiB in flight per SM).
 // The router rows are copied into shared memory once per block when they fit
-// (else read through L1).  The 15 consumer warps split each chunk's d: warp w
+// (else read through L1).  The 16 consumer warps split each chunk's d: warp w
 // takes the 64-wide slice w of the chunk and accumulates, in
 // registers across the tile's chunks, the m16n8k16 tiles of those slices as
 // router_mma_kernel does (lane (g, q) uses 32 contiguous bytes of token rows g
 // and g + 8 and of router row g of each n8 tile, in the same k order for A and
 // B); rows are padded by 16 bytes in shared memory so the fragment reads are
-// conflict-free.  At the tile's end the 15 partial logits are summed in warp
-// order (fixed, so the logits do not depend on timing) and the warps route
-// the 16 tokens with route_token (the bias and previous-layer logits of
-// their tokens loaded before the MMAs), while the producer already streams
-// the next tile.
-constexpr int RS_WARPS = 15;                   // consumer warps (16 warps in all: 4 per SM sub-partition)
+// conflict-free.  At the tile's end the 16 partial logits are summed in warp
+// order (fixed, so the logits do not depend on timing) and each warp routes
+// one token with route_token (its bias and previous-layer logits loaded
+// before the MMAs), while the producer already streams the next tile.
+constexpr int RS_WARPS = 16;                   // consumer warps
 constexpr int RS_THREADS = (RS_WARPS + 1) * 32;
 constexpr int RS_KC = 64 * RS_WARPS;           // d elements per chunk: one 64-wide slice per consumer warp
 constexpr int RS_PITCH = RS_KC * 2 + 16;       // bytes per staged row
@@ -584,7 +583,6 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
                 }
             }
         }
-        // (warp 0 also routes token 15, whose values it loads when routing it)
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
@@ -641,7 +639,6 @@ __global__ void __launch_bounds__(RS_THREADS, 1) router_stream_kernel(const Rout
         }
         rs_consumer_sync();
         if (t0 + warp < a.T) route_token(a, t0 + warp, zsum + warp * zpitch, lane, pre);
-        if (warp == 0 && t0 + 15 < a.T) route_token(a, t0 + 15, zsum + 15 * zpitch, lane);
         rs_consumer_sync();   // zsum and the partials are free for the next tile
     }
 }

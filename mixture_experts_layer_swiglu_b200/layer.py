@@ -79,10 +79,9 @@ class StageBuffers:
             self.y_sorted = torch.empty((max(cap, 1), d), dtype=f32, device=device)
         else:
             self.x_sorted = None
-            # c [T*k] fp32, then at a 256-byte boundary the shared branch's [T, d] fp32 output (full
-            # OmniMoE layer) and the combine's [T, d] fp32 accumulator
+            # c [T*k] fp32, then (full OmniMoE layer) the shared branch's [T, d] fp32 at a 256-byte boundary
             c_floats = (T * k * 4 + 255) // 256 * 64
-            self.y_sorted = torch.empty((max(c_floats + (desc.n_shared + 1) * T * d, 1),), dtype=f32, device=device)
+            self.y_sorted = torch.empty((max(c_floats + desc.n_shared * T * d, 1),), dtype=f32, device=device)
         self.workspace = torch.empty((abi.moe_workspace_size(desc),), dtype=torch.uint8, device=device)
         fw = abi.moe_fused_workspace_size(desc)        # -1: the fused expert step does not apply
         self.fused_workspace = torch.empty((fw,), dtype=torch.uint8, device=device) if fw > 0 else None
