@@ -52,7 +52,7 @@ constexpr int STAGE_BYTES = TILE_A + TILE_B;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 192;
-constexpr int SMEM_TABLE_INTS = 3 * kMaxGemmGroups + 1;
+constexpr int SMEM_TABLE_INTS = 3 * kMaxGemmGroups + 2;   // + the token-column schedule flag
 constexpr int EPI_STAGE_BYTES = 32 * 128;      // one 32-row x 128-byte output box per epilogue warp
 constexpr int EPI_WARPS = 4;
 __host__ __device__ constexpr int epi_stage_offset(int stage_bytes)
@@ -713,6 +713,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 #ifndef MOE_TN_SWIGLU_MIN_K
 #define MOE_TN_SWIGLU_MIN_K 2048
 #endif
+#ifndef MOE_TN_INTERLEAVE
+#define MOE_TN_INTERLEAVE 1
+#endif
 
 struct TnTile {
     int g;        // group
@@ -755,13 +758,37 @@ __device__ __forceinline__ TnTile decode_tn(int tile, const int* tile_start, con
     return ti;
 }
 
+// Schedule position s (tile s of the round-robin over n_clusters pairs) ->
+// tile id.  Plain: the identity (group, weight block, token tile order).
+// Mixed: the positions of each wave are dealt alternately from the front and
+// from the back of the tile list, and a pair alternates between the two from
+// one wave to the next.  With long-tail groups the front holds the head
+// experts' wide tiles (MMA-bound: N = 256 with the weight block shared by
+// several token tiles in L2) and the back the tail experts' narrow ones
+// (bound by streaming a weight block for N = 16..64 columns), so every wave
+// keeps both the tensor pipes and the DRAM busy instead of running the MMA
+// phase and then the streaming phase.  The token tiles of a weight block stay
+// next to one another in each half.  A bijection of [0, total): the front
+// takes tiles [0, F) in order and the back tiles [F, total) from the end,
+// where F is the number of front positions.
+__device__ __forceinline__ int tn_order(int s, int total, int n_clusters, bool mixed)
+{
+    if (!mixed) return s;
+    if (n_clusters & 1)   // odd: the position's parity alternates per pair and wave by itself
+        return (s & 1) ? total - 1 - (s >> 1) : (s >> 1);
+    const int half = n_clusters >> 1;
+    const int w = s / n_clusters, p = s - w * n_clusters;
+    const int f = (w & 1) ? (p >> 1) : ((p + 1) >> 1);   // front positions before p in wave w
+    return ((p + w) & 1) == 0 ? w * half + f : total - 1 - (w * half + (p - f));
+}
+
 __device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, int lane, int* tile_start,
-                                                     int* g_lo, int* g_cnt)
+                                                     int* g_lo, int* g_cnt, int* mixed)
 {
     const int n = a.n_groups;
     const int chunk = cdiv(n, 32);
     const int g0 = min(n, lane * chunk), g1 = min(n, g0 + chunk);
-    int local = 0;
+    int local = 0, wmin = 1 << 30, wmax = 0;
     for (int g = g0; g < g1; ++g) {
         int lo, hi;
         if (a.offsets) { lo = a.offsets[g]; hi = a.offsets[g + 1]; }
@@ -771,7 +798,12 @@ __device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, 
         g_lo[g] = lo;
         g_cnt[g] = cnt;
         local += tn_tiles(cnt, ntm);
+        if (cnt > 0) { wmin = min(wmin, tn_width(cnt)); wmax = max(wmax, tn_width(cnt)); }
     }
+    // groups whose tiles differ in width by 2x or more: the interleaved schedule
+    wmin = __reduce_min_sync(0xffffffffu, wmin);
+    wmax = __reduce_max_sync(0xffffffffu, wmax);
+    if (lane == 0) *mixed = MOE_TN_INTERLEAVE && wmax >= 2 * wmin;
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -865,6 +897,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     int* tile_start = reinterpret_cast<int*>(smem + P_STAGES * P_STAGE_BYTES + 256);
     int* g_lo = tile_start + (kMaxGemmGroups + 1);
     int* g_cnt = g_lo + kMaxGemmGroups;
+    int* sched_mixed = g_cnt + kMaxGemmGroups;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -872,7 +905,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     const bool leader = rank == 0;
     const int ntm = (EPI == EPI_SWIGLU) ? a.N / 128 : a.N / 256;   // weight blocks per expert
 
-    if (warp == 0) build_group_table_tn(a, ntm, lane, tile_start, g_lo, g_cnt);
+    if (warp == 0) build_group_table_tn(a, ntm, lane, tile_start, g_lo, g_cnt, sched_mixed);
     if (threadIdx.x == 32) {
         for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
@@ -893,6 +926,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     const int total = tile_start[a.n_groups];
     const int pnk = cdiv(a.K, BKE * P_KH);
     const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const bool mixed = *sched_mixed != 0;
     const uint32_t full_leader = mapa_shared(smem_u32(&full[0]), 0);
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
 
@@ -905,7 +939,8 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             uint32_t ph = 0;
             bool bad = false;
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
-                const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+                                            a.n_groups, ntm);
                 const bool first = ti.g < a.n_first;
                 const int gb = first ? ti.g : ti.g - a.n_first;
                 // A: weight rows of this CTA's half of M; B: this CTA's half of the tokens
@@ -973,7 +1008,8 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
             const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
-                const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+                                            a.n_groups, ntm);
                 const uint32_t idesc = FP8 ? idesc_e4m3_f32(P_BM, ti.nt) : idesc_bf16_f32(P_BM, ti.nt);
                 if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
@@ -1015,7 +1051,8 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
         int acc = 0;
         uint32_t aph = 0;
         for (int tile = cluster; tile < total; tile += n_clusters) {
-            const TnTile ti = decode_tn(tile, tile_start, g_lo, g_cnt, a.n_groups, ntm);
+            const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+                                            a.n_groups, ntm);
             bool ok = !*abort_flag && mbar_wait(&acc_full[acc], aph);
             if (EPI == EPI_SWIGLU) ok = team_all(ok, team);   // both warps of a team leave together
             if (!ok) { *abort_flag = 1; break; }
