@@ -95,11 +95,18 @@ __device__ __forceinline__ void store8(void* p, long long i8, const float (&v)[8
 // One token per group of CMB_SPLIT warps, each warp a contiguous quarter of
 // the row (more rows in flight per SM than one warp per token).
 constexpr int CMB_SPLIT = 4;
+#ifndef CMB_CHUNKS
+#define CMB_CHUNKS 1
+#endif
+#ifndef CMB_MINB
+#define CMB_MINB 4
+#endif
 
 template <typename T, typename TO>
-__global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
+__global__ void __launch_bounds__(256, CMB_MINB) combine_kernel(const CombineArgs a)
 {
     constexpr int V = 8;
+    constexpr int C = CMB_CHUNKS;                   // 8-element chunks per lane and step
     constexpr int WPB = 256 / 32;                    // warps per block
     constexpr int TPB = WPB / CMB_SPLIT;             // tokens per block
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -141,74 +148,91 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const CombineArgs a)
         }
         __syncthreads();
         if (live) {
-            // two chunks per lane and step: their row loads are independent
-            for (int i = i0 + lane; i < i1; i += 64) {
-                const bool two = i + 32 < i1;
-                float acc[2][V];
+            // CMB_CHUNKS chunks of 8 elements per lane and step; the slots are
+            // taken in pairs, the rows of both (expert output, or constant
+            // vector) loaded before either is added, so 2 CMB_CHUNKS independent
+            // 32-byte row loads per lane are in flight; the sum runs in slot order
+            for (int i = i0 + lane; i < i1; i += 32 * C) {
+                float acc[C][V];
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
+                for (int u = 0; u < C; ++u)
 #pragma unroll
                     for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
                 if (a.acc_rows && s_ffn[tib]) {      // the FFN slots' sum, formed by the down GEMM
-                    load8<float>(a.ys, t * vecs + i, acc[0]);
-                    if (two) load8<float>(a.ys, t * vecs + i + 32, acc[1]);
+                    for (int u = 0; u < C; ++u)
+                        if (i + 32 * u < i1) load8<float>(a.ys, t * vecs + i + 32 * u, acc[u]);
                 }
                 for (int s = 0; s < a.n_shared; ++s) {
                     const long long r = (long long)a.offsets[a.n_ffn + s] + t;
                     if (r < a.rows_cap) {
-                        float w[2][V];
-                        load8<float>(a.ys, r * vecs + i, w[0]);
-                        if (two) load8<float>(a.ys, r * vecs + i + 32, w[1]);
+                        float w[C][V];
+                        for (int u = 0; u < C; ++u)
+                            if (i + 32 * u < i1) load8<float>(a.ys, r * vecs + i + 32 * u, w[u]);
 #pragma unroll
-                        for (int u = 0; u < 2; ++u)
+                        for (int u = 0; u < C; ++u)
 #pragma unroll
                             for (int v = 0; v < V; ++v) acc[u][v] += w[u][v];
                     }
                 }
                 bool have_x = false;
-                float xv[2][V];
-                for (int j = 0; j < a.k; ++j) {
-                    const int e = s_e[tib][j];
-                    const float g = s_g[tib][j];
-                    if (e < 0) continue;
-                    if (e < zero0) {
-                        if (a.acc_rows) continue;         // already in the accumulator row
-                        const long long rb = (long long)s_r[tib][j] * vecs;
-                        float w[2][V];
-                        load8<float>(a.ys, rb + i, w[0]);
-                        if (two) load8<float>(a.ys, rb + i + 32, w[1]);
+                float xv[C][V];
+                for (int j0 = 0; j0 < a.k; j0 += 2) {
+                    float pw[2][C][V];                       // slot j0 + p: its row (FFN output or constant vector)
 #pragma unroll
-                        for (int u = 0; u < 2; ++u)
-#pragma unroll
-                            for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, w[u][v], acc[u][v]);
-                    } else if (e < copy0) {
-                        // zero expert: contributes nothing
-                    } else {
-                        if (!have_x) {
-                            load8<T>(a.x, t * vecs + i, xv[0]);
-                            if (two) load8<T>(a.x, t * vecs + i + 32, xv[1]);
-                            have_x = true;
+                    for (int p = 0; p < 2; ++p) {
+                        const int j = j0 + p;
+                        const int e = j < a.k ? s_e[tib][j] : -1;
+                        if (e < 0) continue;
+                        if (e < zero0) {
+                            if (!a.acc_rows) {
+                                const long long rb = (long long)s_r[tib][j] * vecs;
+                                for (int u = 0; u < C; ++u)
+                                    if (i + 32 * u < i1) load8<float>(a.ys, rb + i + 32 * u, pw[p][u]);
+                            }
+                        } else if (e >= copy0) {             // copy and constant experts read x
+                            if (!have_x) {
+                                for (int u = 0; u < C; ++u)
+                                    if (i + 32 * u < i1) load8<T>(a.x, t * vecs + i + 32 * u, xv[u]);
+                                have_x = true;
+                            }
+                            if (e >= const0) {
+                                const long long cb = (long long)(e - const0) * vecs;
+                                for (int u = 0; u < C; ++u)
+                                    if (i + 32 * u < i1) load8<T>(a.const_vec, cb + i + 32 * u, pw[p][u]);
+                            }
                         }
-                        if (e < const0) {
+                    }
 #pragma unroll
-                            for (int u = 0; u < 2; ++u)
+                    for (int p = 0; p < 2; ++p) {
+                        const int j = j0 + p;
+                        const int e = j < a.k ? s_e[tib][j] : -1;
+                        if (e < 0) continue;
+                        const float g = s_g[tib][j];
+                        if (e < zero0) {
+                            if (a.acc_rows) continue;            // already in the accumulator row
+#pragma unroll
+                            for (int u = 0; u < C; ++u)
+#pragma unroll
+                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, pw[p][u][v], acc[u][v]);
+                        } else if (e < copy0) {
+                            // zero expert: contributes nothing
+                        } else if (e < const0) {
+#pragma unroll
+                            for (int u = 0; u < C; ++u)
 #pragma unroll
                                 for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, xv[u][v], acc[u][v]);
                         } else {
                             const float a1 = s_a1[tib][j], a2 = s_a2[tib][j];
-                            const long long cb = (long long)(e - const0) * vecs;
-                            float cv[2][V];
-                            load8<T>(a.const_vec, cb + i, cv[0]);
-                            if (two) load8<T>(a.const_vec, cb + i + 32, cv[1]);
 #pragma unroll
-                            for (int u = 0; u < 2; ++u)
+                            for (int u = 0; u < C; ++u)
 #pragma unroll
-                                for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, a1 * xv[u][v] + a2 * cv[u][v], acc[u][v]);
+                                for (int v = 0; v < V; ++v)
+                                    acc[u][v] = fmaf(g, a1 * xv[u][v] + a2 * pw[p][u][v], acc[u][v]);
                         }
                     }
                 }
-                store8<TO>(a.y, t * vecs + i, acc[0]);
-                if (two) store8<TO>(a.y, t * vecs + i + 32, acc[1]);
+                for (int u = 0; u < C; ++u)
+                    if (i + 32 * u < i1) store8<TO>(a.y, t * vecs + i + 32 * u, acc[u]);
             }
         }
         __syncthreads();

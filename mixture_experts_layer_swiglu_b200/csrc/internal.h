@@ -120,6 +120,7 @@ struct PermuteArgs {
     int32_t* ws_blocksum; // atomic scan: [scan blocks]
     int T, k, d, n_ffn, n_shared, n_ids, elt_bytes;
     float* xs_scale;      // non-null: x_sorted gets e4m3 codes of the rows and these their scales
+    unsigned* bar;        // SwiGLU: grid-barrier counter of the one-launch form (null: the four kernels)
 };
 moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st);
 moe_status launch_permute_atomic(const PermuteArgs& a, cudaStream_t st);

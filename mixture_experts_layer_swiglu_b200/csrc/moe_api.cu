@@ -122,7 +122,8 @@ Scratch scratch_sizes(const moe_layer_desc* d)
     Scratch s{0, 0, 0};
     const long long cap = moe_row_capacity(d);
     if (d->kind == MOE_EXPERT_SWIGLU) {
-        s.permute = al((size_t)permute_blocks(d->T) * std::max(d->n_ffn, 1) * 4);
+        // the counts of every 256-token chunk and expert, then the grid-barrier counter
+        s.permute = al((size_t)permute_blocks(d->T) * std::max(d->n_ffn, 1) * 4) + 256;
         s.ffn = (d->n_ffn + d->n_shared > 0) ? al((size_t)cap * d->hidden * elt(d)) : 0;
         if (d->expert_fp8 && s.ffn)   // h (bf16), then its e4m3 codes and row scales
             s.ffn += al((size_t)cap * d->hidden) + al((size_t)cap * 4);
@@ -354,6 +355,8 @@ moe_status permute_impl(const moe_layer_desc* d, const int32_t* idx, const void*
         if (xs && d->expert_fp8)   // e4m3 codes of the rows, then their scales
             a.xs_scale = reinterpret_cast<float*>(static_cast<char*>(xs) + al((size_t)moe_row_capacity(d) * d->d_model));
         a.ws_counts = static_cast<int32_t*>(ws);
+        a.bar = reinterpret_cast<unsigned*>(static_cast<char*>(ws) +
+                                            al((size_t)permute_blocks(d->T) * std::max(d->n_ffn, 1) * 4));
         a.n_ffn = d->n_ffn;
         a.n_shared = d->n_shared;
         a.n_ids = n_router_rows(d);

@@ -235,6 +235,171 @@ __device__ __forceinline__ int ap_block_sum(int v, int* red)
     return t;
 }
 
+// ---- the SwiGLU-kind permutation in one cooperative kernel
+//
+// The same count / scan / scatter steps as the kernels above, in one launch
+// (every block resident, two grid barriers), with the gather turned around:
+// each block takes an equal range of tokens, rebuilds the expert masks of the
+// 256-token chunks its range touches, places its tokens' tasks, and copies
+// each of its tokens' x row once from HBM into all its destination rows (the
+// token's FFN slots and the shared experts' rows), 16-byte vectors, eight in
+// flight per lane.  The small steps then cost no launch of their own and the
+// row copies start as soon as the offsets exist.
+constexpr int PF_THREADS = 512;
+constexpr int PF_MAXDST = 8;        // destination rows per token held in shared memory (k + n_shared)
+
+// Expert masks of chunk c (threads < P_TOK each take one token); false on a bad id.
+__device__ __forceinline__ bool pf_masks(const PermuteArgs& a, uint32_t (*mask)[8], int c)
+{
+    for (int i = threadIdx.x; i < a.n_ffn * 8; i += blockDim.x) mask[i >> 3][i & 7] = 0u;
+    __syncthreads();
+    bool ok = true;
+    const int t = c * P_TOK + threadIdx.x;
+    if (threadIdx.x < P_TOK && t < a.T) {
+        for (int j = 0; j < a.k; ++j) {
+            const int e = a.idx[(long long)t * a.k + j];
+            if (e < 0 || e >= a.n_ids) { ok = false; continue; }
+            if (e < a.n_ffn) {
+                const uint32_t bit = 1u << (threadIdx.x & 31);
+                const uint32_t old = atomicOr(&mask[e][threadIdx.x >> 5], bit);
+                if (old & bit) ok = false;      // same expert twice in one token
+            }
+        }
+    }
+    __syncthreads();
+    return ok;
+}
+
+__global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const PermuteArgs a, unsigned* bar, int nb)
+{
+    __shared__ uint32_t mask[P_MAXE][8];
+    __shared__ int s_dst[P_TOK][PF_MAXDST];        // destination rows of the chunk-range's tokens
+    __shared__ int warp_tot[32];
+    __shared__ int s_total, s_ok;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = PF_THREADS / 32;
+
+    // 1. counts of chunk c in [blocks x experts]
+    for (int c = blockIdx.x; c < nb; c += gridDim.x) {
+        if (!pf_masks(a, mask, c)) set_status(MOE_ERR_DEVICE_BOUNDS);
+        for (int e = tid; e < a.n_ffn; e += PF_THREADS) {
+            int n = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) n += __popc(mask[e][w]);
+            a.ws_counts[(long long)c * a.n_ffn + e] = n;
+        }
+        __syncthreads();   // the masks are rebuilt for the next chunk
+    }
+    if (!ap_grid_sync(bar, 1, &s_ok)) return;
+
+    // 2. block 0: exclusive scan in (expert, chunk) order, in place; the offsets
+    if (blockIdx.x == 0) {
+        const long long L = (long long)a.n_ffn * nb;
+        const long long per = (L + PF_THREADS - 1) / PF_THREADS;
+        const long long lo = std::min<long long>(L, tid * per), hi = std::min<long long>(L, lo + per);
+        int s = 0;
+        for (long long l = lo; l < hi; ++l) s += a.ws_counts[(l % nb) * a.n_ffn + l / nb];
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = lane < NW ? warp_tot[lane] : 0;
+            int wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += v;
+            }
+            if (lane < NW) warp_tot[lane] = wi - w;
+            if (lane == 31) s_total = wi;
+        }
+        __syncthreads();
+        int base = warp_tot[warp] + incl - s;
+        for (long long l = lo; l < hi; ++l) {
+            const long long e = l / nb, c = l % nb;
+            const long long ix = c * a.n_ffn + e;
+            const int n = a.ws_counts[ix];
+            a.ws_counts[ix] = base;
+            if (c == 0) a.offsets[e] = base;
+            base += n;
+        }
+        if (nb == 0)
+            for (int e = tid; e < a.n_ffn; e += PF_THREADS) a.offsets[e] = 0;
+        if (tid == 0) {
+            const int R = nb == 0 ? 0 : s_total;
+            a.offsets[a.n_ffn] = R;
+            for (int sh = 0; sh < a.n_shared; ++sh) a.offsets[a.n_ffn + sh + 1] = R + (sh + 1) * a.T;
+        }
+    }
+    if (!ap_grid_sync(bar, 2, &s_ok)) return;
+
+    // 3. this block's tokens: their rows, then the row copies
+    const int tpb = cdiv(a.T, gridDim.x);
+    const int lo = min(a.T, (int)blockIdx.x * tpb), hi = min(a.T, lo + tpb);
+    const int R = a.offsets[a.n_ffn];
+    const int ndst = a.k + a.n_shared;
+    const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
+    const int vecs = a.d * a.elt_bytes / 16;
+    const uint4* x = reinterpret_cast<const uint4*>(a.x);
+    uint4* xs = reinterpret_cast<uint4*>(a.x_sorted);
+    for (int c = lo / P_TOK; c * P_TOK < hi; ++c) {
+        pf_masks(a, mask, c);
+        const int t0 = max(lo, c * P_TOK), t1 = min(hi, c * P_TOK + P_TOK);
+        const int t = c * P_TOK + tid;
+        if (tid < P_TOK && t >= t0 && t < t1) {
+            const int w = tid >> 5;
+            const uint32_t below = (1u << (tid & 31)) - 1u;
+            for (int j = 0; j < a.k; ++j) {
+                const int e = a.idx[(long long)t * a.k + j];
+                int r = -1;
+                if (e >= 0 && e < a.n_ffn) {
+                    r = a.ws_counts[(long long)c * a.n_ffn + e];
+                    for (int ww = 0; ww < w; ++ww) r += __popc(mask[e][ww]);
+                    r += __popc(mask[e][w] & below);
+                    a.token_of[r] = t;
+                }
+                a.row_of[(long long)t * a.k + j] = r;
+                if (j < PF_MAXDST) s_dst[tid][j] = r;
+            }
+            for (int sh = 0; sh < a.n_shared; ++sh) {
+                const long long r = (long long)R + (long long)sh * a.T + t;
+                a.token_of[r] = t;
+                if (a.k + sh < PF_MAXDST) s_dst[tid][a.k + sh] = (int)r;
+            }
+        }
+        __syncthreads();
+        if (xs) {
+            // one warp per token: each 16-byte vector of x[t] is read once and
+            // stored to every destination row
+            for (int tt = t0 + warp; tt < t1; tt += NW) {
+                const int ti = tt - c * P_TOK;
+                const uint4* src = x + (long long)tt * vecs;
+                for (int i0 = 0; i0 < vecs; i0 += 32 * 8) {
+                    uint4 v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (i0 + u * 32 + lane < vecs) v[u] = __ldg(src + i0 + u * 32 + lane);
+                    for (int j = 0; j < ndst && j < PF_MAXDST; ++j) {
+                        const int r = s_dst[ti][j];
+                        if (r < 0) continue;
+                        if (r >= rows_cap) { if (lane == 0) set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
+                        uint4* dst = xs + (long long)r * vecs;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if (i0 + u * 32 + lane < vecs) dst[i0 + u * 32 + lane] = v[u];
+                    }
+                }
+            }
+        }
+        __syncthreads();   // s_dst and the masks are rebuilt for the next chunk
+    }
+}
+
 __global__ void __launch_bounds__(AP_THREADS) atomic_permute_kernel(const PermuteArgs a, unsigned* bar)
 {
     __shared__ int red[AP_THREADS / 32];
@@ -328,10 +493,45 @@ int permute_blocks(int T) { return std::max(1, cdiv(T, P_TOK)); }
 // ints after the counts in the atomic kind's workspace: the block totals, then the barrier counter
 int atomic_scan_blocks(int N) { (void)N; return AP_MAX_BLOCKS + 64; }
 
+// Blocks of the fused kernel that are resident together (0 if none fit).
+static int pf_grid()
+{
+    static int per_sm[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (per_sm[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, perm_fused_kernel, PF_THREADS, 0) != cudaSuccess) n = 0;
+        per_sm[dev] = n > 0 ? n : -1;
+    }
+    return per_sm[dev] > 0 ? std::min(per_sm[dev], 2) * num_sms() : 0;
+}
+
 moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
 {
     if (a.n_ffn > P_MAXE) return MOE_ERR_UNSUPPORTED;
     const int nb = permute_blocks(a.T);
+    const int grid = a.bar && a.T > 0 && a.k + a.n_shared <= PF_MAXDST ? pf_grid() : 0;
+    if (grid > 0) {   // one cooperative launch (its barrier counter zeroed first)
+        cudaError_t e = cudaMemsetAsync(a.bar, 0, sizeof(unsigned), st);
+        if (e != cudaSuccess) return cuda_status(e);
+        PermuteArgs args = a;
+        if (a.xs_scale) args.x_sorted = nullptr;   // e4m3 rows: the quantizing gather below writes them
+        unsigned* bar = a.bar;
+        int nbv = nb;
+        void* params[3] = {&args, &bar, &nbv};
+        e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(perm_fused_kernel), dim3(grid), dim3(PF_THREADS),
+                                        params, 0, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        count_launch();
+        if (a.x_sorted && a.xs_scale) {
+            const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
+            moe_status s = launch_gather_quant(a.token_of, a.offsets, a.n_ffn + a.n_shared, a.x, a.d, a.T, a.x_sorted,
+                                               a.xs_scale, rows_cap, st);
+            if (s != MOE_OK) return s;
+        }
+        return cuda_status(cudaGetLastError());
+    }
     if (a.T > 0 && a.n_ffn > 0) {
         perm_count_kernel<<<nb, P_TOK, 0, st>>>(a);
         count_launch();
