@@ -194,6 +194,10 @@ MOE_API moe_status moe_route(const moe_layer_desc* desc, const moe_layer_weights
  *   expert_offsets[groups] are untouched.
  * An id outside [0, n_ffn + n_zero + n_copy + n_const) (or the atomic grid)
  * sets MOE_ERR_DEVICE_BOUNDS in the device status and is skipped.
+ * Both kinds run as a cooperative launch (every block resident, grid barriers
+ * on a counter in the workspace, cleared first on `stream`; each wait bounded,
+ * MOE_ERR_TIMEOUT in the device status if one gives up), so two calls must
+ * not share a workspace while both may run.
  */
 MOE_API moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x,
                        int32_t* expert_offsets, int32_t* row_of, int32_t* token_of,
