@@ -210,7 +210,7 @@ __device__ __forceinline__ bool ap_grid_sync(unsigned* bar, unsigned phase, int*
         for (uint32_t i = 0;; ++i) {
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
             if (v >= target) break;
-            __nanosleep(64);                                // back off: every block polls one line
+            if (i >= 32) __nanosleep(64);                   // then back off: every block polls one line
             if ((i & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) { ok = false; break; }
         }
         if (!ok) set_status(MOE_ERR_TIMEOUT);
@@ -238,15 +238,19 @@ __device__ __forceinline__ int ap_block_sum(int v, int* red)
 // ---- the SwiGLU-kind permutation in one cooperative kernel
 //
 // The same count / scan / scatter steps as the kernels above, in one launch
-// (every block resident, two grid barriers), with the gather turned around:
-// each block takes an equal range of tokens, rebuilds the expert masks of the
-// 256-token chunks its range touches, places its tokens' tasks, and copies
-// each of its tokens' x row once from HBM into all its destination rows (the
-// token's FFN slots and the shared experts' rows), 16-byte vectors, eight in
-// flight per lane.  The small steps then cost no launch of their own and the
-// row copies start as soon as the offsets exist.
+// (every block resident, one grid barrier after the counts), with the scan
+// done by every block for itself (it reads all [chunks x experts] counts and
+// keeps the bases of the chunks it places: no second barrier) and the gather
+// turned around: each block takes an equal range of tokens, rebuilds the
+// expert masks of the 256-token chunks its range touches, places its tokens'
+// tasks, and copies each of its tokens' x row once from HBM into all its
+// destination rows (the token's FFN slots and the shared experts' rows),
+// 16-byte vectors, eight in flight per lane.  The small steps then cost no
+// launch of their own and the row copies start right after the barrier.
 constexpr int PF_THREADS = 512;
 constexpr int PF_MAXDST = 8;        // destination rows per token held in shared memory (k + n_shared)
+constexpr int PF_MAXCOUNTS = 16384; // [chunks x experts] counts that every block reads
+static_assert(P_TOK * PF_MAXDST >= 2 * P_MAXE, "per-expert sums share s_dst's storage");
 
 // Expert masks of chunk c (threads < P_TOK each take one token); false on a bad id.
 __device__ __forceinline__ bool pf_masks(const PermuteArgs& a, uint32_t (*mask)[8], int c)
@@ -270,12 +274,38 @@ __device__ __forceinline__ bool pf_masks(const PermuteArgs& a, uint32_t (*mask)[
     return ok;
 }
 
+// Exclusive prefix of v over the block's threads in thread order, and the
+// block total in *total (all threads).
+__device__ __forceinline__ int pf_block_scan(int v, int* warp_tot, int* total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    __syncthreads();                        // warp_tot of an earlier call read by everyone
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < PF_THREADS / 32; ++w) {
+        const int x = warp_tot[w];
+        before += w < warp ? x : 0;
+        all += x;
+    }
+    *total = all;
+    return before + incl - v;
+}
+
 __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const PermuteArgs a, unsigned* bar, int nb)
 {
     __shared__ uint32_t mask[P_MAXE][8];
     __shared__ int s_dst[P_TOK][PF_MAXDST];        // destination rows of the chunk-range's tokens
+    __shared__ int sbase[P_MAXE];                  // next row of each expert's tasks
     __shared__ int warp_tot[32];
-    __shared__ int s_total, s_ok;
+    __shared__ int s_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = PF_THREADS / 32;
 
@@ -292,56 +322,56 @@ __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const Permute
     }
     if (!ap_grid_sync(bar, 1, &s_ok)) return;
 
-    // 2. block 0: exclusive scan in (expert, chunk) order, in place; the offsets
-    if (blockIdx.x == 0) {
-        const long long L = (long long)a.n_ffn * nb;
-        const long long per = (L + PF_THREADS - 1) / PF_THREADS;
-        const long long lo = std::min<long long>(L, tid * per), hi = std::min<long long>(L, lo + per);
-        int s = 0;
-        for (long long l = lo; l < hi; ++l) s += a.ws_counts[(l % nb) * a.n_ffn + l / nb];
-        int incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int w = lane < NW ? warp_tot[lane] : 0;
-            int wi = w;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, wi, o);
-                if (lane >= o) wi += v;
+    // 2. every block: from all the counts, the row at which each expert's
+    //    tasks of the first chunk it places begin (the exclusive sum in
+    //    (expert, chunk) order); block 0 also writes the offsets
+    const int tpb = cdiv(a.T, gridDim.x);
+    const int lo = min(a.T, (int)blockIdx.x * tpb), hi = min(a.T, lo + tpb);
+    const int cfirst = lo / P_TOK;
+    // per expert, its total and its count before chunk cfirst: every thread
+    // adds a strided share of the counts with shared-memory integer atomics
+    // (into s_dst's storage, free until the placement)
+    int* tot_s = &s_dst[0][0];
+    int* cum_s = tot_s + P_MAXE;
+    for (int e = tid; e < a.n_ffn; e += PF_THREADS) { tot_s[e] = 0; cum_s[e] = 0; }
+    __syncthreads();
+    {
+        const int L = nb * a.n_ffn;
+        const int lim = cfirst * a.n_ffn;          // entries of the chunks before cfirst
+#pragma unroll 4
+        for (int l = tid; l < L; l += PF_THREADS) {
+            const int v = a.ws_counts[l];
+            const int e = l % a.n_ffn;
+            if (v) {
+                atomicAdd(&tot_s[e], v);
+                if (l < lim) atomicAdd(&cum_s[e], v);
             }
-            if (lane < NW) warp_tot[lane] = wi - w;
-            if (lane == 31) s_total = wi;
         }
-        __syncthreads();
-        int base = warp_tot[warp] + incl - s;
-        for (long long l = lo; l < hi; ++l) {
-            const long long e = l / nb, c = l % nb;
-            const long long ix = c * a.n_ffn + e;
-            const int n = a.ws_counts[ix];
-            a.ws_counts[ix] = base;
-            if (c == 0) a.offsets[e] = base;
-            base += n;
-        }
-        if (nb == 0)
-            for (int e = tid; e < a.n_ffn; e += PF_THREADS) a.offsets[e] = 0;
+    }
+    __syncthreads();
+    int tot[2] = {0, 0}, cum[2] = {0, 0};       // experts tid and tid + PF_THREADS
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int e = tid + u * PF_THREADS;
+        if (e < a.n_ffn) { tot[u] = tot_s[e]; cum[u] = cum_s[e]; }
+    }
+    int tot0, tot1;
+    const int ex0 = pf_block_scan(tot[0], warp_tot, &tot0);
+    const int ex1 = pf_block_scan(tot[1], warp_tot, &tot1) + tot0;
+    const int R = tot0 + tot1;                  // rows of the FFN experts
+    if (tid < a.n_ffn) sbase[tid] = ex0 + cum[0];
+    if (tid + PF_THREADS < a.n_ffn) sbase[tid + PF_THREADS] = ex1 + cum[1];
+    if (blockIdx.x == 0) {
+        if (tid < a.n_ffn) a.offsets[tid] = ex0;
+        if (tid + PF_THREADS < a.n_ffn) a.offsets[tid + PF_THREADS] = ex1;
         if (tid == 0) {
-            const int R = nb == 0 ? 0 : s_total;
             a.offsets[a.n_ffn] = R;
             for (int sh = 0; sh < a.n_shared; ++sh) a.offsets[a.n_ffn + sh + 1] = R + (sh + 1) * a.T;
         }
     }
-    if (!ap_grid_sync(bar, 2, &s_ok)) return;
+    __syncthreads();
 
     // 3. this block's tokens: their rows, then the row copies
-    const int tpb = cdiv(a.T, gridDim.x);
-    const int lo = min(a.T, (int)blockIdx.x * tpb), hi = min(a.T, lo + tpb);
-    const int R = a.offsets[a.n_ffn];
     const int ndst = a.k + a.n_shared;
     const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
     const int vecs = a.d * a.elt_bytes / 16;
@@ -358,7 +388,7 @@ __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const Permute
                 const int e = a.idx[(long long)t * a.k + j];
                 int r = -1;
                 if (e >= 0 && e < a.n_ffn) {
-                    r = a.ws_counts[(long long)c * a.n_ffn + e];
+                    r = sbase[e];
                     for (int ww = 0; ww < w; ++ww) r += __popc(mask[e][ww]);
                     r += __popc(mask[e][w] & below);
                     a.token_of[r] = t;
@@ -373,6 +403,13 @@ __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const Permute
             }
         }
         __syncthreads();
+        // the next chunk's tasks of expert e begin after this chunk's
+        for (int e = tid; e < a.n_ffn; e += PF_THREADS) {
+            int n = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) n += __popc(mask[e][w]);
+            sbase[e] += n;
+        }
         if (xs) {
             // one warp per token: each 16-byte vector of x[t] is read once and
             // stored to every destination row
@@ -511,8 +548,10 @@ moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
 {
     if (a.n_ffn > P_MAXE) return MOE_ERR_UNSUPPORTED;
     const int nb = permute_blocks(a.T);
-    const int grid = a.bar && a.T > 0 && a.k + a.n_shared <= PF_MAXDST ? pf_grid() : 0;
-    if (grid > 0) {   // one cooperative launch (its barrier counter zeroed first)
+    // (every block reads all the counts: the one-launch form is for up to PF_MAXCOUNTS of them)
+    const int grid = a.bar && a.T > 0 && a.k + a.n_shared <= PF_MAXDST && (long long)nb * a.n_ffn <= PF_MAXCOUNTS
+                         ? pf_grid() : 0;
+    if (grid > 0) {   // one cooperative launch (its barrier counter cleared first)
         cudaError_t e = cudaMemsetAsync(a.bar, 0, sizeof(unsigned), st);
         if (e != cudaSuccess) return cuda_status(e);
         PermuteArgs args = a;
