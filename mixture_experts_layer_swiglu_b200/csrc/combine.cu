@@ -95,18 +95,14 @@ __device__ __forceinline__ void store8(void* p, long long i8, const float (&v)[8
 // One token per group of CMB_SPLIT warps, each warp a contiguous quarter of
 // the row (more rows in flight per SM than one warp per token).
 constexpr int CMB_SPLIT = 4;
-#ifndef CMB_CHUNKS
-#define CMB_CHUNKS 1
-#endif
-#ifndef CMB_MINB
-#define CMB_MINB 4
-#endif
 
-template <typename T, typename TO>
-__global__ void __launch_bounds__(256, CMB_MINB) combine_kernel(const CombineArgs a)
+// C: 8-element chunks per lane and step; BYP: the layer has zero-computation
+// experts (without them the x and constant-vector paths are compiled out and
+// the registers go to more loads in flight).
+template <typename T, typename TO, int C, int MINB, bool BYP>
+__global__ void __launch_bounds__(256, MINB) combine_kernel(const CombineArgs a)
 {
     constexpr int V = 8;
-    constexpr int C = CMB_CHUNKS;                   // 8-element chunks per lane and step
     constexpr int WPB = 256 / 32;                    // warps per block
     constexpr int TPB = WPB / CMB_SPLIT;             // tokens per block
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -148,9 +144,9 @@ __global__ void __launch_bounds__(256, CMB_MINB) combine_kernel(const CombineArg
         }
         __syncthreads();
         if (live) {
-            // CMB_CHUNKS chunks of 8 elements per lane and step; the slots are
+            // C chunks of 8 elements per lane and step; the slots are
             // taken in pairs, the rows of both (expert output, or constant
-            // vector) loaded before either is added, so 2 CMB_CHUNKS independent
+            // vector) loaded before either is added, so 2 C independent
             // 32-byte row loads per lane are in flight; the sum runs in slot order
             for (int i = i0 + lane; i < i1; i += 32 * C) {
                 float acc[C][V];
@@ -189,7 +185,7 @@ __global__ void __launch_bounds__(256, CMB_MINB) combine_kernel(const CombineArg
                                 for (int u = 0; u < C; ++u)
                                     if (i + 32 * u < i1) load8<float>(a.ys, rb + i + 32 * u, pw[p][u]);
                             }
-                        } else if (e >= copy0) {             // copy and constant experts read x
+                        } else if (BYP && e >= copy0) {      // copy and constant experts read x
                             if (!have_x) {
                                 for (int u = 0; u < C; ++u)
                                     if (i + 32 * u < i1) load8<T>(a.x, t * vecs + i + 32 * u, xv[u]);
@@ -214,7 +210,7 @@ __global__ void __launch_bounds__(256, CMB_MINB) combine_kernel(const CombineArg
                             for (int u = 0; u < C; ++u)
 #pragma unroll
                                 for (int v = 0; v < V; ++v) acc[u][v] = fmaf(g, pw[p][u][v], acc[u][v]);
-                        } else if (e < copy0) {
+                        } else if (!BYP || e < copy0) {
                             // zero expert: contributes nothing
                         } else if (e < const0) {
 #pragma unroll
@@ -619,9 +615,13 @@ moe_status launch_combine(int dtype, const CombineArgs& a, cudaStream_t st)
     if (a.T == 0) return MOE_OK;
     if (a.k > CMB_MAXK) return MOE_ERR_UNSUPPORTED;
     const int grid = std::max(1, std::min(cdiv(a.T, 256 / 32 / CMB_SPLIT), num_sms() * 16));
-    if (dtype == MOE_BF16 && !a.out_f32) combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
-    else if (dtype == MOE_BF16) combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(a);
-    else combine_kernel<float, float><<<grid, 256, 0, st>>>(a);
+    // FFN slots only (no zero-computation experts, no shared rows): two chunks per lane
+    // (measured on the Mixtral-shaped layer: 38.4 -> 37.0 us; with shared rows it did not gain)
+    const bool ffn_only = a.n_zero + a.n_copy + a.n_const == 0 && a.n_shared == 0;
+    if (dtype == MOE_BF16 && !a.out_f32 && ffn_only) combine_kernel<__nv_bfloat16, __nv_bfloat16, 2, 3, false><<<grid, 256, 0, st>>>(a);
+    else if (dtype == MOE_BF16 && !a.out_f32) combine_kernel<__nv_bfloat16, __nv_bfloat16, 1, 4, true><<<grid, 256, 0, st>>>(a);
+    else if (dtype == MOE_BF16) combine_kernel<__nv_bfloat16, float, 1, 4, true><<<grid, 256, 0, st>>>(a);
+    else combine_kernel<float, float, 1, 4, true><<<grid, 256, 0, st>>>(a);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
