@@ -52,7 +52,7 @@ constexpr int STAGE_BYTES = TILE_A + TILE_B;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 192;
-constexpr int SMEM_TABLE_INTS = 3 * kMaxGemmGroups + 2;   // + the token-column schedule flag
+constexpr int SMEM_TABLE_INTS = 4 * kMaxGemmGroups + 2;   // + the token-column tile widths and schedule flag
 constexpr int EPI_STAGE_BYTES = 32 * 128;      // one 32-row x 128-byte output box per epilogue warp
 constexpr int EPI_WARPS = 4;
 __host__ __device__ constexpr int epi_stage_offset(int stage_bytes)
@@ -716,6 +716,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 #ifndef MOE_TN_INTERLEAVE
 #define MOE_TN_INTERLEAVE 1
 #endif
+#ifndef MOE_TN_FILL
+#define MOE_TN_FILL 1
+#endif
 
 struct TnTile {
     int g;        // group
@@ -731,13 +734,14 @@ __device__ __forceinline__ int tn_width(int cnt)
     return (cdiv(cnt, t) + 15) & ~15;
 }
 
-__device__ __forceinline__ int tn_tiles(int cnt, int ntm)
+// Token-tile width of a group of cnt rows cut into t tiles (t >= ceil(cnt / 256)).
+__device__ __forceinline__ int tn_width_t(int cnt, int t)
 {
-    return cnt > 0 ? cdiv(cnt, tn_width(cnt)) * ntm : 0;
+    return (cdiv(cnt, t) + 15) & ~15;
 }
 
 __device__ __forceinline__ TnTile decode_tn(int tile, const int* tile_start, const int* g_lo, const int* g_cnt,
-                                            int n_groups, int ntm)
+                                            const int* g_w, int n_groups, int ntm)
 {
     int lo = 0, hi = n_groups - 1;   // last g with tile_start[g] <= tile
     while (lo < hi) {
@@ -747,7 +751,7 @@ __device__ __forceinline__ TnTile decode_tn(int tile, const int* tile_start, con
     TnTile ti;
     ti.g = lo;
     const int cnt = g_cnt[lo];
-    const int w = tn_width(cnt);
+    const int w = g_w[lo];
     const int nj = cdiv(cnt, w);
     const int local = tile - tile_start[lo];
     ti.m = local / nj;
@@ -782,8 +786,18 @@ __device__ __forceinline__ int tn_order(int s, int total, int n_clusters, bool m
     return ((p + w) & 1) == 0 ? w * half + f : total - 1 - (w * half + (p - f));
 }
 
-__device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, int lane, int* tile_start,
-                                                     int* g_lo, int* g_cnt, int* mixed)
+// Warp 0 builds the token-column tile table: each group's first row, row
+// count and token-tile width, the first tile of each group, and the schedule
+// flag.  A group of c rows starts with ceil(c / 256) token tiles of one width
+// (tn_width).  When the groups are alike (not mixed), the round-robin's last
+// wave is then often a fraction of the pairs (Mixtral-shaped down GEMM: 608
+// tiles of 208-256 columns on 74 pairs, 8.2 waves), so token tiles are added
+// one at a time to the group whose tiles are widest for as long as the tile
+// count stays within the same number of waves: the waves fill up with tiles
+// of nearly equal width (656 tiles of 176-256 columns) and the pairs finish
+// together.  The MMA columns stay those of the rows, rounded to 16 per tile.
+__device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, int n_clusters, int lane,
+                                                     int* tile_start, int* g_lo, int* g_cnt, int* g_w, int* mixed)
 {
     const int n = a.n_groups;
     const int chunk = cdiv(n, 32);
@@ -797,13 +811,48 @@ __device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, 
         if (cnt < 0 || lo < 0) { set_status(MOE_ERR_DEVICE_BOUNDS); cnt = 0; lo = 0; }
         g_lo[g] = lo;
         g_cnt[g] = cnt;
-        local += tn_tiles(cnt, ntm);
         if (cnt > 0) { wmin = min(wmin, tn_width(cnt)); wmax = max(wmax, tn_width(cnt)); }
     }
     // groups whose tiles differ in width by 2x or more: the interleaved schedule
     wmin = __reduce_min_sync(0xffffffffu, wmin);
     wmax = __reduce_max_sync(0xffffffffu, wmax);
-    if (lane == 0) *mixed = MOE_TN_INTERLEAVE && wmax >= 2 * wmin;
+    const bool mix = MOE_TN_INTERLEAVE && wmax >= 2 * wmin;
+    if (lane == 0) *mixed = mix;
+    // token tiles per group (kept in g_w until the widths are set)
+    int tsum = 0;
+    for (int g = g0; g < g1; ++g) {
+        const int t = g_cnt[g] > 0 ? cdiv(g_cnt[g], 256) : 0;
+        g_w[g] = t;
+        tsum += t;
+    }
+    tsum = __reduce_add_sync(0xffffffffu, tsum);
+    if (MOE_TN_FILL && !mix && tsum > 0) {
+        const long long cap = (long long)cdiv(ntm * tsum, n_clusters) * n_clusters;   // whole waves
+        int budget = min((int)(cap / ntm) - tsum, 256);
+        __syncwarp();
+        for (; budget > 0; --budget) {
+            // the group with the widest token tiles (ties: the lower id) that can still narrow
+            int bw = 0, bg = -1;
+            for (int g = g0; g < g1; ++g) {
+                const int c = g_cnt[g];
+                if (c <= 0) continue;
+                const int w = tn_width_t(c, g_w[g]);
+                if (w > 16 && w > bw) { bw = w; bg = g; }
+            }
+            const int best = __reduce_max_sync(0xffffffffu, bw);
+            if (best == 0) break;
+            const unsigned cand = __ballot_sync(0xffffffffu, bw == best);
+            if (lane == __ffs(cand) - 1) g_w[bg] += 1;   // lower lanes own lower ids
+            __syncwarp();
+        }
+    }
+    local = 0;
+    for (int g = g0; g < g1; ++g) {
+        const int c = g_cnt[g];
+        const int w = c > 0 ? tn_width_t(c, g_w[g]) : 16;
+        g_w[g] = w;
+        local += c > 0 ? cdiv(c, w) * ntm : 0;
+    }
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -813,7 +862,7 @@ __device__ __forceinline__ void build_group_table_tn(const DevArgs& a, int ntm, 
     int run = incl - local;
     for (int g = g0; g < g1; ++g) {
         tile_start[g] = run;
-        run += tn_tiles(g_cnt[g], ntm);
+        run += g_cnt[g] > 0 ? cdiv(g_cnt[g], g_w[g]) * ntm : 0;
     }
     if (lane == 31) tile_start[n] = incl;
 }
@@ -897,7 +946,8 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     int* tile_start = reinterpret_cast<int*>(smem + P_STAGES * P_STAGE_BYTES + 256);
     int* g_lo = tile_start + (kMaxGemmGroups + 1);
     int* g_cnt = g_lo + kMaxGemmGroups;
-    int* sched_mixed = g_cnt + kMaxGemmGroups;
+    int* g_w = g_cnt + kMaxGemmGroups;
+    int* sched_mixed = g_w + kMaxGemmGroups;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -905,7 +955,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     const bool leader = rank == 0;
     const int ntm = (EPI == EPI_SWIGLU) ? a.N / 128 : a.N / 256;   // weight blocks per expert
 
-    if (warp == 0) build_group_table_tn(a, ntm, lane, tile_start, g_lo, g_cnt, sched_mixed);
+    if (warp == 0) build_group_table_tn(a, ntm, (int)gridDim.x >> 1, lane, tile_start, g_lo, g_cnt, g_w, sched_mixed);
     if (threadIdx.x == 32) {
         for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
@@ -939,7 +989,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             uint32_t ph = 0;
             bool bad = false;
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
-                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt, g_w,
                                             a.n_groups, ntm);
                 const bool first = ti.g < a.n_first;
                 const int gb = first ? ti.g : ti.g - a.n_first;
@@ -1008,7 +1058,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
             const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
             for (int tile = cluster; tile < total && !bad; tile += n_clusters) {
-                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+                const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt, g_w,
                                             a.n_groups, ntm);
                 const uint32_t idesc = FP8 ? idesc_e4m3_f32(P_BM, ti.nt) : idesc_bf16_f32(P_BM, ti.nt);
                 if (*abort_flag || !mbar_wait(&acc_empty[acc], aph ^ 1)) { *abort_flag = 1; break; }
@@ -1051,7 +1101,7 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
         int acc = 0;
         uint32_t aph = 0;
         for (int tile = cluster; tile < total; tile += n_clusters) {
-            const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt,
+            const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt, g_w,
                                             a.n_groups, ntm);
             bool ok = !*abort_flag && mbar_wait(&acc_full[acc], aph);
             if (EPI == EPI_SWIGLU) ok = team_all(ok, team);   // both warps of a team leave together
