@@ -791,10 +791,13 @@ HostPipe* host_pipe()
 
 int host_chunks(const moe_layer_desc* d, int chunks)
 {
-    // Measured on B200 (PCIe ~54 GB/s per direction): two ranges hide about
-    // half of the copies; more ranges cost more than they hide (every range
-    // re-reads the expert weights and pays the fixed routing costs).
-    if (chunks <= 0) chunks = d->T >= 4096 ? 2 : 1;
+    // Ranges of about 2048-4096 tokens.  Measured on B200 (end-to-end ms for
+    // 1 / 2 / 3 / 4 ranges): Mixtral-shaped (T 4096) 3.29 / 2.95 / 3.18 / 3.43;
+    // MoE++ (T 16384) 3.73 / 2.71 / 2.46 / 2.41, with FP8 experts 3.48 / 2.50 /
+    // 2.25 / 2.10; atomic (T 8192) 1.14 / 0.97 / 0.97 / 1.05; long-tail
+    // (T 2048) 0.78 / 0.86 / 1.07 / 1.27.  A range hides the copies of the
+    // next, but re-reads the expert weights and pays the fixed routing costs.
+    if (chunks <= 0) chunks = d->T >= 4096 ? std::max(2, d->T / 4096) : 1;
     return std::max(1, std::min(std::min(chunks, kMaxHostChunks), std::max(d->T, 1)));
 }
 
