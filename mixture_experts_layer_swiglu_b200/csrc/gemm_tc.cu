@@ -1103,6 +1103,27 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
         for (int tile = cluster; tile < total; tile += n_clusters) {
             const TnTile ti = decode_tn(tn_order(tile, total, n_clusters, mixed), tile_start, g_lo, g_cnt, g_w,
                                             a.n_groups, ntm);
+            // e4m3: the scales this tile's epilogue applies, loaded before the wait for
+            // the accumulator so their latency hides behind it (loaded per chunk, the
+            // scale of the token rows stalled every chunk: the short-K e4m3 SwiGLU GEMMs
+            // were bound by their epilogue)
+            float slp[8];                             // token-row scale of column c * 32 + lane
+            float s_lane = 1.f;                       // this lane's weight-row scale
+            if constexpr (FP8) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int cl = c * 32 + lane;
+                    slp[c] = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
+                }
+                const bool first = ti.g < a.n_first;
+                const int gb = first ? ti.g : ti.g - a.n_first;
+                if constexpr (EPI == EPI_F32) {
+                    s_lane = (first ? a.sa0 : a.sa2)[(long long)gb * a.N + ti.m * 256 + (int)rank * 128 + q * 32 + lane];
+                } else {
+                    const float* sa = gate_warp ? (first ? a.sa0 : a.sa2) : (first ? a.sa1 : a.sa3);
+                    s_lane = sa[(long long)gb * a.N + ti.m * 128 + (int)rank * 64 + (q & 1) * 32 + lane];
+                }
+            }
             bool ok = !*abort_flag && mbar_wait(&acc_full[acc], aph);
             if (EPI == EPI_SWIGLU) ok = team_all(ok, team);   // both warps of a team leave together
             if (!ok) { *abort_flag = 1; break; }
@@ -1115,17 +1136,10 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                 float* out = reinterpret_cast<float*>(a.out);
                 float* stg = mine;                        // [32 tokens][32 features]
                 const int f0 = ti.m * 256 + (int)rank * 128 + q * 32;
-                float s_lane = 1.f;                       // e4m3: this lane's weight-row scale
-                if constexpr (FP8) {
-                    const bool first = ti.g < a.n_first;
-                    const int gb = first ? ti.g : ti.g - a.n_first;
-                    s_lane = (first ? a.sa0 : a.sa2)[(long long)gb * a.N + f0 + lane];
-                }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     __syncwarp();                         // the previous chunk has been read
                     if constexpr (FP8) {                  // out = acc * s_weight_row * s_token_row
-                        const int cl = ch * 32 + lane;
-                        const float sl = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
+                        const float sl = slp[ch];
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             stg[i * 32 + lane] = __uint_as_float(v[i]) * s_lane * __shfl_sync(0xffffffffu, sl, i);
@@ -1193,19 +1207,11 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                                 *reinterpret_cast<const uint4*>(stg + row * 32 + piece * 8);
                     }
                 };
-                float s_lane = 1.f;                       // e4m3: this lane's gate or up row scale
-                if constexpr (FP8) {
-                    const bool first = ti.g < a.n_first;
-                    const int gb = first ? ti.g : ti.g - a.n_first;
-                    const float* sa = gate_warp ? (first ? a.sa0 : a.sa2) : (first ? a.sa1 : a.sa3);
-                    s_lane = sa[(long long)gb * a.N + unit0 + lane];
-                }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     team_sync(team);                      // the partner has read the previous chunk
                     float vv[32];                         // (e4m3: acc * s_weight_row * s_token_row)
                     if constexpr (FP8) {
-                        const int cl = ch * 32 + lane;
-                        const float sl = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
+                        const float sl = slp[ch];
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             vv[i] = __uint_as_float(v[i]) * s_lane * __shfl_sync(0xffffffffu, sl, i);
