@@ -1207,14 +1207,28 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                                 *reinterpret_cast<const uint4*>(stg + row * 32 + piece * 8);
                     }
                 };
+                // e4m3: the tile's token-row scales in this warp's staging box (bytes
+                // 3072-4095, untouched by the exchange and the bf16 rows), read back
+                // as broadcast vectors instead of one shuffle per column
+                float* scs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(mine) + 3072);
+                if constexpr (FP8) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) scs[c * 32 + lane] = slp[c];
+                    __syncwarp();
+                }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     team_sync(team);                      // the partner has read the previous chunk
                     float vv[32];                         // (e4m3: acc * s_weight_row * s_token_row)
                     if constexpr (FP8) {
-                        const float sl = slp[ch];
+                        const float4* sc4 = reinterpret_cast<const float4*>(scs + ch * 32);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            vv[i] = __uint_as_float(v[i]) * s_lane * __shfl_sync(0xffffffffu, sl, i);
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 sc = sc4[i4];
+                            vv[4 * i4 + 0] = __uint_as_float(v[4 * i4 + 0]) * s_lane * sc.x;
+                            vv[4 * i4 + 1] = __uint_as_float(v[4 * i4 + 1]) * s_lane * sc.y;
+                            vv[4 * i4 + 2] = __uint_as_float(v[4 * i4 + 2]) * s_lane * sc.z;
+                            vv[4 * i4 + 3] = __uint_as_float(v[4 * i4 + 3]) * s_lane * sc.w;
+                        }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) vv[i] = __uint_as_float(v[i]);
