@@ -20,7 +20,8 @@
 // Two more forms run on clusters of two CTAs (tcgen05.mma.cta_group::2,
 // M = 256): 256-row tiles of a group's rows, and the token-column form
 // (weight rows as M, a group's rows as N in steps of 16), which the pair form
-// uses for the fp32 down projection and for SwiGLU from K = 2048.
+// uses for the fp32 down projection and for SwiGLU from K = 2048; its SwiGLU
+// instance runs eight epilogue warps (10 in all).
 // Every mbarrier wait is bounded (2 s); a timeout sets MOE_ERR_TIMEOUT, all
 // roles leave their loops, in-flight TMA copies are drained and TMEM freed.
 
@@ -720,6 +721,23 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 #define MOE_TN_FILL 1
 #endif
 
+// Token-column kernel layout.  Its tile table holds at most TN_MAX_GROUPS
+// groups.  SwiGLU runs eight epilogue warps (two per TMEM lane quarter, each
+// taking every other 32-column chunk of a tile): with short K (e4m3 MoE++,
+// K = 2048: a ~7 us mainloop per tile) four warps did not finish a tile's
+// SwiGLU before the next accumulator was ready.  Each SwiGLU epilogue warp
+// has a 3.5 KiB box: the exchange with its partner warp (2 KiB), the bf16
+// output rows (1 KiB), and the e4m3 token-row scales of its chunks (512 B);
+// an fp32 epilogue warp a 4 KiB box (one 32 x 32 fp32 chunk).
+constexpr int TN_MAX_GROUPS = 256;
+constexpr int TN_TABLE_INTS = 4 * TN_MAX_GROUPS + 2;
+template <int EPI> constexpr int tn_epi_warps() { return EPI == EPI_SWIGLU ? 8 : 4; }
+template <int EPI> constexpr int tn_threads() { return 64 + 32 * tn_epi_warps<EPI>(); }
+template <int EPI> constexpr int tn_box_bytes() { return EPI == EPI_SWIGLU ? 3584 : 4096; }
+constexpr int tn_epi_offset() { return ((P_STAGES * P_STAGE_BYTES + 256 + TN_TABLE_INTS * 4) + 1023) / 1024 * 1024; }
+template <int EPI> constexpr int tn_smem_bytes() { return 1024 + tn_epi_offset() + tn_epi_warps<EPI>() * tn_box_bytes<EPI>(); }
+static_assert(tn_smem_bytes<EPI_SWIGLU>() <= 232448 && tn_smem_bytes<EPI_F32>() <= 232448, "shared memory per block");
+
 struct TnTile {
     int g;        // group
     int m;        // weight block (256 output features, or 128 hidden units for SwiGLU)
@@ -886,24 +904,26 @@ __device__ __forceinline__ bool team_all(bool v, int id)
     return r != 0;
 }
 
-// Runs body(v, ch) over the 32-column chunks 0..nch-1 of an accumulator,
-// loading chunk ch + 1 from TMEM while chunk ch is processed.
+// Runs body(v, ch) over the 32-column chunks ch0, ch0 + step, ... < nch of an
+// accumulator, loading the next of them from TMEM while one is processed.
 template <typename F>
-__device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body)
+__device__ __forceinline__ void tmem_chunks(uint32_t tacc, int nch, F&& body, int ch0 = 0, int step = 1)
 {
+    if (ch0 >= nch) return;
     uint32_t va[32], vb[32];
-    tmem_ld32(tacc, va);
+    tmem_ld32(tacc + ch0 * 32, va);
     tc_wait_ld_regs(va);
 #pragma unroll 1
-    for (int ch = 0; ch < nch; ch += 2) {
-        const bool more = ch + 1 < nch;
-        if (more) tmem_ld32(tacc + (ch + 1) * 32, vb);
+    for (int ch = ch0; ch < nch; ch += 2 * step) {
+        const int c1 = ch + step, c2 = ch + 2 * step;
+        const bool more = c1 < nch;
+        if (more) tmem_ld32(tacc + c1 * 32, vb);
         body(va, ch);
         if (more) {
             tc_wait_ld_regs(vb);
-            if (ch + 2 < nch) tmem_ld32(tacc + (ch + 2) * 32, va);
-            body(vb, ch + 1);
-            if (ch + 2 < nch) tc_wait_ld_regs(va);
+            if (c2 < nch) tmem_ld32(tacc + c2 * 32, va);
+            body(vb, c1);
+            if (c2 < nch) tc_wait_ld_regs(va);
         }
     }
 }
@@ -919,7 +939,7 @@ enum TnMode { TN_PLAIN = 0, TN_GATHER = 1, TN_SCATTER_ADD = 2, TN_ZERO_ACC = 4 }
 // FP8: both operands e4m3 (kind::f8f6f4); a 128-byte box row holds 128
 // elements of K instead of 64, and the epilogue applies the row scales.
 template <int EPI, int MODE, bool FP8 = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tn_threads<EPI>(), 1)
 grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW0,
                        const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                        const __grid_constant__ CUtensorMap tmW3, const DevArgs a)
@@ -944,10 +964,11 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* tile_start = reinterpret_cast<int*>(smem + P_STAGES * P_STAGE_BYTES + 256);
-    int* g_lo = tile_start + (kMaxGemmGroups + 1);
-    int* g_cnt = g_lo + kMaxGemmGroups;
-    int* g_w = g_cnt + kMaxGemmGroups;
-    int* sched_mixed = g_w + kMaxGemmGroups;
+    int* g_lo = tile_start + (TN_MAX_GROUPS + 1);
+    int* g_cnt = g_lo + TN_MAX_GROUPS;
+    int* g_w = g_cnt + TN_MAX_GROUPS;
+    int* sched_mixed = g_w + TN_MAX_GROUPS;
+    constexpr int EW = tn_epi_warps<EPI>();
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -958,7 +979,8 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     if (warp == 0) build_group_table_tn(a, ntm, (int)gridDim.x >> 1, lane, tile_start, g_lo, g_cnt, g_w, sched_mixed);
     if (threadIdx.x == 32) {
         for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
+        // every epilogue warp of both CTAs releases an accumulator
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 2 * EW); }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -1093,11 +1115,14 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;                   // TMEM lanes 32q .. 32q + 31
-        uint8_t* epi0 = smem + epi_stage_offset(P_STAGES * P_STAGE_BYTES);
-        float* mine = reinterpret_cast<float*>(epi0 + (warp - 2) * EPI_STAGE_BYTES);
-        const float* theirs = reinterpret_cast<const float*>(epi0 + ((warp - 2) ^ 2) * EPI_STAGE_BYTES);
+        const int ew = warp - 2;                  // epilogue warp 0 .. EW - 1
+        const int half = ew >> 2;                 // SwiGLU: this warp's chunks are half, half + 2, ...
+        constexpr int CSTEP = EW / 4;             // chunk step (1 with four epilogue warps)
+        uint8_t* epi0 = smem + tn_epi_offset();
+        float* mine = reinterpret_cast<float*>(epi0 + ew * tn_box_bytes<EPI>());
+        const float* theirs = reinterpret_cast<const float*>(epi0 + (ew ^ 2) * tn_box_bytes<EPI>());
         const bool gate_warp = q < 2;
-        const int team = 1 + (q & 1);             // named barrier id of warps q and q ^ 2
+        const int team = 1 + (q & 1) + 2 * half;  // named barrier id of warps q and q ^ 2 of this half
         int acc = 0;
         uint32_t aph = 0;
         for (int tile = cluster; tile < total; tile += n_clusters) {
@@ -1107,12 +1132,12 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
             // the accumulator so their latency hides behind it (loaded per chunk, the
             // scale of the token rows stalled every chunk: the short-K e4m3 SwiGLU GEMMs
             // were bound by their epilogue)
-            float slp[8];                             // token-row scale of column c * 32 + lane
+            float slp[8];                             // token-row scale of column (half + CSTEP c) * 32 + lane
             float s_lane = 1.f;                       // this lane's weight-row scale
             if constexpr (FP8) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int cl = c * 32 + lane;
+                for (int c = 0; c < 8 / CSTEP; ++c) {
+                    const int cl = (half + CSTEP * c) * 32 + lane;
                     slp[c] = cl < ti.valid ? a.sb[ti.tok0 + cl] : 0.f;
                 }
                 const bool first = ti.g < a.n_first;
@@ -1213,14 +1238,14 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                 float* scs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(mine) + 3072);
                 if constexpr (FP8) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) scs[c * 32 + lane] = slp[c];
+                    for (int c = 0; c < 8 / CSTEP; ++c) scs[c * 32 + lane] = slp[c];
                     __syncwarp();
                 }
                 tmem_chunks(tacc, nch, [&](const uint32_t (&v)[32], int ch) {
                     team_sync(team);                      // the partner has read the previous chunk
                     float vv[32];                         // (e4m3: acc * s_weight_row * s_token_row)
                     if constexpr (FP8) {
-                        const float4* sc4 = reinterpret_cast<const float4*>(scs + ch * 32);
+                        const float4* sc4 = reinterpret_cast<const float4*>(scs + (ch - half) / CSTEP * 32);
 #pragma unroll
                         for (int i4 = 0; i4 < 8; ++i4) {
                             const float4 sc = sc4[i4];
@@ -1249,14 +1274,16 @@ grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
                         for (int i = 0; i < 16; ++i) { g[i] = theirs[i * 32 + lane]; u[i] = vv[16 + i]; }
                         finish(g, u, ch * 32 + 16);
                     }
-                });
+                }, half, CSTEP);
                 if constexpr (ZERO_ACC) {
                     // this tile's share of zeroing its tokens' combine accumulator rows:
                     // 16-byte units [m U / ntm, (m + 1) U / ntm) of each row, so the
                     // ntm weight blocks of a token tile clear its rows between them
                     const int U = a.acc_d / 4;
-                    const int u0 = (int)((long long)ti.m * U / ntm), u1 = (int)((long long)(ti.m + 1) * U / ntm);
-                    const int c = (int)rank * 128 + (warp - 2) * 32 + lane;
+                    const int v0 = (int)((long long)ti.m * U / ntm), v1 = (int)((long long)(ti.m + 1) * U / ntm);
+                    // (with eight warps, each half of them clears half of the units)
+                    const int u0 = v0 + (v1 - v0) * half / CSTEP, u1 = v0 + (v1 - v0) * (half + 1) / CSTEP;
+                    const int c = (int)rank * 128 + (ew & 3) * 32 + lane;
                     if (c < ti.valid) {
                         const int t = a.rows[ti.tok0 + c];
                         if (t >= 0 && t < a.rows_T) {
@@ -1357,6 +1384,7 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
     // (its epilogue writes 16-byte pieces of output rows: row stride and base aligned)
     // (the fused and e4m3 forms exist only in the token-column form, for any K)
     const bool tn = MOE_GEMM_TN && (p.pair || p.tn_any || p.fuse) && p.b_kmod == 0 && p.ldo % 8 == 0 &&
+                    p.n_groups <= TN_MAX_GROUPS &&
                     reinterpret_cast<uintptr_t>(p.out) % 16 == 0 &&
                     ((EPI == EPI_SWIGLU && p.N % 128 == 0 && (p.K >= MOE_TN_SWIGLU_MIN_K || p.fuse || p.fp8)) ||
                      (EPI == EPI_F32 && p.N % 256 == 0));
@@ -1415,9 +1443,9 @@ moe_status launch_epi(const GemmProblem& p, cudaStream_t st)
             const long long tiles_ub = (long long)(cdiv((int)rows, P_BM) + p.n_groups) * ntn;
             const int clusters = (int)std::max<long long>(1, std::min<long long>(tiles_ub, num_sms() / 2));
             auto go = [&](auto kernel) {
-                cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), P_SMEM_BYTES);
+                cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), tn_smem_bytes<EPI>());
                 if (e != cudaSuccess) return cuda_status(e);
-                kernel<<<2 * clusters, NTHREADS, P_SMEM_BYTES, st>>>(mA, m0, m1, m2, m3, a);
+                kernel<<<2 * clusters, tn_threads<EPI>(), tn_smem_bytes<EPI>(), st>>>(mA, m0, m1, m2, m3, a);
                 count_launch();
                 return cuda_status(cudaGetLastError());
             };
