@@ -105,6 +105,23 @@ def test_atomic_cta_pair_router():
     check_atomic_layer(cfg, make_inputs(cfg))
 
 
+def test_more_groups_than_the_token_column_table():
+    """255 routed experts and 2 shared ones, 257 groups (the token-column tile
+    table holds 256): the grouped GEMMs take the row-tiled forms; the router
+    has more than 64 rows."""
+    cfg = scaled(get_config("mixtral"), T=700, d=2048, hidden=256, n_ffn=255, n_shared=2, hidden_shared=256, top_k=4)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["R"] == 700 * 4
+
+
+def test_more_destination_rows_than_the_one_launch_permutation_holds():
+    """top-7 plus 2 shared experts: 9 destination rows per token, more than the
+    one-launch permutation keeps per token, so the four-kernel form runs."""
+    cfg = scaled(get_config("longtail"), T=300, top_k=7)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["R"] == 300 * 7
+
+
 @pytest.mark.parametrize("T", [1, 2, 127, 129])
 def test_bf16_token_counts_across_tile_edges(T):
     cfg = scaled(get_config("mixtral"), T=T, d=256, hidden=384, n_ffn=4)
