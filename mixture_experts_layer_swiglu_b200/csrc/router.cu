@@ -77,9 +77,14 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane)
 }
 
 // (value desc, id asc) order; NaN values never win.
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi)
+// An unsigned key with the order of the float comparison: a > b exactly when
+// key(a) > key(b), -0 and +0 equal, -inf the smallest (key > 0); NaN key 0.
+__device__ __forceinline__ uint32_t logit_key(float v)
 {
-    return v > bv || (v == bv && i < bi);
+    if (v != v) return 0u;
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
 // Block: 8 warps x 4 tokens = a tile of 32 tokens.  The tile's x rows are
@@ -132,20 +137,21 @@ __device__ __forceinline__ void route_token(const RouterArgs& a, int t, float* z
     float zsel = 0.f, z0 = 0.f;
     int isel = -1;
     for (int j = 0; j < a.k; ++j) {
-        float bv = -INFINITY;
+        // the best untaken logit (value desc, ties to the lower id): each lane
+        // its own best as an order-preserving key (NaN never selected, as
+        // with the float comparison), then the largest key of the warp and the
+        // lowest id holding it, two warp reductions instead of a shuffle tree
+        uint32_t bk = 0;
         int bi = INT_MAX;
         for (int i = 0; lane + 32 * i < a.E_r; ++i) {
             if ((taken >> i) & 1u) continue;
             const int e = lane + 32 * i;
-            const float v = z[e];
-            if (better(v, e, bv, bi)) { bv = v; bi = e; }
+            const uint32_t kk = logit_key(z[e]);
+            if (kk > bk) { bk = kk; bi = e; }
         }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(FULL, bv, o);
-            const int oi = __shfl_xor_sync(FULL, bi, o);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
+        const uint32_t mk = __reduce_max_sync(FULL, bk);
+        bi = __reduce_min_sync(FULL, (mk != 0u && bk == mk) ? bi : INT_MAX);
+        const float bv = bi != INT_MAX ? z[bi] : -INFINITY;
         if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (lane == j) { zsel = bv; isel = (bi == INT_MAX) ? -1 : bi; }
         if (j == 0) z0 = bv;
