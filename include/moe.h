@@ -320,9 +320,10 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
 /*
  * The whole layer from host memory to host memory, for a caller whose tokens
  * arrive on the host (a serving loop).  The T tokens are processed in
- * `chunks` consecutive token ranges (0: automatic, max(2, T / 4096) for
- * T >= 4096, else 1; at most 8); the host->device copy of range c + 1 and the
- * device->host copy of range c - 1 run on two internal copy streams while
+ * `chunks` consecutive token ranges (0: automatic, max(2, (T + 2048) / 3584)
+ * for T >= 4096, else 1; at most 8; with three or more, the first and the last
+ * are half as long as the others); the host->device copy of range c + 1 and
+ * the device->host copy of range c - 1 run on two internal copy streams while
  * range c is computed on `stream`, so PCIe transfers overlap the layer.  Every
  * token's result equals moe_layer_forward's bit for bit (tokens are
  * independent).  The pages (OmniMoE's serving scenario) name no such call.

@@ -791,13 +791,14 @@ HostPipe* host_pipe()
 
 int host_chunks(const moe_layer_desc* d, int chunks)
 {
-    // Ranges of about 2048-4096 tokens.  Measured on B200 (end-to-end ms for
-    // 1 / 2 / 3 / 4 ranges): Mixtral-shaped (T 4096) 3.29 / 2.95 / 3.18 / 3.43;
-    // MoE++ (T 16384) 3.73 / 2.71 / 2.46 / 2.41, with FP8 experts 3.48 / 2.50 /
-    // 2.25 / 2.10; atomic (T 8192) 1.14 / 0.97 / 0.97 / 1.05; long-tail
-    // (T 2048) 0.78 / 0.86 / 1.07 / 1.27.  A range hides the copies of the
-    // next, but re-reads the expert weights and pays the fixed routing costs.
-    if (chunks <= 0) chunks = d->T >= 4096 ? std::max(2, d->T / 4096) : 1;
+    // About 3.5k tokens a range (host_range_start gives the lengths).  Measured
+    // on B200, end-to-end ms by range count: Mixtral-shaped (T 4096) 1 / 2 / 3
+    // / 4: 3.29 / 2.97 / 3.05 / 3.28; MoE++ (T 16384) 3 / 4 / 5 / 6: 2.68 /
+    // 2.40 / 2.33 / 2.51, with FP8 experts 2.43 / 2.20 / 2.06 / 2.04; atomic
+    // (T 8192) 1 / 2 / 3: 1.14 / 0.95-1.11 / 0.95-1.10; long-tail (T 2048) 1 /
+    // 2: 0.78 / 0.86.  A range hides the copies of the next, but re-reads the
+    // expert weights and pays the fixed routing costs.
+    if (chunks <= 0) chunks = d->T >= 4096 ? std::max(2, (d->T + 2048) / 3584) : 1;
     return std::max(1, std::min(std::min(chunks, kMaxHostChunks), std::max(d->T, 1)));
 }
 
@@ -806,11 +807,26 @@ struct HostLayout {
     size_t layer_bytes, x_bytes, y_bytes, z_bytes, total;
 };
 
+// First token of range c of nch (c = nch: T).  With three or more ranges the
+// first and the last are half as long as the others: only the first range's
+// host->device copy and the last range's device->host copy are not hidden
+// behind computation.
+int host_range_start(int T, int nch, int c)
+{
+    if (nch < 3 || T < 2 * (nch - 1)) return (int)((long long)T * c / nch);   // (every range non-empty)
+    const long long W = 2ll * (nch - 1);                  // weights 1, 2, ..., 2, 1
+    const long long before = c == 0 ? 0 : (c >= nch ? W : 2ll * c - 1);
+    return (int)((long long)T * before / W);
+}
+
 HostLayout host_layout(const moe_layer_desc* d, int nch)
 {
     HostLayout h;
     h.dc = *d;
-    h.dc.T = cdiv(std::max(d->T, 1), nch);
+    int longest = 1;
+    for (int c = 0; c < nch; ++c)
+        longest = std::max(longest, host_range_start(d->T, nch, c + 1) - host_range_start(d->T, nch, c));
+    h.dc.T = longest;
     h.layer_bytes = al((size_t)moe_layer_workspace_size(&h.dc));
     h.x_bytes = al((size_t)h.dc.T * d->d_model * elt(d));
     h.y_bytes = al((size_t)h.dc.T * d->d_model * (d->out_f32 ? 4 : elt(d)));
@@ -1008,8 +1024,8 @@ moe_status moe_layer_forward_host(const moe_layer_desc* d, const moe_layer_weigh
         if ((call) != cudaSuccess) return MOE_ERR_CUDA;           \
     } while (0)
         for (int c = 0; c < nch; ++c) {
-            const int t0 = c * h.dc.T;
-            const int tc = std::min(h.dc.T, d->T - t0);
+            const int t0 = host_range_start(d->T, nch, c);
+            const int tc = host_range_start(d->T, nch, c + 1) - t0;
             if (tc <= 0) break;
             const int b = c & 1;
             if (c >= 2) MOE_CU(cudaStreamWaitEvent(pp->in, pp->comp_done[c - 2], 0));   // staging b read
