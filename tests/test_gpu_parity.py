@@ -48,6 +48,16 @@ def test_tiny_f32_full_layer():
     assert rep["rel_err"] <= 1e-4
 
 
+def test_f32_layer_long_k_ragged():
+    """fp32 layer whose K exceeds one 256-element staging step of the FMA
+    GEMMs, with ragged tails everywhere: d = 264 (gate/up K in steps of 256
+    and 8; down N = 4 x 64 + 8), H = 300 (down K 256 + 44; gate/up N =
+    4 x 64 + 44), 300 rows over 8 experts (row tiles of 32 with short ends)."""
+    cfg = scaled(get_config("tiny_f32"), T=150, d=264, hidden=300)
+    rep = check_swiglu_layer(cfg, make_inputs(cfg))
+    assert rep["rel_err"] <= 1e-4
+
+
 def test_mixtral_shaped_small_ragged():
     cfg = scaled(get_config("mixtral"), T=333, d=512, hidden=1024)
     rep = check_swiglu_layer(cfg, make_inputs(cfg))
