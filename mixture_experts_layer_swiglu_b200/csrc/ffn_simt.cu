@@ -2,15 +2,16 @@
 //
 // The fp32 layer keeps fp32 end to end (a 1e-4 relative bar that TF32 or
 // bf16 tensor-core inputs cannot meet), so its grouped GEMMs run on the FMA
-// pipes: 32-row x 64-column tiles per expert group, each thread 2 rows x 4
+// pipes: 16-row x 32-column tiles per expert group, each thread 1 row x 2
 // columns (x2 for gate/up).
 //   phase 1: h[r, :] = silu(x_s[r] . W_gate[e]^T) * (x_s[r] . W_up[e]^T)
 //   phase 2: y_s[r, :] = h[r] . W_down[e]^T
-// The layers on this path are small (a few MB of weights), so a tile's time
-// is load latency, not FMAs: each block copies its rows of A and of the
+// The layers on this path are small (a few MB of weights, a few rows per
+// expert), so a tile's time is load latency and the length of each thread's
+// FMA chain, not the FMA rate: each block copies its rows of A and of the
 // weights for up to 256 elements of K at once (16-byte cp.async, all in
-// flight together) and waits once, instead of a round trip per small K
-// chunk.  Tiles are enumerated on the device from the group offsets, as in
+// flight together) and waits once, and tiles are small so that the work
+// spreads over many SMs.  Tiles are enumerated on the device from the group offsets, as in
 // the tensor-core path.
 
 #include <algorithm>
@@ -25,7 +26,7 @@ namespace moe {
 
 namespace {
 
-constexpr int FM = 32, FN = 64;
+constexpr int FM = 16, FN = 32;
 constexpr int FKMAX = 256;              // K elements staged per step
 constexpr int fpitch(int kc) { return kc + 4; }   // floats per staged row (16-byte aligned rows)
 
@@ -73,12 +74,10 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(const float* __restrict__ 
     const float* Wa = (first ? B0 : B2) + gb * (long long)N * K;
     const float* Wb = SWIGLU ? (first ? B1 : B3) + gb * (long long)N * K : nullptr;
 
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16
-    float acc[2][4], acc2[2][4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 columns (x2) x 16 rows
+    float acc[2], acc2[2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) { acc[i][j] = 0.f; acc2[i][j] = 0.f; }
+    for (int j = 0; j < 2; ++j) { acc[j] = 0.f; acc2[j] = 0.f; }
 
     const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int k0 = 0; k0 < K; k0 += KC) {
@@ -106,39 +105,32 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(const float* __restrict__ 
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
-#pragma unroll 2
+#pragma unroll 4
         for (int k = 0; k < kc; k += 4) {
             const float4 a0 = *reinterpret_cast<const float4*>(As + ty * pitch + k);
-            const float4 a1 = *reinterpret_cast<const float4*>(As + (ty + 16) * pitch + k);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 const float4 b = *reinterpret_cast<const float4*>(Bs + (tx + 16 * j) * pitch + k);
-                acc[0][j] = fmaf(a0.x, b.x, acc[0][j]); acc[0][j] = fmaf(a0.y, b.y, acc[0][j]);
-                acc[0][j] = fmaf(a0.z, b.z, acc[0][j]); acc[0][j] = fmaf(a0.w, b.w, acc[0][j]);
-                acc[1][j] = fmaf(a1.x, b.x, acc[1][j]); acc[1][j] = fmaf(a1.y, b.y, acc[1][j]);
-                acc[1][j] = fmaf(a1.z, b.z, acc[1][j]); acc[1][j] = fmaf(a1.w, b.w, acc[1][j]);
+                acc[j] = fmaf(a0.x, b.x, acc[j]); acc[j] = fmaf(a0.y, b.y, acc[j]);
+                acc[j] = fmaf(a0.z, b.z, acc[j]); acc[j] = fmaf(a0.w, b.w, acc[j]);
                 if (SWIGLU) {
                     const float4 c = *reinterpret_cast<const float4*>(Cs + (tx + 16 * j) * pitch + k);
-                    acc2[0][j] = fmaf(a0.x, c.x, acc2[0][j]); acc2[0][j] = fmaf(a0.y, c.y, acc2[0][j]);
-                    acc2[0][j] = fmaf(a0.z, c.z, acc2[0][j]); acc2[0][j] = fmaf(a0.w, c.w, acc2[0][j]);
-                    acc2[1][j] = fmaf(a1.x, c.x, acc2[1][j]); acc2[1][j] = fmaf(a1.y, c.y, acc2[1][j]);
-                    acc2[1][j] = fmaf(a1.z, c.z, acc2[1][j]); acc2[1][j] = fmaf(a1.w, c.w, acc2[1][j]);
+                    acc2[j] = fmaf(a0.x, c.x, acc2[j]); acc2[j] = fmaf(a0.y, c.y, acc2[j]);
+                    acc2[j] = fmaf(a0.z, c.z, acc2[j]); acc2[j] = fmaf(a0.w, c.w, acc2[j]);
                 }
             }
         }
         __syncthreads();
     }
+    const int r = ty;
+    const long long grow = (long long)row0 + r;
+    if (r < rows && grow < rows_cap) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int r = ty + 16 * i;
-        const long long grow = (long long)row0 + r;
-        if (r >= rows || grow >= rows_cap) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
             const int c = col0 + tx + 16 * j;
             if (c >= N) continue;
-            float v = acc[i][j];
-            if (SWIGLU) v = v / (1.0f + expf(-v)) * acc2[i][j];
+            float v = acc[j];
+            if (SWIGLU) v = v / (1.0f + expf(-v)) * acc2[j];
             out[grow * N + c] = v;
         }
     }
