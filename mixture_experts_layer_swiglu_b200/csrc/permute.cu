@@ -590,9 +590,10 @@ moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
 {
     if (a.n_ffn > P_MAXE) return MOE_ERR_UNSUPPORTED;
     const int nb = permute_blocks(a.T);
-    // (every block reads all the counts: the one-launch form is for up to PF_MAXCOUNTS of them)
+    // (every block reads all the counts: the one-launch form is for up to PF_MAXCOUNTS of them;
+    // small batches take one block per 8 tokens, so the grid barrier waits on few blocks)
     const int grid = a.bar && a.T > 0 && a.k + a.n_shared <= PF_MAXDST && (long long)nb * a.n_ffn <= PF_MAXCOUNTS
-                         ? pf_grid() : 0;
+                         ? std::min(pf_grid(), std::max(1, cdiv(a.T, 8))) : 0;
     if (grid > 0) {   // one cooperative launch (its barrier counter cleared first)
         cudaError_t e = cudaMemsetAsync(a.bar, 0, sizeof(unsigned), st);
         if (e != cudaSuccess) return cuda_status(e);
