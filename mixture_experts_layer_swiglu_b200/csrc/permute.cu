@@ -18,8 +18,9 @@
 //
 // Atomic kind (N up to millions of experts, ~2 tasks each), two launches:
 //   a kernel zeroes the counts and a barrier counter; one cooperative kernel
-//   (every block resident) then runs histogram (integer atomics) -> per-block
-//   totals -> exclusive scan -> placement through per-expert cursors ->
+//   (every block resident) then runs histogram (integer atomics, each slot
+//   keeping the count its atomic returned as its rank) -> per-block totals ->
+//   exclusive scan -> placement at the expert's offset plus the rank ->
 //   per-expert sort of each short segment by slot id (= token order), which
 //   fixes the order whatever order the atomics took; the phases are separated
 //   by a grid barrier whose waits are bounded (2 s, then MOE_ERR_TIMEOUT).
@@ -468,11 +469,27 @@ __global__ void __launch_bounds__(AP_THREADS) atomic_permute_kernel(const Permut
     const int N = a.n_ids;
     const long long gstride = (long long)gridDim.x * blockDim.x;
     const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-    // 1. histogram
-    for (long long s = gtid; s < n; s += gstride) {
-        const int e = a.idx[s];
-        if (e < 0 || e >= N) { set_status(MOE_ERR_DEVICE_BOUNDS); continue; }
-        atomicAdd(&a.ws_counts[e], 1);
+    // 1. histogram; each slot keeps the count its atomic returned (its rank
+    //    among its expert's tasks, in whatever order the atomics took) in
+    //    row_of until the placement, four slots per thread and step
+    for (long long s0 = gtid; s0 < n; s0 += 4 * gstride) {
+        int e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long sl = s0 + u * gstride;
+            e[u] = sl < n ? a.idx[sl] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long sl = s0 + u * gstride;
+            if (sl >= n) continue;
+            if (e[u] < 0 || e[u] >= N) {
+                set_status(MOE_ERR_DEVICE_BOUNDS);
+                a.row_of[sl] = -1;
+            } else {
+                a.row_of[sl] = atomicAdd(&a.ws_counts[e[u]], 1);
+            }
+        }
     }
     if (!ap_grid_sync(bar, 1, &s_ok)) return;
     // 2. this block's chunk of experts and its total
@@ -510,12 +527,21 @@ __global__ void __launch_bounds__(AP_THREADS) atomic_permute_kernel(const Permut
     }
     if (hi == N && lo < hi && threadIdx.x == 0) a.offsets[N] = run;
     if (!ap_grid_sync(bar, 3, &s_ok)) return;
-    // 4. placement through per-expert cursors (any order; sorted next)
-    for (long long s = gtid; s < n; s += gstride) {
-        const int e = a.idx[s];
-        if (e < 0 || e >= N) { a.row_of[s] = -1; continue; }
-        const int pos = a.offsets[e] + atomicSub(&a.ws_counts[e], 1) - 1;
-        a.token_of[pos] = (int)s;
+    // 4. placement at the expert's offset plus the slot's rank from the
+    //    histogram (any order inside a segment; sorted next): no atomics
+    for (long long s0 = gtid; s0 < n; s0 += 4 * gstride) {
+        int e[4], r[4], o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long sl = s0 + u * gstride;
+            e[u] = sl < n ? a.idx[sl] : -1;
+            r[u] = sl < n ? a.row_of[sl] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[u] = (e[u] >= 0 && e[u] < N && r[u] >= 0) ? a.offsets[e[u]] : -1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (o[u] >= 0) a.token_of[o[u] + r[u]] = (int)(s0 + u * gstride);
     }
     if (!ap_grid_sync(bar, 4, &s_ok)) return;
     // 5. each expert's segment sorted by slot id, and row_of.  A segment of
@@ -525,8 +551,11 @@ __global__ void __launch_bounds__(AP_THREADS) atomic_permute_kernel(const Permut
     // written back: one memory round trip instead of the dependent global
     // reads and writes of an in-place insertion sort, whose longest segments
     // bounded the whole phase.  Longer segments are sorted in place.
+    // (the next expert's offsets are loaded while this one is sorted)
+    int nx0 = gtid < N ? a.offsets[gtid] : 0, nx1 = gtid < N ? a.offsets[gtid + 1] : 0;
     for (long long e = gtid; e < N; e += gstride) {
-        const int s0 = a.offsets[e], s1 = a.offsets[e + 1];
+        const int s0 = nx0, s1 = nx1;
+        if (e + gstride < N) { nx0 = a.offsets[e + gstride]; nx1 = a.offsets[e + gstride + 1]; }
         if (s1 - s0 <= AP_SORT) {
             int v[AP_SORT];
 #pragma unroll
