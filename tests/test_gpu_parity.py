@@ -203,6 +203,8 @@ def test_cuda_graph_replay_matches_eager(name, T, changes):
     ("atomic", 1000, {}, 4),
     ("mixtral", 600, {"d": 512, "hidden": 512}, 0),
     ("tiny_f32", 64, {}, 2),
+    ("longtail", 300, {}, 3),                    # shared experts: their groups hold every token of a range
+    ("mixtral_fp8", 600, {"d": 512, "hidden": 512}, 2),   # e4m3 experts
 ])
 def test_host_call_equals_device_call(name, T, changes, chunks):
     """moe_layer_forward_host (host buffers, copies pipelined over token
