@@ -33,6 +33,7 @@
 #include <climits>
 
 #include "common.cuh"
+#include "e4m3.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -301,6 +302,9 @@ __device__ __forceinline__ int pf_block_scan(int v, int* warp_tot, int* total)
     return before + incl - v;
 }
 
+// QUANT: the destination rows get the e4m3 codes of the token's row (and its
+// scale); a separate instance, so the bf16 copy keeps its registers.
+template <bool QUANT>
 __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const PermuteArgs a, unsigned* bar, int nb)
 {
     __shared__ uint32_t mask[P_MAXE][8];
@@ -412,7 +416,44 @@ __global__ void __launch_bounds__(PF_THREADS, 2) perm_fused_kernel(const Permute
             for (int w = 0; w < 8; ++w) n += __popc(mask[e][w]);
             sbase[e] += n;
         }
-        if (xs) {
+        if (QUANT && xs) {
+            // e4m3 rows (d a multiple of 256): one warp per token reads x[t]
+            // for its max, then again (from L1 / L2) to write the same codes
+            // into every destination row, and the row scale beside each
+            uint8_t* xq = static_cast<uint8_t*>(a.x_sorted);
+            const int nv = a.d / 256;                      // 8-element vectors per lane
+            for (int tt = t0 + warp; tt < t1; tt += NW) {
+                const int ti = tt - c * P_TOK;
+                const uint4* src = x + (long long)tt * vecs;
+                float amax = 0.f;
+                for (int i = 0; i < nv; ++i) {
+                    float v[8];
+                    bf16x8(__ldg(src + i * 32 + lane), v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                const float sc = pow2_scale(amax), inv = 1.f / sc;   // inverse of a power of two: exact
+                for (int i = 0; i < nv; ++i) {
+                    float v[8];
+                    bf16x8(__ldg(src + i * 32 + lane), v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] *= inv;
+                    const uint2 q = to_e4m3x8(v);
+                    for (int j = 0; j < ndst && j < PF_MAXDST; ++j) {
+                        const int r = s_dst[ti][j];
+                        if (r < 0 || r >= rows_cap) continue;
+                        reinterpret_cast<uint2*>(xq + (long long)r * a.d)[i * 32 + lane] = q;
+                    }
+                }
+                if (lane < ndst && lane < PF_MAXDST) {
+                    const int r = s_dst[ti][lane];
+                    if (r >= rows_cap) set_status(MOE_ERR_DEVICE_BOUNDS);
+                    else if (r >= 0) a.xs_scale[r] = sc;
+                }
+            }
+        } else if (!QUANT && xs) {
             // one warp per token: each 16-byte vector of x[t] is read once and
             // stored to every destination row
             for (int tt = t0 + warp; tt < t1; tt += NW) {
@@ -608,8 +649,11 @@ static int pf_grid()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (per_sm[dev] == 0) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, perm_fused_kernel, PF_THREADS, 0) != cudaSuccess) n = 0;
+        int n = 0, m = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, perm_fused_kernel<false>, PF_THREADS, 0) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, perm_fused_kernel<true>, PF_THREADS, 0) != cudaSuccess)
+            n = 0;
+        n = std::min(n, m);
         per_sm[dev] = n > 0 ? n : -1;
     }
     return per_sm[dev] > 0 ? std::min(per_sm[dev], 2) * num_sms() : 0;
@@ -627,15 +671,21 @@ moe_status launch_permute_swiglu(const PermuteArgs& a, cudaStream_t st)
         cudaError_t e = cudaMemsetAsync(a.bar, 0, sizeof(unsigned), st);
         if (e != cudaSuccess) return cuda_status(e);
         PermuteArgs args = a;
-        if (a.xs_scale) args.x_sorted = nullptr;   // e4m3 rows: the quantizing gather below writes them
+        // e4m3 rows: with four or more destination rows per token (shared
+        // experts, large k) this kernel quantizes each token's row once and
+        // writes its codes to all of them; with fewer, the quantizing gather
+        // below (one warp per permuted row) measured faster
+        const bool quant_here = a.xs_scale && a.d % 256 == 0 && a.k + a.n_shared >= 4;
+        if (a.xs_scale && !quant_here) args.x_sorted = nullptr;
         unsigned* bar = a.bar;
         int nbv = nb;
         void* params[3] = {&args, &bar, &nbv};
-        e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(perm_fused_kernel), dim3(grid), dim3(PF_THREADS),
-                                        params, 0, st);
+        e = cudaLaunchCooperativeKernel(quant_here ? reinterpret_cast<const void*>(perm_fused_kernel<true>)
+                                                   : reinterpret_cast<const void*>(perm_fused_kernel<false>),
+                                        dim3(grid), dim3(PF_THREADS), params, 0, st);
         if (e != cudaSuccess) return cuda_status(e);
         count_launch();
-        if (a.x_sorted && a.xs_scale) {
+        if (a.x_sorted && a.xs_scale && !quant_here) {
             const long long rows_cap = (long long)a.T * a.k + (long long)a.n_shared * a.T;
             moe_status s = launch_gather_quant(a.token_of, a.offsets, a.n_ffn + a.n_shared, a.x, a.d, a.T, a.x_sorted,
                                                a.xs_scale, rows_cap, st);

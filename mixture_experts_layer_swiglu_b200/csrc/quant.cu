@@ -8,8 +8,11 @@
 // saturating).  Dividing by a power of two is exact, so the rounding is the
 // only approximation, and s is kept beside the row for the GEMM's epilogue.
 //   gather_quant_kernel: x_sorted codes[r] = e4m3(x[token_of[r]] / s_r), one
-//     warp per row (the permutation's gather and the quantization in one pass);
+//     warp per row (the permutation's gather and the quantization in one pass;
+//     layers with four or more destination rows per token quantize each
+//     token's row once inside the one-launch permutation instead);
 //   quant_rows_kernel: h8[r] = e4m3(h[r] / s_r), one block per row.
+// The row scale and the code conversion are in e4m3.cuh.
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -17,6 +20,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "e4m3.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -24,35 +28,6 @@ namespace moe {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-
-// The smallest power of two s with 448 s >= amax (1 for amax == 0).  448 * 2^e
-// is exact in fp32, so the comparisons decide exactly.
-__device__ __forceinline__ float pow2_scale(float amax)
-{
-    if (!(amax > 0.f)) return 1.f;
-    int ex;
-    frexpf(amax, &ex);                  // amax in [2^(ex-1), 2^ex)
-    int e = max(ex - 9, -126);
-    while (448.f * ldexpf(1.f, e) < amax) ++e;
-    while (e > -126 && 448.f * ldexpf(1.f, e - 1) >= amax) --e;
-    return ldexpf(1.f, e);
-}
-
-// Eight values -> eight e4m3 codes (nearest, ties to even, saturating).
-__device__ __forceinline__ uint2 to_e4m3x8(const float (&v)[8])
-{
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        w[i] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * i], v[2 * i + 1]), __NV_SATFINITE, __NV_E4M3);
-    return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-}
-
-__device__ __forceinline__ void bf16x8(const uint4 u, float (&v)[8])
-{
-    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-}
 
 // Rows r < offsets[n_last] (capped at rows_cap): codes[r] = e4m3(x[t] / s),
 // scale[r] = s, t = token_of[r].  d a multiple of 256 (32 lanes x 8).
