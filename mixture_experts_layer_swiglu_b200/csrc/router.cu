@@ -133,28 +133,53 @@ __device__ __forceinline__ void route_token(const RouterArgs& a, int t, float* z
         }
     }
     __syncwarp();
-    uint32_t taken = 0;   // bit i: expert lane + 32 i already selected
     float zsel = 0.f, z0 = 0.f;
     int isel = -1;
-    for (int j = 0; j < a.k; ++j) {
-        // the best untaken logit (value desc, ties to the lower id): each lane
-        // its own best as an order-preserving key (NaN never selected, as
-        // with the float comparison), then the largest key of the warp and the
-        // lowest id holding it, two warp reductions instead of a shuffle tree
-        uint32_t bk = 0;
-        int bi = INT_MAX;
-        for (int i = 0; lane + 32 * i < a.E_r; ++i) {
-            if ((taken >> i) & 1u) continue;
-            const int e = lane + 32 * i;
-            const uint32_t kk = logit_key(z[e]);
-            if (kk > bk) { bk = kk; bi = e; }
+    if (a.E_r <= 32 && a.k <= 2) {
+        // one logit per lane: the best two of the warp in one butterfly that
+        // carries each lane's best pair of keys (order-preserving value, then
+        // the complemented id, so equal values go to the lower id; a NaN has
+        // key 0 and is never chosen) -- the same choice as the loop below
+        unsigned long long k1 = 0ull, k2 = 0ull;
+        if (lane < a.E_r) {
+            const uint32_t kv = logit_key(z[lane]);
+            if (kv) k1 = ((unsigned long long)kv << 32) | (uint32_t)~(uint32_t)lane;
         }
-        const uint32_t mk = __reduce_max_sync(FULL, bk);
-        bi = __reduce_min_sync(FULL, (mk != 0u && bk == mk) ? bi : INT_MAX);
-        const float bv = bi != INT_MAX ? z[bi] : -INFINITY;
-        if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == j) { zsel = bv; isel = (bi == INT_MAX) ? -1 : bi; }
-        if (j == 0) z0 = bv;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const unsigned long long b1 = __shfl_xor_sync(FULL, k1, o), b2 = __shfl_xor_sync(FULL, k2, o);
+            const unsigned long long lo = k1 > b1 ? b1 : k1, m2 = k2 > b2 ? k2 : b2;
+            k1 = k1 > b1 ? k1 : b1;
+            k2 = lo > m2 ? lo : m2;
+        }
+        const unsigned long long mine = lane == 0 ? k1 : k2;
+        if (lane < a.k) {
+            isel = mine != 0ull ? (int)~(uint32_t)mine : -1;
+            zsel = isel >= 0 ? z[isel] : -INFINITY;
+        }
+        z0 = k1 != 0ull ? z[(int)~(uint32_t)k1] : -INFINITY;
+    } else {
+        uint32_t taken = 0;   // bit i: expert lane + 32 i already selected
+        for (int j = 0; j < a.k; ++j) {
+            // the best untaken logit (value desc, ties to the lower id): each lane
+            // its own best as an order-preserving key (NaN never selected, as
+            // with the float comparison), then the largest key of the warp and the
+            // lowest id holding it, two warp reductions instead of a shuffle tree
+            uint32_t bk = 0;
+            int bi = INT_MAX;
+            for (int i = 0; lane + 32 * i < a.E_r; ++i) {
+                if ((taken >> i) & 1u) continue;
+                const int e = lane + 32 * i;
+                const uint32_t kk = logit_key(z[e]);
+                if (kk > bk) { bk = kk; bi = e; }
+            }
+            const uint32_t mk = __reduce_max_sync(FULL, bk);
+            bi = __reduce_min_sync(FULL, (mk != 0u && bk == mk) ? bi : INT_MAX);
+            const float bv = bi != INT_MAX ? z[bi] : -INFINITY;
+            if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == j) { zsel = bv; isel = (bi == INT_MAX) ? -1 : bi; }
+            if (j == 0) z0 = bv;
+        }
     }
     const float ex = (lane < a.k) ? expf(zsel - z0) : 0.f;
     float sum = ex;
